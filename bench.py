@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Benchmark of the Ulysses SP hot path on B200 (one JSON line on rank 0).
+
+One step = the whole path on one batch of seeded synthetic input already in
+HBM:  seq_to_head(q, k, v) -> attention forward -> head_to_seq(O);
+seq_to_head(dO) -> attention backward -> head_to_seq(dQ, dK, dV).
+Outputs are stored fp32 (the precision the parity tests gate).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+`value` is the algorithmic fwd+bwd attention FLOP rate of the whole step
+(12 * d * H_q * pairs per step, pairs = sum over samples of L(L+1)/2, i.e.
+only key/query pairs the causal, sample-segmented mask allows), over all
+ranks.  Under torchrun each GPU runs its own copy of the workload (weak
+scaling, no data-path collective); time is the max over ranks.
+`--impl reference` times the CPU fp64 oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "causal attn TFLOP/s fwd & fwd+bwd (% bf16 peak); re-layout GB/s (% HBM)"
+DEFAULT_WORKLOAD = "llama8b_p4_n32k"
+
+
+def pairs_of(lengths):
+    return sum(L * (L + 1) // 2 for row in lengths for L in row)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.sw_power_cap,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, reasons = [], None, set()
+        names = ("sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+def oracle_sample(w, x, rows: int, heads: int):
+    """fwd + bwd of the CPU oracle on the last `rows` query rows of `heads`
+    query heads (their full visible key ranges).  Returns (flops, seconds)."""
+    import oracle
+    q = synthetic.bf16_bits_to_f64(x["q"][0])
+    k = synthetic.bf16_bits_to_f64(x["k"][0])
+    v = synthetic.bf16_bits_to_f64(x["v"][0])
+    do = synthetic.bf16_bits_to_f64(x["do"][0]) if "do" in x else None
+    ss = oracle.segment_starts(x["position_ids"])[0]
+    rows = min(rows, w.n)
+    lo = w.n - rows
+    visible = int(sum(i - ss[i] + 1 for i in range(lo, w.n)))
+    scale = oracle.default_scale(w.d)
+    t0 = time.perf_counter()
+    for h in range(heads):
+        g = h // w.group
+        oracle.attention_fwd_head(q[:, h], k[:, g], v[:, g], ss, scale, row_lo=lo)
+        if do is not None:
+            oracle.attention_bwd_head(q[:, h], k[:, g], v[:, g], do[:, h], ss, scale, row_lo=lo)
+    dt = time.perf_counter() - t0
+    per = (12 if do is not None else 4) * w.d
+    return per * visible * heads, dt
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = synthetic.make_inputs(w)
+    rows, heads = 512, 2
+    for _ in range(args.warmup):
+        oracle_sample(w, x, rows, heads)
+    flops, secs = 0, 0.0
+    for _ in range(args.steps):
+        f, s = oracle_sample(w, x, rows, heads)
+        flops += f
+        secs += s
+    value = flops / secs / 1e12
+    cores = len(os.sched_getaffinity(0))
+    sample = f"oracle fwd+bwd of the last {rows} query rows of {heads} query heads per step"
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "P": w.P, "b": w.b, "n": w.n, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d},
+           "impl": "reference",
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    import ulysses_head_attention_b200 as uly
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+
+    P, b, n, hq, hkv, d = w.P, w.b, w.n, w.h_q, w.h_kv, w.d
+    m = n // P
+    x = synthetic.make_inputs(w)
+    pairs = pairs_of(x["lengths"])
+    fwd_flops = 4 * d * hq * pairs
+    bwd_flops = 8 * d * hq * pairs
+
+    def pinned(bits):
+        t = torch.from_numpy(bits.reshape(P, b, m, bits.shape[2], d).view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory()
+
+    host = {k: pinned(x[k]) for k in ("q", "k", "v", "do")}
+    host_pos = torch.from_numpy(x["position_ids"]).pin_memory()
+    seq = {k: host[k].to(dev) for k in host}
+    pos = host_pos.to(dev)
+    bf, f32 = torch.bfloat16, torch.float32
+    head = {"q": torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev),
+            "k": torch.empty((P, b, n, hkv // P, d), dtype=bf, device=dev),
+            "v": torch.empty((P, b, n, hkv // P, d), dtype=bf, device=dev),
+            "do": torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev)}
+    o_head = torch.empty((P, b, n, hq // P, d), dtype=f32, device=dev)
+    lse = torch.empty((P, b, hq // P, n), dtype=f32, device=dev)
+    o_seq = torch.empty((P, b, m, hq, d), dtype=f32, device=dev)
+    g_head = {"q": torch.empty_like(o_head), "k": torch.empty((P, b, n, hkv // P, d), dtype=f32, device=dev),
+              "v": torch.empty((P, b, n, hkv // P, d), dtype=f32, device=dev)}
+    g_seq = {"q": torch.empty((P, b, m, hq, d), dtype=f32, device=dev),
+             "k": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev),
+             "v": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev)}
+    shape = uly.make_shape(b, n, hq, hkv, d, P)
+    ws_f = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(shape), dev)
+    ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, uly.ULY_F32), dev)
+    stream = torch.cuda.current_stream()
+    launches_per_step = 3 + 2 + 1 + 1 + 3 + 3     # s2h x3, fwd (2), h2s O, s2h dO, bwd (3), h2s x3
+
+    relayout_bytes = 2 * sum(t.numel() * t.element_size() for t in (seq["q"], seq["k"], seq["v"], seq["do"]))
+    relayout_bytes += 2 * sum(t.numel() * t.element_size() for t in (o_seq, g_seq["q"], g_seq["k"], g_seq["v"]))
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        for k in ("q", "k", "v"):
+            uly.ulysses_seq_to_head(seq[k], head[k])
+        if ev is not None:
+            ev[1].record(stream)
+        uly.ulysses_attn_fwd(head["q"], head["k"], head["v"], pos, o_head, lse, ws_f)
+        if ev is not None:
+            ev[2].record(stream)
+        uly.ulysses_head_to_seq(o_head, o_seq)
+        uly.ulysses_seq_to_head(seq["do"], head["do"])
+        if ev is not None:
+            ev[3].record(stream)
+        uly.ulysses_attn_bwd(head["q"], head["k"], head["v"], o_head, lse, head["do"], pos,
+                             g_head["q"], g_head["k"], g_head["v"], ws_b)
+        if ev is not None:
+            ev[4].record(stream)
+        for k in ("q", "k", "v"):
+            uly.ulysses_head_to_seq(g_head[k], g_seq[k])
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    for ws in (ws_f, ws_b):
+        if uly.ulysses_workspace_status(ws) != 0:
+            raise RuntimeError("a kernel reported a pipeline timeout during warm-up")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(val):
+        if world == 1:
+            return val
+        t = torch.tensor([val], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-timed region: K steps, inputs resident in HBM
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(start.elapsed_time(end))
+    ms_step = ms_total / args.steps
+    stage = {"s2h_qkv": [], "attn_fwd": [], "h2s_o_s2h_do": [], "attn_bwd": [], "h2s_grads": []}
+    for e in evs:
+        for k, (a, bnd) in zip(stage, ((0, 1), (1, 2), (2, 3), (3, 4), (4, 5))):
+            stage[k].append(e[a].elapsed_time(e[bnd]))
+    st_ms = {k: statistics.mean(v) for k, v in stage.items()}
+    for ws in (ws_f, ws_b):
+        if uly.ulysses_workspace_status(ws) != 0:
+            raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
+
+    value = world * (fwd_flops + bwd_flops) / (ms_step * 1e-3) / 1e12
+    fwd_tf = fwd_flops / (st_ms["attn_fwd"] * 1e-3) / 1e12
+    bwd_tf = bwd_flops / (st_ms["attn_bwd"] * 1e-3) / 1e12
+    relayout_ms = st_ms["s2h_qkv"] + st_ms["h2s_o_s2h_do"] + st_ms["h2s_grads"]
+    relayout_gbs = relayout_bytes / (relayout_ms * 1e-3) / 1e9
+    peak_t = peaks["bf16_tflops_sustained"]
+
+    # ---- end to end: pinned host inputs in, all outputs back to pinned host
+    h_out = {"o": torch.empty(o_seq.shape, dtype=f32, pin_memory=True)}
+    for k in g_seq:
+        h_out[k] = torch.empty(g_seq[k].shape, dtype=f32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_pos.numel() * 8
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+    def e2e_step():
+        for k in host:
+            seq[k].copy_(host[k], non_blocking=True)
+        pos.copy_(host_pos, non_blocking=True)
+        step()
+        h_out["o"].copy_(o_seq, non_blocking=True)
+        for k in g_seq:
+            h_out[k].copy_(g_seq[k], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2)) / args.steps
+    e2e_value = world * (fwd_flops + bwd_flops) / (e2e_ms * 1e-3) / 1e12
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "P": P, "b": b, "n": n, "h_q": hq, "h_kv": hkv, "d": d,
+                   "samples": sum(len(r) for r in x["lengths"]), "pairs": pairs,
+                   "outputs": "fp32", "l2": "inputs larger than L2 (q 256 MiB, dO 256 MiB per step)",
+                   "parallelism": f"{world} independent replica(s), one per GPU"},
+        "detail": {
+            "attn_fwd_tflops": fwd_tf, "attn_fwd_frac": fwd_tf / peak_t,
+            "attn_bwd_tflops": bwd_tf, "attn_bwd_frac": bwd_tf / peak_t,
+            "attn_fwd_bwd_tflops": (fwd_flops + bwd_flops) / ((st_ms["attn_fwd"] + st_ms["attn_bwd"]) * 1e-3) / 1e12,
+            "relayout_gbs": relayout_gbs, "relayout_frac": relayout_gbs / peaks["hbm_gbs"],
+            "stage_ms": st_ms, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
+            "bwd_flops_with_recompute_convention": 10 * d * hq * pairs,
+            "peaks": peaks,
+        },
+        "roofline": {"bound": "tensor", "kernel": "attn_bwd (ulysses_attn_bwd call: segments + pre + main)",
+                     "achieved": bwd_tf, "peak": peak_t, "unit": "TFLOP/s", "frac": bwd_tf / peak_t,
+                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "traffic": None},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops, secs = 0, 0.0
+        rows, heads = 512, 2
+        for _ in range(4):
+            f, s = oracle_sample(w, x, rows, heads)
+            flops += f
+            secs += s
+        out["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+                               "kind": "oracle",
+                               "sample": f"4 x oracle fwd+bwd of the last {rows} query rows of {heads} heads"}
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synthetic.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,161 @@
+/*
+ * ulysses.h -- C ABI of the single-GPU Ulysses sequence-parallel hot path.
+ *
+ * Ulysses sequence parallelism (the SP part of Arctic Long Sequence Training)
+ * shards a sequence over P ranks, uses an all-to-all to trade the sequence
+ * sharding for a head sharding, runs ordinary attention per head over the
+ * whole sequence, and uses a second all-to-all to return to the sequence
+ * sharding (blog "Ulysses Sequence Parallelism: Training with Million-Token
+ * Contexts", "How Ulysses works", steps 1-6; Transformers docs "Ulysses
+ * sequence parallelism", the figure at the top of the page).  This library
+ * runs that path for P *virtual* ranks that all live in one GPU's memory: the
+ * two all-to-alls become the re-layouts below, and the local attention is the
+ * forward/backward kernels below.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Sizes are full (unsharded) sizes: b = batch rows, n = tokens per row,
+ *    h_q / h_kv = query / key-value heads, d = head dimension, P = ranks.
+ *  - Layouts (row-major, innermost last, elements contiguous):
+ *      seq-sharded   X_seq [P][b][n/P][H][d]   rank r holds tokens
+ *                    [r*n/P, (r+1)*n/P) with all H heads ("How Ulysses
+ *                    works", step 1).  For b == 1 this is byte-identical to
+ *                    an unsharded [n][H][d] tensor.
+ *      head-sharded  X_head[P][b][n][H/P][d]   rank r holds all n tokens of
+ *                    heads [r*H/P, (r+1)*H/P) ("How Ulysses works", step 3).
+ *      LSE           [P][b][h_q/P][n] float32, natural log.
+ *      position_ids  [b][n] int64 on the device; a sample starts at t == 0
+ *                    and wherever position_ids[t] == 0.
+ *  - GQA: query head h reads kv head h / (h_q/h_kv); ranks split both head
+ *    counts contiguously, so each rank's query heads read its own kv heads.
+ *  - Pointers are device pointers owned by the caller, 16-byte aligned.
+ *    `stream` is a cudaStream_t (NULL = legacy default stream), passed as
+ *    void* so this header needs no CUDA header.
+ *  - Calls only enqueue work on `stream` and return; results are valid once
+ *    the stream has run.  Outputs are fully overwritten.  The library
+ *    allocates no device memory and keeps no mutable global state; scratch
+ *    space is the caller's workspace, sized by the *_workspace queries.
+ *  - Errors: every argument is checked on the host before anything is
+ *    launched; a bad argument returns ULY_ERR_INVALID_ARG (or
+ *    ULY_ERR_UNSUPPORTED for a valid but unimplemented size/type) and
+ *    enqueues nothing.  A failed launch returns ULY_ERR_CUDA.  Kernels that
+ *    wait on their own pipeline stages give up after a bounded time and
+ *    record ULY_ERR_TIMEOUT in the workspace status word, which
+ *    ulysses_workspace_status() reads.  No call throws or aborts.
+ *  - position_ids contents are not validated (that would need a device
+ *    sync); whatever they hold is read by the sample-start rule above.
+ */
+#ifndef ULYSSES_H_
+#define ULYSSES_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ULY_OK = 0,
+  ULY_ERR_INVALID_ARG = 1,
+  ULY_ERR_UNSUPPORTED = 2,
+  ULY_ERR_CUDA = 3,
+  ULY_ERR_WORKSPACE = 4,
+  ULY_ERR_TIMEOUT = 5
+} uly_status;
+
+typedef enum { ULY_BF16 = 0, ULY_F32 = 1 } uly_dtype;
+
+/* Full (unsharded) problem sizes. */
+typedef struct {
+  int64_t b, n, h_q, h_kv, d;
+  int32_t P;
+} uly_shape;
+
+/*
+ * ulysses_seq_to_head -- the first all-to-all ("How Ulysses works", step 3):
+ *   x_head[r][bb][t][j][:] = x_seq[t / (n/P)][bb][t % (n/P)][r*(H/P) + j][:]
+ * x_seq [P][b][n/P][H][d] -> x_head [P][b][n][H/P][d], elements of `dt`.
+ * Requires n % P == 0 and H % P == 0 (Transformers docs "Ulysses sequence
+ * parallelism", "Configuration": heads divisible by sp_size, sequence padded
+ * to a multiple of sp_size).  Out of place: the buffers must not overlap.
+ * Bit-exact copy.
+ */
+uly_status ulysses_seq_to_head(const void* x_seq, void* x_head, int64_t b, int64_t n, int64_t H,
+                               int64_t d, int32_t P, uly_dtype dt, void* stream);
+
+/*
+ * ulysses_head_to_seq -- the second all-to-all ("How Ulysses works", step 5),
+ * the exact inverse of ulysses_seq_to_head:
+ *   x_seq[s][bb][u][g][:] = x_head[g / (H/P)][bb][s*(n/P) + u][g % (H/P)][:]
+ * Same requirements.  Also the backward of ulysses_seq_to_head.
+ */
+uly_status ulysses_head_to_seq(const void* x_head, void* x_seq, int64_t b, int64_t n, int64_t H,
+                               int64_t d, int32_t P, uly_dtype dt, void* stream);
+
+/* Workspace bytes ulysses_attn_fwd needs for `shape` (0 on invalid shape). */
+size_t ulysses_attn_fwd_workspace(const uly_shape* shape);
+
+/*
+ * ulysses_attn_fwd -- local causal attention of each rank on its head slice
+ * ("How Ulysses works", step 4), with causality and sample boundaries from
+ * position_ids (blog, position_ids paragraph; Accelerate guide "Sequence
+ * parallelism", "ALST/Ulysses SP backend configuration": packed samples must
+ * not attend to one another).  For rank r, local query head j (kv head j/G),
+ * and row i:  O_i = sum_j softmax_j(scale * q_i . k_j) v_j over keys j <= i
+ * in i's sample;  LSE_i = log sum_j exp(scale * q_i . k_j).
+ *   q_head [P][b][n][h_q/P][d] bf16, k_head / v_head [P][b][n][h_kv/P][d]
+ *   bf16, position_ids [b][n] int64 (device).
+ *   rank: -1 computes every rank; 0 <= rank < P computes only that rank's
+ *   slice (rows of other ranks in o_head / lse are left untouched).
+ *   softmax_scale <= 0 selects 1/sqrt(d).
+ *   o_head [P][b][n][h_q/P][d] of o_dtype (ULY_BF16 or ULY_F32);
+ *   lse [P][b][h_q/P][n] float32.
+ *   ws / ws_bytes: device workspace of at least ulysses_attn_fwd_workspace()
+ *   bytes, 256-byte aligned (else ULY_ERR_WORKSPACE).
+ * Supports d in {64, 128} (else ULY_ERR_UNSUPPORTED).
+ */
+uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, const void* v_head,
+                            const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                            float softmax_scale, void* o_head, uly_dtype o_dtype, float* lse,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes ulysses_attn_bwd needs for `shape` and gradient dtype. */
+size_t ulysses_attn_bwd_workspace(const uly_shape* shape, uly_dtype g_dtype);
+
+/*
+ * ulysses_attn_bwd -- gradients of the local attention (training through the
+ * layer, Accelerate guide "Sequence parallelism", custom training loop):
+ *   D_i = dO_i . O_i;  P_ij = exp(scale * q_i . k_j - LSE_i);
+ *   dS_ij = P_ij (dO_i . v_j - D_i);
+ *   dQ_i = scale * sum_j dS_ij k_j;
+ *   dK_j = scale * sum_{query heads of j's group} sum_i dS_ij q_i;
+ *   dV_j = sum_{query heads of j's group} sum_i P_ij dO_i.
+ * Inputs in head layout as for ulysses_attn_fwd; o_head / lse are that call's
+ * outputs (o_dtype must match); do_head has q_head's layout (bf16).
+ * Outputs dq_head (q_head's layout), dk_head / dv_head (k_head's layout), of
+ * g_dtype.  rank / softmax_scale as for the forward.
+ */
+uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* v_head,
+                            const void* o_head, uly_dtype o_dtype, const float* lse,
+                            const void* do_head, const int64_t* position_ids,
+                            const uly_shape* shape, int32_t rank, float softmax_scale,
+                            void* dq_head, void* dk_head, void* dv_head, uly_dtype g_dtype,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ulysses_workspace_status -- synchronizes `stream`, then reads and clears
+ * the status word kept at the start of an attention workspace.  *code gets
+ * ULY_OK, or ULY_ERR_TIMEOUT when a kernel gave up waiting on one of its own
+ * pipeline stages (its outputs are then invalid).
+ */
+uly_status ulysses_workspace_status(void* ws, void* stream, int32_t* code);
+
+/* Static English text for a status code. */
+const char* ulysses_status_string(uly_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ULYSSES_H_ */

@@ -44,7 +44,7 @@ import numpy as np
 
 __all__ = [
     "check_shape", "valid_sp_sizes",
-    "shard", "unshard", "seq_to_head", "head_to_seq",
+    "shard", "unshard", "seq_to_head", "head_to_seq", "seq_to_head_window", "head_to_seq_window",
     "segment_ids", "segment_starts", "segment_ends", "allowed_matrix",
     "attention_brute_head", "attention_bwd_brute_head",
     "attention_fwd_head", "attention_bwd_head",
@@ -145,6 +145,32 @@ def head_to_seq(x_head: np.ndarray, P: int) -> np.ndarray:
     src_head = np.broadcast_to(g % h, (P, m, H))
     gathered = x_head[src_rank, :, src_tok, src_head]          # (P, m, H, b, d)
     return np.ascontiguousarray(gathered.transpose(0, 3, 1, 2, 4))
+
+
+def seq_to_head_window(x_seq: np.ndarray, P: int, r: int, t_lo: int, t_hi: int) -> np.ndarray:
+    """Tokens [t_lo, t_hi) of rank r's head-sharded buffer, [b][T][H/P][d].
+
+    The same index formula as seq_to_head, evaluated only for those rows, so
+    multi-GiB buffers can be checked window by window.
+    """
+    Ps, b, m, H, d = x_seq.shape
+    h = H // P
+    t = np.arange(t_lo, t_hi)[:, None]
+    j = np.arange(h)[None, :]
+    shape = (t_hi - t_lo, h)
+    g = x_seq[np.broadcast_to(t // m, shape), :, np.broadcast_to(t % m, shape), np.broadcast_to(r * h + j, shape)]
+    return np.ascontiguousarray(g.transpose(2, 0, 1, 3))
+
+
+def head_to_seq_window(x_head: np.ndarray, P: int, s: int, u_lo: int, u_hi: int) -> np.ndarray:
+    """Tokens [u_lo, u_hi) of rank s's seq-sharded buffer, [b][U][H][d]."""
+    Ps, b, n, h, d = x_head.shape
+    m, H = n // P, h * P
+    u = np.arange(u_lo, u_hi)[:, None]
+    g = np.arange(H)[None, :]
+    shape = (u_hi - u_lo, H)
+    x = x_head[np.broadcast_to(g // h, shape), :, np.broadcast_to(s * m + u, shape), np.broadcast_to(g % h, shape)]
+    return np.ascontiguousarray(x.transpose(2, 0, 1, 3))
 
 
 # --------------------------------------------------------------------------

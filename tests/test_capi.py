@@ -1,0 +1,108 @@
+"""The C ABI on the CPU host: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any launch.
+
+The argument checks below pass fake (never dereferenced) device pointers, so
+they only run where no GPU is present: a check that wrongly let one through
+must not reach a real device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "ulysses.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ulysses_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    import ulysses_head_attention_b200 as uly
+    names = header_functions()
+    assert names == sorted(uly.EXPORTS)
+    for n in names:
+        assert hasattr(uly.lib, n), n
+
+
+def test_status_strings():
+    import ulysses_head_attention_b200 as uly
+    for code in range(6):
+        assert uly.status_string(code) and uly.status_string(code) != "unknown status"
+    assert uly.status_string(99) == "unknown status"
+
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake-pointer checks run only without a GPU")
+F = 0x100000          # fake, 256-byte aligned "device" addresses, never dereferenced
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 4
+
+
+@no_gpu
+@pytest.mark.parametrize("args,want", [
+    ((F, F + 1 << 30, 1, 100, 32, 128, 8), INVALID),        # n % P != 0 (padding rule)
+    ((F, F + 1 << 30, 1, 64, 12, 128, 8), INVALID),         # H % P != 0 (head rule)
+    ((F, F + 1 << 30, 1, 64, 32, 128, 0), INVALID),         # P < 1
+    ((0, F + 1 << 30, 1, 64, 32, 128, 4), INVALID),         # null input
+    ((F + 8, F + 1 << 30, 1, 64, 32, 128, 4), INVALID),     # misaligned
+    ((F, F + 1024, 1, 64, 32, 128, 4), INVALID),            # overlapping buffers
+])
+def test_relayout_rejects(args, want):
+    import ulysses_head_attention_b200 as uly
+    src, dst, b, n, H, d, P = args
+    for fn in (uly.lib.ulysses_seq_to_head, uly.lib.ulysses_head_to_seq):
+        assert fn(src, dst, b, n, H, d, P, 0, None) == want
+
+
+def shape(b=1, n=1024, hq=32, hkv=8, d=128, P=4):
+    import ulysses_head_attention_b200 as uly
+    return uly.make_shape(b, n, hq, hkv, d, P)
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,rank,want", [
+    (dict(n=1000, P=16), -1, INVALID),       # n % P
+    (dict(hkv=8, P=16), -1, INVALID),        # H_kv % P
+    (dict(hq=12, hkv=8, P=4), -1, INVALID),  # H_q % H_kv
+    (dict(P=0), -1, INVALID),
+    ({}, 4, INVALID),                        # rank out of range
+    ({}, -2, INVALID),
+    (dict(d=96), -1, UNSUPPORTED),           # head dim not implemented
+])
+def test_attention_rejects_shapes(kw, rank, want):
+    import ulysses_head_attention_b200 as uly
+    s = shape(**kw)
+    G = 1 << 30
+    ws_bytes = 1 << 24
+    st = uly.lib.ulysses_attn_fwd(F, F + G, F + 2 * G, F + 3 * G, ctypes.byref(s), rank, 0.0, F + 4 * G, 1,
+                                  F + 5 * G, F + 6 * G, ws_bytes, None)
+    assert st == want
+    st = uly.lib.ulysses_attn_bwd(F, F + G, F + 2 * G, F + 3 * G, 1, F + 4 * G, F + 5 * G, F + 6 * G,
+                                  ctypes.byref(s), rank, 0.0, F + 7 * G, F + 8 * G, F + 9 * G, 1,
+                                  F + 10 * G, ws_bytes, None)
+    assert st == want
+
+
+@no_gpu
+def test_attention_rejects_workspace():
+    import ulysses_head_attention_b200 as uly
+    s = shape()
+    need = uly.ulysses_attn_fwd_workspace(s)
+    assert need > 0
+    G = 1 << 30
+    for ws, nbytes in ((0, need), (F + 6 * G, need - 1), (F + 6 * G + 16, need)):
+        st = uly.lib.ulysses_attn_fwd(F, F + G, F + 2 * G, F + 3 * G, ctypes.byref(s), -1, 0.0, F + 4 * G, 1,
+                                      F + 5 * G, ws, nbytes, None)
+        assert st == WORKSPACE
+
+
+def test_workspace_queries_reject_bad_shapes():
+    import ulysses_head_attention_b200 as uly
+    assert uly.ulysses_attn_fwd_workspace(shape(n=1001)) == 0
+    assert uly.ulysses_attn_bwd_workspace(shape(P=3), 1) == 0
+    assert uly.ulysses_attn_fwd_workspace(shape()) >= 256 + 2 * 4 * 1024

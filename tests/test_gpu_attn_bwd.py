@@ -1,0 +1,119 @@
+"""GPU parity of the attention backward against the fp64 oracle.
+
+The GPU forward produces O (fp32) and LSE; the GPU backward then produces
+dQ, dK, dV.  The oracle's backward recomputes everything in fp64 from the
+same bf16 inputs (its own O, not the GPU's).  Tolerance for fp32-stored
+gradients: sum|g-r|/sum|r| <= 2e-3 and max-abs <= 1e-2, element by element;
+on these short-row shapes the absolute bound scales with the output
+magnitude (gpu_util.edge_max_abs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from gpu_util import MAX_ABS_BF16, MEAN_REL_BF16, assert_close, edge_max_abs, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _uly():
+    import ulysses_head_attention_b200 as uly
+    return uly
+
+
+def head_layout(bits, P):
+    return oracle.seq_to_head(oracle.shard(bits, P), P)
+
+
+def gpu_fwd_bwd(x, P, dev, g_dtype=torch.float32, o_dtype=torch.float32, rank=-1, sentinel=None):
+    uly = _uly()
+    heads = [head_layout(x[k], P) for k in ("q", "k", "v", "do")]
+    q, k, v, do = (to_dev_bf16(t, dev) for t in heads)
+    pos = torch.from_numpy(x["position_ids"]).to(dev)
+    Ps, b, n, hq, d = heads[0].shape
+    hkv = heads[1].shape[3]
+    shape = uly.make_shape(b, n, hq * P, hkv * P, d, P)
+    o = torch.zeros((P, b, n, hq, d), dtype=o_dtype, device=dev)
+    lse = torch.zeros((P, b, hq, n), dtype=torch.float32, device=dev)
+    ws_f = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(shape), dev)
+    uly.ulysses_attn_fwd(q, k, v, pos, o, lse, ws_f, rank=rank)
+    code = 0 if g_dtype == torch.bfloat16 else 1
+    ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, code), dev)
+    dq = torch.empty_like(q, dtype=g_dtype)
+    dk = torch.empty_like(k, dtype=g_dtype)
+    dv = torch.empty_like(v, dtype=g_dtype)
+    if sentinel is not None:
+        for t in (dq, dk, dv):
+            t.fill_(sentinel)
+    uly.ulysses_attn_bwd(q, k, v, o, lse, do, pos, dq, dk, dv, ws_b, rank=rank)
+    assert uly.ulysses_workspace_status(ws_f) == 0
+    assert uly.ulysses_workspace_status(ws_b) == 0
+    return [t.float().cpu().numpy() for t in (dq, dk, dv)], heads
+
+
+def oracle_bwd(heads, pos, P, rank=None):
+    qh, kh, vh, doh = (synthetic.bf16_bits_to_f64(t) for t in heads)
+    return oracle.ulysses_attn_bwd(qh, kh, vh, doh, pos, P, rank=rank)
+
+
+CASES = [
+    # (id, P, b, n, h_q, h_kv, d, lengths)
+    ("single_256", 2, 1, 256, 4, 2, 128, None),
+    ("ragged_gqa2", 4, 1, 1000, 8, 4, 128, None),
+    ("packed_tile_edges", 2, 1, 640, 4, 2, 128, [[128, 1, 127, 256, 100, 28]]),
+    ("batch2_packed_d64", 2, 2, 384, 4, 2, 64, [[384], [200, 184]]),
+    ("gqa_g4", 2, 1, 512, 16, 4, 128, [[300, 212]]),
+    ("gqa_g8_d64", 1, 1, 520, 8, 1, 64, [[1, 1, 1, 517]]),
+    ("mha_g1_odd", 1, 1, 300, 2, 2, 128, [[77, 223]]),
+    ("long_2k", 2, 1, 2048, 4, 2, 128, None),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_bwd_matches_oracle(cuda_device, case):
+    name, P, b, n, hq, hkv, d, lengths = case
+    x = synthetic.custom_inputs(200 + CASES.index(case), b, n, hq, hkv, d, lengths=lengths)
+    (dq, dk, dv), heads = gpu_fwd_bwd(x, P, cuda_device)
+    dq_r, dk_r, dv_r = oracle_bwd(heads, x["position_ids"], P)
+    for got, ref, nm in ((dq, dq_r, "dQ"), (dk, dk_r, "dK"), (dv, dv_r, "dV")):
+        assert_close(got, ref, f"{name} {nm}", max_abs=edge_max_abs(ref))
+
+
+def test_bwd_bf16_storage(cuda_device):
+    """bf16 O in, bf16 dQ/dK/dV out (dQ through the fp32 workspace)."""
+    x = synthetic.custom_inputs(230, 1, 768, 8, 2, 128, lengths=[[500, 268]])
+    (dq, dk, dv), heads = gpu_fwd_bwd(x, 2, cuda_device, g_dtype=torch.bfloat16, o_dtype=torch.bfloat16)
+    dq_r, dk_r, dv_r = oracle_bwd(heads, x["position_ids"], 2)
+    for got, ref, nm in ((dq, dq_r, "dQ"), (dk, dk_r, "dK"), (dv, dv_r, "dV")):
+        assert_close(got, ref, f"bf16 {nm}", edge_max_abs(ref, MAX_ABS_BF16), MEAN_REL_BF16)
+
+
+def test_bwd_single_rank_leaves_others_untouched(cuda_device):
+    P = 4
+    x = synthetic.custom_inputs(231, 1, 512, 8, 4, 128, lengths=[[256, 256]])
+    rank = 1
+    (dq, dk, dv), heads = gpu_fwd_bwd(x, P, cuda_device, rank=rank, sentinel=7.0)
+    dq_r, dk_r, dv_r = oracle_bwd(heads, x["position_ids"], P, rank=rank)
+    for got, ref, nm in ((dq[rank], dq_r[rank], "dQ"), (dk[rank], dk_r[rank], "dK"), (dv[rank], dv_r[rank], "dV")):
+        assert_close(got, ref, f"rank {nm}", max_abs=edge_max_abs(ref))
+    others = [s for s in range(P) if s != rank]
+    for t in (dq, dk, dv):
+        assert (t[others] == 7.0).all()
+
+
+def test_bwd_column_sums(cuda_device):
+    """Properties that hold at any size: sum_j dK_j = 0 and
+    sum_j dV_j = sum over the group's heads and rows of dO."""
+    x = synthetic.custom_inputs(232, 1, 1024, 8, 2, 128, lengths=[[700, 324]])
+    P = 2
+    (dq, dk, dv), heads = gpu_fwd_bwd(x, P, cuda_device)
+    do = synthetic.bf16_bits_to_f64(heads[3])
+    G = 4
+    for r in range(P):
+        s = dk[r, 0].sum(axis=0)
+        assert np.abs(s).max() <= 1e-3 * np.abs(dk[r, 0]).sum(axis=0).max()
+        for g in range(dv.shape[3]):
+            want = do[r, 0, :, g * G:(g + 1) * G].sum(axis=(0, 1))
+            assert np.abs(dv[r, 0, :, g].sum(axis=0) - want).max() <= 1e-3 * max(1.0, np.abs(want).max())

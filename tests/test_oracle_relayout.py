@@ -121,3 +121,16 @@ def test_sp_sizes_for_32_heads():
 def test_check_shape_rejects(args):
     with pytest.raises(ValueError):
         oracle.check_shape(*args)
+
+
+@pytest.mark.parametrize("b,n,H,d,P", SHAPES)
+def test_windows_match_full(b, n, H, d, P):
+    x_seq = oracle.shard(iota((b, n, H, d)), P)
+    x_head = oracle.seq_to_head(x_seq, P)
+    for r in range(P):
+        for lo, hi in ((0, n), (1, n - 1), (n // 2, n // 2 + 1)):
+            assert np.array_equal(oracle.seq_to_head_window(x_seq, P, r, lo, hi), x_head[r][:, lo:hi])
+    m = n // P
+    for s in range(P):
+        for lo, hi in ((0, m), (m - 1, m)):
+            assert np.array_equal(oracle.head_to_seq_window(x_head, P, s, lo, hi), x_seq[s][:, lo:hi])

@@ -1,0 +1,181 @@
+"""Python binding of libulysses.so (the Ulysses SP hot path on one B200).
+
+Argument marshalling only: every function below checks that the tensors it
+is handed are CUDA tensors of the documented shape/dtype, then calls the C
+entry point of the same name (declared in include/ulysses.h) with their
+device pointers and the current CUDA stream.  All arithmetic runs in the
+library's kernels; there is no Python or CPU fallback.  Importing this module
+fails loudly when the library has not been built.
+
+Shapes (full sizes b, n, H, d; P virtual ranks):
+    seq-sharded   (P, b, n/P, H, d)
+    head-sharded  (P, b, n, H/P, d)
+    lse           (P, b, h_q/P, n) float32
+    position_ids  (b, n) int64, on the device
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libulysses.so")
+
+ULY_BF16, ULY_F32 = 0, 1
+STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED", 3: "ULY_ERR_CUDA",
+                4: "ULY_ERR_WORKSPACE", 5: "ULY_ERR_TIMEOUT"}
+# Every symbol include/ulysses.h declares.
+EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
+           "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_workspace_status", "ulysses_status_string")
+
+
+class UlyShape(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("n", ctypes.c_int64), ("h_q", ctypes.c_int64),
+                ("h_kv", ctypes.c_int64), ("d", ctypes.c_int64), ("P", ctypes.c_int32)]
+
+
+class UlyssesError(RuntimeError):
+    def __init__(self, what: str, status: int):
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m ulysses_head_attention_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    shp = ctypes.POINTER(UlyShape)
+    sig = {
+        "ulysses_seq_to_head": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
+        "ulysses_head_to_seq": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
+        "ulysses_attn_fwd_workspace": ([shp], sz),
+        "ulysses_attn_fwd": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp, sz, vp], i32),
+        "ulysses_attn_bwd_workspace": ([shp, i32], sz),
+        "ulysses_attn_bwd": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i32, f32, vp, vp, vp, i32, vp, sz, vp], i32),
+        "ulysses_workspace_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
+        "ulysses_status_string": ([i32], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.ulysses_status_string(status).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise UlyssesError(what, status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ULY_BF16
+    if t.dtype == torch.float32:
+        return ULY_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_shape(b: int, n: int, h_q: int, h_kv: int, d: int, P: int) -> UlyShape:
+    return UlyShape(b, n, h_q, h_kv, d, P)
+
+
+def ulysses_seq_to_head(x_seq: torch.Tensor, x_head: torch.Tensor, stream=None) -> None:
+    """x_seq (P, b, n/P, H, d) -> x_head (P, b, n, H/P, d)."""
+    P, b, m, H, d = x_seq.shape
+    if tuple(x_head.shape) != (P, b, m * P, H // P, d) or x_head.dtype != x_seq.dtype:
+        raise ValueError("x_head shape/dtype does not match x_seq")
+    _check(lib.ulysses_seq_to_head(_dev(x_seq, "x_seq"), _dev(x_head, "x_head"), b, m * P, H, d, P,
+                                   _dtype_code(x_seq), _stream(stream)), "ulysses_seq_to_head")
+
+
+def ulysses_head_to_seq(x_head: torch.Tensor, x_seq: torch.Tensor, stream=None) -> None:
+    """x_head (P, b, n, H/P, d) -> x_seq (P, b, n/P, H, d)."""
+    P, b, n, h, d = x_head.shape
+    if tuple(x_seq.shape) != (P, b, n // P, h * P, d) or x_seq.dtype != x_head.dtype:
+        raise ValueError("x_seq shape/dtype does not match x_head")
+    _check(lib.ulysses_head_to_seq(_dev(x_head, "x_head"), _dev(x_seq, "x_seq"), b, n, h * P, d, P,
+                                   _dtype_code(x_head), _stream(stream)), "ulysses_head_to_seq")
+
+
+def _attn_shape(q_head: torch.Tensor, k_head: torch.Tensor) -> UlyShape:
+    P, b, n, hq, d = q_head.shape
+    Pk, bk, nk, hkv, dk = k_head.shape
+    if (Pk, bk, nk, dk) != (P, b, n, d):
+        raise ValueError("k_head shape does not match q_head")
+    return UlyShape(b, n, hq * P, hkv * P, d, P)
+
+
+def ulysses_attn_fwd_workspace(shape: UlyShape) -> int:
+    return int(lib.ulysses_attn_fwd_workspace(ctypes.byref(shape)))
+
+
+def ulysses_attn_bwd_workspace(shape: UlyShape, g_dtype: int) -> int:
+    return int(lib.ulysses_attn_bwd_workspace(ctypes.byref(shape), g_dtype))
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    """A zeroed uint8 workspace tensor (torch's allocator aligns to >= 256 B)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def ulysses_attn_fwd(q_head, k_head, v_head, position_ids, o_head, lse, ws, rank: int = -1,
+                     softmax_scale: float = 0.0, stream=None) -> None:
+    """Local causal attention of every rank (or `rank`) on its head slice."""
+    shape = _attn_shape(q_head, k_head)
+    for t, nm in ((k_head, "k_head"), (v_head, "v_head"), (q_head, "q_head")):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{nm} must be bfloat16")
+    if position_ids.dtype != torch.int64:
+        raise TypeError("position_ids must be int64")
+    _check(lib.ulysses_attn_fwd(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
+                                _dev(position_ids, "position_ids"), ctypes.byref(shape), rank, softmax_scale,
+                                _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
+                                _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+           "ulysses_attn_fwd")
+
+
+def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse, do_head, position_ids, dq_head, dk_head, dv_head, ws,
+                     rank: int = -1, softmax_scale: float = 0.0, stream=None) -> None:
+    """Gradients dQ, dK, dV of the local attention (head layout)."""
+    shape = _attn_shape(q_head, k_head)
+    if dk_head.dtype != dq_head.dtype or dv_head.dtype != dq_head.dtype:
+        raise TypeError("dq/dk/dv must share one dtype")
+    _check(lib.ulysses_attn_bwd(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
+                                _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
+                                _dev(do_head, "do_head"), _dev(position_ids, "position_ids"), ctypes.byref(shape),
+                                rank, softmax_scale, _dev(dq_head, "dq_head"), _dev(dk_head, "dk_head"),
+                                _dev(dv_head, "dv_head"), _dtype_code(dq_head), _dev(ws, "ws"),
+                                ws.numel() * ws.element_size(), _stream(stream)),
+           "ulysses_attn_bwd")
+
+
+def ulysses_workspace_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronize, then read and clear the workspace status word (0 = ok)."""
+    code = ctypes.c_int32(-1)
+    _check(lib.ulysses_workspace_status(_dev(ws, "ws"), _stream(stream), ctypes.byref(code)),
+           "ulysses_workspace_status")
+    return int(code.value)

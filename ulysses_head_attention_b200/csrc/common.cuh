@@ -1,0 +1,65 @@
+// Host-side helpers shared by the entry points: argument checks, status
+// mapping, tensor-map encoding through the driver entry point.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/ulysses.h"
+
+namespace uly {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+inline size_t dtype_size(uly_dtype t) { return t == ULY_F32 ? 4 : 2; }
+inline bool dtype_ok(uly_dtype t) { return t == ULY_BF16 || t == ULY_F32; }
+
+// Product of non-negative sizes, false on overflow past 2^62.
+inline bool checked_mul(int64_t a, int64_t b, int64_t* out) {
+  if (a < 0 || b < 0) return false;
+  if (a != 0 && b > (int64_t(1) << 62) / a) return false;
+  *out = a * b;
+  return true;
+}
+
+inline bool elems(int64_t b, int64_t n, int64_t H, int64_t d, int64_t* out) {
+  int64_t t;
+  return checked_mul(b, n, &t) && checked_mul(t, H, &t) && checked_mul(t, d, out);
+}
+
+// The divisibility rules of the pages: n and both head counts divisible by
+// P; H_q a multiple of H_kv.
+inline uly_status check_shape(const uly_shape* s) {
+  if (!s) return ULY_ERR_INVALID_ARG;
+  if (s->P < 1 || s->b < 1 || s->n < 1 || s->h_q < 1 || s->h_kv < 1 || s->d < 1) return ULY_ERR_INVALID_ARG;
+  if (s->n % s->P || s->h_q % s->P || s->h_kv % s->P || s->h_q % s->h_kv) return ULY_ERR_INVALID_ARG;
+  if (s->n > (int64_t(1) << 31) - 256) return ULY_ERR_UNSUPPORTED;   // TMA coordinates are int32
+  int64_t e;
+  if (!elems(s->b, s->n, s->h_q, s->d, &e)) return ULY_ERR_INVALID_ARG;
+  return ULY_OK;
+}
+
+inline uly_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA; }
+
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).  Looked up once; the lookup result is immutable.
+TensorMapEncodeFn tensor_map_encoder();
+
+// 4-D bf16 tensor map over a head-layout tensor [P*b][n][h][d] viewed as
+// dims {d, h, n, P*b}; box {64, 1, rows, 1}, 128-byte swizzle.
+bool make_head_map(CUtensorMap* map, const void* base, int64_t Pb, int64_t n, int64_t h, int64_t d,
+                   uint32_t box_rows);
+
+}  // namespace uly
