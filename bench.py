@@ -205,7 +205,8 @@ def run_ours(args, w):
     ws_f = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(shape), dev)
     ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, uly.ULY_F32), dev)
     stream = torch.cuda.current_stream()
-    launches_per_step = 3 + 2 + 1 + 1 + 3 + 3     # s2h x3, fwd (2), h2s O, s2h dO, bwd (3), h2s x3
+    # s2h x3; fwd: segments + attn_fwd; h2s O; s2h dO; bwd: segments + bwd_pre + bwd_dkdv + bwd_dq; h2s x3
+    launches_per_step = 3 + 2 + 1 + 1 + 4 + 3
 
     relayout_bytes = 2 * sum(t.numel() * t.element_size() for t in (seq["q"], seq["k"], seq["v"], seq["do"]))
     relayout_bytes += 2 * sum(t.numel() * t.element_size() for t in (o_seq, g_seq["q"], g_seq["k"], g_seq["v"]))
@@ -331,7 +332,7 @@ def run_ours(args, w):
             "bwd_flops_with_recompute_convention": 10 * d * hq * pairs,
             "peaks": peaks,
         },
-        "roofline": {"bound": "tensor", "kernel": "attn_bwd (ulysses_attn_bwd call: segments + pre + main)",
+        "roofline": {"bound": "tensor", "kernel": "attn_bwd: one ulysses_attn_bwd call (segments, bwd_pre, bwd_dkdv, bwd_dq kernels)",
                      "achieved": bwd_tf, "peak": peak_t, "unit": "TFLOP/s", "frac": bwd_tf / peak_t,
                      "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "traffic": None},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

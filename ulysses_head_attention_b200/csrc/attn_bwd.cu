@@ -4,34 +4,36 @@
 // parallelism", custom training loop: the loss is backpropagated through the
 // attention); the gradient of the local attention of blog "Ulysses Sequence
 // Parallelism: Training with Million-Token Contexts", "How Ulysses works",
-// step 4, with the same position_ids causality as the forward.
+// step 4, with the forward's position_ids causality.
 //
-//   D_i   = dO_i . O_i                       (bwd_pre kernel)
-//   P_ij  = exp(scale q_i.k_j - LSE_i)        recomputed from the forward LSE
+//   D_i   = dO_i . O_i
+//   P_ij  = exp(scale q_i.k_j - LSE_i)        (recomputed from the forward LSE)
 //   dS_ij = P_ij (dO_i . v_j - D_i)
 //   dV_j  = sum_{group heads} sum_i P_ij dO_i
 //   dK_j  = scale sum_{group heads} sum_i dS_ij q_i
-//   dQ_i  = scale sum_j dS_ij k_j             (fp32 reductions across key tiles)
+//   dQ_i  = scale sum_j dS_ij k_j
 //
-// Main kernel: one CTA per (rank, batch row, kv head, 128-key tile), heaviest
-// (earliest) key tiles first.  It loops over the G query heads of the kv
-// head and the 64-row query tiles that can see the key tile:
-//   warp 0      TMA producer (K, V once; Q / dO tiles into a 2-stage ring)
-//   warp 1      TMEM owner, single-thread tcgen05 MMA issuer
-//   warps 4..7  thread = key row: P^T and dS^T from S^T, dP^T (TMEM) into
-//               128B-swizzled shared memory; at the end dK, dV to global
-//   warps 8..11 thread = head-dim index: dQ^T tile (TMEM) -> red.add into
-//               an fp32 dQ accumulator
-// MMAs per query tile (M = 128 always):
-//   S^T  = K  Q^T   (A: K  K-major,  B: Q  K-major)        N = 64
-//   dP^T = V  dO^T  (A: V  K-major,  B: dO K-major)        N = 64
-//   dV  += P^T dO   (A: P^T K-major, B: dO MN-major)       N = D
-//   dK  += dS^T Q   (A: dS^T K-major, B: Q MN-major)       N = D
-//   dQ^T = K^T dS^T (A: K MN-major,  B: dS^T MN-major)     N = 64
-// TMEM columns: dK [0,128) dV [128,256) S^T [256,320) dP^T [320,384)
-// dQ^T [384,448).  For D = 64 the dQ^T product still runs with M = 128: its
-// A operand's second 64-row half points at the V tile and those output
-// lanes are ignored.
+// Three kernels, no atomics (results are bitwise reproducible):
+//  * bwd_pre:   D_i and LSE_i*log2(e) per (rank, head, row), written as
+//               interleaved pairs into a padded workspace table.
+//  * bwd_dkdv:  one CTA per (rank, batch row, kv head, 128-key tile),
+//               heaviest first.  Loops over the G query heads of the kv head
+//               and the 64-row query tiles that can see the key tile:
+//                 warp 0      TMA producer (K, V once; Q, dO, row stats ring)
+//                 warp 1      TMEM owner, single-thread MMA issuer
+//                 warps 4..7  thread = key row: P^T, dS^T from S^T, dP^T
+//               S^T = K Q^T and dP^T = V dO^T (M=128 keys, N=64) are double
+//               buffered in TMEM; P^T and dS^T go back to TMEM as bf16 over
+//               them and feed dV += P^T dO, dK += dS^T Q as A-from-TMEM MMAs
+//               accumulating in TMEM across the whole group.
+//               TMEM: dK [0,128) dV [128,256) S^T_b [256+128b, +64)
+//               dP^T_b [320+128b, +64).
+//  * bwd_dq:    one CTA per (rank, batch row, query head, 128-row tile),
+//               heaviest first; the forward's structure.  S = Q K^T into a
+//               double-buffered TMEM tile, dP = dO V^T, two softmax
+//               warpgroups (64 columns each) turn them into dS (bf16, over S)
+//               and dQ += dS K accumulates in TMEM.
+//               TMEM: S_0 [0,128) S_1 [128,256) dP [256,384) dQ [384,512).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -43,22 +45,64 @@
 namespace uly {
 namespace bwd {
 
-constexpr int BKV = 128;   // keys per CTA
-constexpr int BQ = 64;     // query rows per inner tile
-constexpr int NS = 2;      // Q/dO stages
-constexpr int kThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ============================================================================
+// bwd_pre: D = rowsum(dO * O) and LSE*log2(e), one warp per (rank, row, head)
+// ============================================================================
+// stats layout: [P*b][hq][n_pad] x float2 {LSE*log2e, D}; rows n..n_pad-1 zero.
+template <int D, bool kOF32>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const uint16_t* __restrict__ dO,
+                                                      const float* __restrict__ lse, float2* __restrict__ stats,
+                                                      int64_t rb0, int64_t n, int64_t n_pad, int32_t hq,
+                                                      int64_t total) {
+  const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= total) return;
+  const int64_t per_rb = n_pad * hq;
+  const int64_t rb = rb0 + w / per_rb;
+  const int64_t rem = w % per_rb;
+  const int64_t i = rem / hq;          // token (head fastest: consecutive warps read adjacent rows)
+  const int64_t h = rem % hq;
+  const int64_t sidx = (rb * hq + h) * n_pad + i;
+  if (i >= n) {
+    if (lane == 0) stats[sidx] = make_float2(0.f, 0.f);
+    return;
+  }
+  const int64_t row = (rb * n + i) * hq + h;
+  constexpr int E = D / 32;
+  float acc = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int64_t x = row * D + lane * E + e;
+    const float dv = __uint_as_float(uint32_t(dO[x]) << 16);
+    const float ov = kOF32 ? static_cast<const float*>(o)[x]
+                           : __uint_as_float(uint32_t(static_cast<const uint16_t*>(o)[x]) << 16);
+    acc = fmaf(dv, ov, acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) stats[sidx] = make_float2(lse[(rb * hq + h) * n + i] * kLog2e, acc);
+}
+
+// ============================================================================
+// bwd_dkdv
+// ============================================================================
+namespace dkdv {
+
+constexpr int BKV = 128;
+constexpr int BQ = 64;
+constexpr int NS = 3;
+constexpr int kThreads = 256;
 
 struct Params {
-  const int32_t* segstart;
   const int32_t* segend;
-  const float* lse;     // [P*b][hq][n]
-  const float* delta;   // [P*b][hq][n]
-  float* dq_acc;        // [P*b][n][hq][D] fp32, pre-zeroed
-  void* dk;             // [P*b][n][hkv][D]
+  const float2* stats;   // [P*b][hq][n_pad]
+  void* dk;              // [P*b][n][hkv][D]
   void* dv;
   int* status;
-  int64_t n;
-  int32_t b, P_sel, rank0, hq, hkv, G, nkt;
+  int64_t n, n_pad;
+  int32_t b, P_sel, rank0, hq, hkv, G;
   float scale, scale_log2;
   int32_t g_f32;
   uint64_t limit_ns;
@@ -66,42 +110,38 @@ struct Params {
 
 template <int D>
 struct Layout {
-  static constexpr uint32_t kKVBytes = BKV * D * 2;      // K or V tile
-  static constexpr uint32_t kQBytes = BQ * D * 2;        // Q or dO tile
-  static constexpr uint32_t kPBytes = BKV * BQ * 2;      // P^T or dS^T tile
-  static constexpr uint32_t kK = 0;
-  static constexpr uint32_t kV = kK + kKVBytes;
-  static constexpr uint32_t kQ = kV + kKVBytes;          // NS stages of Q
-  static constexpr uint32_t kDO = kQ + NS * kQBytes;     // NS stages of dO
-  static constexpr uint32_t kPt = kDO + NS * kQBytes;
-  static constexpr uint32_t kDSt = kPt + kPBytes;
-  static constexpr uint32_t kRowStats = kDSt + kPBytes;  // 2 x (LSE*log2e, D) x 64 floats
-  static constexpr uint32_t kBar = kRowStats + 2 * 2 * BQ * 4;
-  static constexpr uint32_t kBytes = kBar + 256;
-  static constexpr uint32_t kDynamic = kBytes + 1024;
+  static constexpr uint32_t kKV = BKV * D * 2;
+  static constexpr uint32_t kQ = BQ * D * 2;
+  static constexpr uint32_t kSt = BQ * 8;
+  static constexpr uint32_t oK = 0;
+  static constexpr uint32_t oV = oK + kKV;
+  static constexpr uint32_t oQ = oV + kKV;
+  static constexpr uint32_t oDO = oQ + NS * kQ;
+  static constexpr uint32_t oSt = oDO + NS * kQ;
+  static constexpr uint32_t oBar = oSt + NS * kSt;
+  static constexpr uint32_t kDynamic = oBar + 256 + 1024;
 };
 
 struct Bars {
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
-  uint64_t sdp_full, sdp_free, p_ready, pds_free, dq_full, dq_free, mma_final;
-  uint64_t stats_ready[2];
+  uint64_t s_full[2], p_ready[2];
+  uint64_t mma_final;
   uint32_t tmem_base;
   int abort_flag;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo, const Params p) {
+kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+       const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo, const Params p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + L::kBar);
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::oBar);
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item: earliest key tiles (most query rows) first
   const int per_tile = p.P_sel * p.b * p.hkv;
   const int kt = int(blockIdx.x / per_tile);
   int rem = int(blockIdx.x % per_tile);
@@ -113,11 +153,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   const int64_t k0 = int64_t(kt) * BKV;
   const int64_t last_key = (k0 + BKV - 1 < p.n - 1) ? (k0 + BKV - 1) : (p.n - 1);
   const int32_t* se = p.segend + int64_t(bb) * p.n;
-  const int64_t q_end = se[last_key];          // rows that see this tile: [k0, q_end)
+  const int64_t q_end = se[last_key];      // query rows that see this key tile: [k0, q_end)
   const int64_t seg_end_min = se[k0];
   const int qt_first = int(k0 / BQ);
   const int nqt = int((q_end + BQ - 1) / BQ) - qt_first;
-  const int niter = nqt * p.G;                 // (head, query tile) pairs, head-major
+  const int niter = nqt * p.G;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -125,15 +165,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
     }
-    mbar_init(&bars->sdp_full, 1);
-    mbar_init(&bars->sdp_free, 128);
-    mbar_init(&bars->p_ready, 128);
-    mbar_init(&bars->pds_free, 1);
-    mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_free, 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_ready[s], 128);
+    }
     mbar_init(&bars->mma_final, 1);
-    mbar_init(&bars->stats_ready[0], 128);
-    mbar_init(&bars->stats_ready[1], 128);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -145,17 +181,18 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tDK = tmem, tDV = tmem + 128, tS = tmem + 256, tDP = tmem + 320, tDQ = tmem + 384;
+  const uint32_t tDK = tmem, tDV = tmem + 128;
+  auto tS = [&](int b) { return tmem + 256u + 128u * uint32_t(b); };
+  auto tDP = [&](int b) { return tmem + 320u + 128u * uint32_t(b); };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&mq);
       tma_prefetch_desc(&mdo);
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKVBytes);
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKV);
       for (int dc = 0; dc < D / 64; ++dc) {
-        tma_load_4d(&mk, &bars->kv_full, smem + L::kK + dc * BKV * 128, dc * 64, g, int(k0), rb);
-        tma_load_4d(&mv, &bars->kv_full, smem + L::kV + dc * BKV * 128, dc * 64, g, int(k0), rb);
+        tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0), rb);
+        tma_load_4d(&mv, &bars->kv_full, smem + L::oV + dc * BKV * 128, dc * 64, g, int(k0), rb);
       }
       int issued = 0;
       for (int it = 0; it < niter; ++it) {
@@ -163,147 +200,106 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         const int h = g * p.G + it / nqt;
         const int q0 = (qt_first + it % nqt) * BQ;
         if (rnd > 0 && !mbar_wait(&bars->q_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
-        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kQBytes);
+        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kQ + L::kSt);
         for (int dc = 0; dc < D / 64; ++dc) {
-          tma_load_4d(&mq, &bars->q_full[st], smem + L::kQ + st * L::kQBytes + dc * BQ * 128, dc * 64, h, q0, rb);
-          tma_load_4d(&mdo, &bars->q_full[st], smem + L::kDO + st * L::kQBytes + dc * BQ * 128, dc * 64, h, q0, rb);
+          tma_load_4d(&mq, &bars->q_full[st], smem + L::oQ + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
+          tma_load_4d(&mdo, &bars->q_full[st], smem + L::oDO + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
         }
+        bulk_load(smem + L::oSt + st * L::kSt, p.stats + (int64_t(rb) * p.hq + h) * p.n_pad + q0, L::kSt,
+                  &bars->q_full[st]);
         issued = it + 1;
       }
-      if (*abort_flag) {   // error path: let started copies land before exit
+      if (*abort_flag) {
         mbar_wait(&bars->kv_full, 0, nullptr, nullptr, p.limit_ns);
         for (int x = max(0, issued - NS); x < issued; ++x)
           mbar_wait(&bars->q_full[x % NS], (x / NS) & 1, nullptr, nullptr, p.limit_ns);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id_sdp = idesc_bf16(BKV, BQ, false, false);
-      const uint32_t id_grad = idesc_bf16(BKV, D, false, true);
-      const uint32_t id_dq = idesc_bf16(128, BQ, true, true);
-      const uint32_t k_addr = smem_u32(smem + L::kK), v_addr = smem_u32(smem + L::kV);
-      const uint32_t pt_addr = smem_u32(smem + L::kPt), ds_addr = smem_u32(smem + L::kDSt);
-      // dQ^T A operand (K^T, MN-major): 64-row chunks of the head dim are the
-      // K tile's 16 KB column chunks; for D = 64 the second chunk is the V tile.
-      const uint32_t kt_lbo = (D == 128) ? uint32_t(BKV * 128) : (L::kV - L::kK);
+      const uint32_t id_s = idesc_bf16(BKV, BQ, false, false);
+      const uint32_t id_g = idesc_bf16(BKV, D, false, true);
+      const uint32_t k_addr = smem_u32(smem + L::oK), v_addr = smem_u32(smem + L::oV);
       bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns);
       tc_fence_after();
       auto issue_grads = [&](int jt) -> bool {
-        const int st = jt % NS;
-        if (!mbar_wait(&bars->p_ready, jt & 1, abort_flag, p.status, p.limit_ns)) return false;
-        if (jt >= 1 && !mbar_wait(&bars->dq_free, (jt - 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
+        const int b = jt & 1, st = jt % NS;
+        if (!mbar_wait(&bars->p_ready[b], (jt >> 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + L::kQ + st * L::kQBytes);
-        const uint32_t do_addr = smem_u32(smem + L::kDO + st * L::kQBytes);
+        const uint32_t q_addr = smem_u32(smem + L::oQ + st * L::kQ);
+        const uint32_t do_addr = smem_u32(smem + L::oDO + st * L::kQ);
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint32_t acc = (jt > 0 || kk > 0) ? 1u : 0u;
-          umma_ss(tDV, sdesc_sw128(pt_addr + kk * 32, 16, 1024), sdesc_sw128(do_addr + kk * 2048, BQ * 128, 1024),
-                  id_grad, acc);
-          umma_ss(tDK, sdesc_sw128(ds_addr + kk * 32, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BQ * 128, 1024),
-                  id_grad, acc);
+          umma_ts(tDV, tS(b) + kk * 8, sdesc_sw128(do_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
+          umma_ts(tDK, tDP(b) + kk * 8, sdesc_sw128(q_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
         }
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          umma_ss(tDQ, sdesc_sw128(k_addr + kk * 2048, kt_lbo, 1024), sdesc_sw128(ds_addr + kk * 2048, BQ * 128, 1024),
-                  id_dq, kk > 0 ? 1u : 0u);
-        umma_commit(&bars->dq_full);
-        umma_commit(&bars->pds_free);
         umma_commit(&bars->q_empty[st]);
         return true;
       };
       for (int it = 0; ok && it < niter; ++it) {
-        const int st = it % NS, rnd = it / NS;
+        const int st = it % NS, rnd = it / NS, b = it & 1;
         if (!mbar_wait(&bars->q_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-        if (it >= 1 && !mbar_wait(&bars->sdp_free, (it - 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + L::kQ + st * L::kQBytes);
-        const uint32_t do_addr = smem_u32(smem + L::kDO + st * L::kQBytes);
+        const uint32_t q_addr = smem_u32(smem + L::oQ + st * L::kQ);
+        const uint32_t do_addr = smem_u32(smem + L::oDO + st * L::kQ);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * (BKV * 128) + (kk & 3) * 32;   // K / V chunk offset
-          const uint32_t qa = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;    // Q / dO chunk offset
-          umma_ss(tS, sdesc_sw128(k_addr + ka, 16, 1024), sdesc_sw128(q_addr + qa, 16, 1024), id_sdp, kk > 0 ? 1u : 0u);
-          umma_ss(tDP, sdesc_sw128(v_addr + ka, 16, 1024), sdesc_sw128(do_addr + qa, 16, 1024), id_sdp, kk > 0 ? 1u : 0u);
+          const uint32_t ka = (kk >> 2) * (BKV * 128) + (kk & 3) * 32;
+          const uint32_t qa = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          umma_ss(tS(b), sdesc_sw128(k_addr + ka, 16, 1024), sdesc_sw128(q_addr + qa, 16, 1024), id_s, kk > 0);
+          umma_ss(tDP(b), sdesc_sw128(v_addr + ka, 16, 1024), sdesc_sw128(do_addr + qa, 16, 1024), id_s, kk > 0);
         }
-        umma_commit(&bars->sdp_full);
+        umma_commit(&bars->s_full[b]);
         if (it >= 1 && !issue_grads(it - 1)) { ok = false; break; }
       }
       if (ok && niter > 0) issue_grads(niter - 1);
       umma_commit(&bars->mma_final);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ P^T / dS^T
-    const int row = (warp - 4) * 32 + lane;        // key row within the tile
+  } else if (warp >= 4) {
+    const int row = (warp - 4) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
     const int64_t kj = k0 + row;
-    const int64_t kj_end = kj < p.n ? int64_t(se[kj]) : kj;   // rows i in [kj, kj_end) see key kj
-    float* stats = reinterpret_cast<float*>(smem + L::kRowStats);
-    uint8_t* pt = smem + L::kPt;
-    uint8_t* ds = smem + L::kDSt;
-    const int tid = threadIdx.x - 128;
+    const int64_t kj_end = kj < p.n ? int64_t(se[kj]) : kj;   // query rows [kj, kj_end) see key kj
     bool ok = true;
     for (int it = 0; it < niter; ++it) {
-      const int h = g * p.G + it / nqt;
+      const int b = it & 1, st = it % NS;
       const int64_t q0 = int64_t(qt_first + it % nqt) * BQ;
-      // row statistics of this query tile: LSE*log2(e) and D
-      float* st_l = stats + (it & 1) * 2 * BQ;
-      float* st_d = st_l + BQ;
-      if (tid < BQ) {
-        const int64_t q = q0 + tid;
-        const int64_t idx = (int64_t(rb) * p.hq + h) * p.n + q;
-        st_l[tid] = q < p.n ? p.lse[idx] * 1.4426950408889634f : 0.f;
-      } else {
-        const int64_t q = q0 + tid - BQ;
-        const int64_t idx = (int64_t(rb) * p.hq + h) * p.n + q;
-        st_d[tid - BQ] = q < p.n ? p.delta[idx] : 0.f;
+      if (!mbar_wait(&bars->q_full[st], (it / NS) & 1, abort_flag, p.status, p.limit_ns) ||
+          !mbar_wait(&bars->s_full[b], (it >> 1) & 1, abort_flag, p.status, p.limit_ns)) {
+        ok = false;
+        break;
       }
-      mbar_arrive(&bars->stats_ready[it & 1]);
-      if (!mbar_wait(&bars->stats_ready[it & 1], (it >> 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-      if (!mbar_wait(&bars->sdp_full, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
       tc_fence_after();
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      tmem_ld32(tS + lane_off, s0);
-      tmem_ld32(tS + lane_off + 32, s1);
-      tmem_ld32(tDP + lane_off, d0);
-      tmem_ld32(tDP + lane_off + 32, d1);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->sdp_free);
+      const float4* stt = reinterpret_cast<const float4*>(smem + L::oSt + st * L::kSt);
       const bool need_mask = (q0 < k0 + BKV - 1) || (q0 + BQ > seg_end_min) || (q0 + BQ > p.n);
-      uint32_t pw[32], dw[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float pv[2], dsv[2];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tS(b) + lane_off + 32 * half, s);
+        tmem_ld32(tDP(b) + lane_off + 32 * half, dp);
+        tmem_ld_wait();
+        uint32_t pw[16], dw[16];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = 2 * c + e;
-          const uint32_t sbits = col < 32 ? s0[col] : s1[col - 32];
-          const uint32_t dbits = col < 32 ? d0[col] : d1[col - 32];
-          float pr = ex2_approx(__uint_as_float(sbits) * p.scale_log2 - st_l[col]);
+        for (int c = 0; c < 16; ++c) {
+          const float4 sv = stt[16 * half + c];    // {lse2, D} of columns 2c, 2c+1 of this half
+          float pr0 = ex2_approx(__uint_as_float(s[2 * c]) * p.scale_log2 - sv.x);
+          float pr1 = ex2_approx(__uint_as_float(s[2 * c + 1]) * p.scale_log2 - sv.z);
           if (need_mask) {
-            const int64_t q = q0 + col;
-            if (q < kj || q >= kj_end) pr = 0.f;
+            const int64_t qa = q0 + 32 * half + 2 * c;
+            if (qa < kj || qa >= kj_end) pr0 = 0.f;
+            if (qa + 1 < kj || qa + 1 >= kj_end) pr1 = 0.f;
           }
-          pv[e] = pr;
-          dsv[e] = pr * (__uint_as_float(dbits) - st_d[col]);
+          pw[c] = pack_bf16x2(pr0, pr1);
+          dw[c] = pack_bf16x2(pr0 * (__uint_as_float(dp[2 * c]) - sv.y), pr1 * (__uint_as_float(dp[2 * c + 1]) - sv.w));
         }
-        pw[c] = pack_bf16x2(pv[0], pv[1]);
-        dw[c] = pack_bf16x2(dsv[0], dsv[1]);
+        tmem_st16(tS(b) + lane_off + 16 * half, pw);
+        tmem_st16(tDP(b) + lane_off + 16 * half, dw);
       }
-      if (it >= 1 && !mbar_wait(&bars->pds_free, (it - 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-      // row `row` of the [128][64] bf16 tiles: 8 chunks of 16 B, 128B-swizzled
-#pragma unroll
-      for (int c16 = 0; c16 < 8; ++c16) {
-        const uint32_t off = sw128_offset(row, c16 * 16);
-        *reinterpret_cast<uint4*>(pt + off) = make_uint4(pw[4 * c16], pw[4 * c16 + 1], pw[4 * c16 + 2], pw[4 * c16 + 3]);
-        *reinterpret_cast<uint4*>(ds + off) = make_uint4(dw[4 * c16], dw[4 * c16 + 1], dw[4 * c16 + 2], dw[4 * c16 + 3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars->p_ready);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_ready[b]);
     }
-    // ---- epilogue: dK (scaled), dV
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
       const bool valid = kj < p.n;
@@ -338,29 +334,279 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         }
       }
     }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ dQ reduction
-    const int dd = (warp - 8) * 32 + lane;          // head-dim index (TMEM lane)
-    const uint32_t lane_off = uint32_t((warp - 8) * 32) << 16;
-    for (int it = 0; it < niter; ++it) {
-      const int h = g * p.G + it / nqt;
-      const int64_t q0 = int64_t(qt_first + it % nqt) * BQ;
-      if (!mbar_wait(&bars->dq_full, it & 1, abort_flag, p.status, p.limit_ns)) break;
+  }
+
+  if (warp == 1 && lane == 0) mbar_wait(&bars->mma_final, 0, nullptr, nullptr, p.limit_ns);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dkdv
+
+// ============================================================================
+// bwd_dq
+// ============================================================================
+namespace dq {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int NS = 2;
+constexpr int kThreads = 384;
+
+struct Params {
+  const int32_t* segstart;
+  const float2* stats;
+  void* dq;              // [P*b][n][hq][D]
+  int* status;
+  int64_t n, n_pad;
+  int32_t b, P_sel, rank0, hq, G, ntiles;
+  float scale, scale_log2;
+  int32_t g_f32;
+  uint64_t limit_ns;
+};
+
+template <int D>
+struct Layout {
+  static constexpr uint32_t kTile = BM * D * 2;
+  static constexpr uint32_t oQ = 0;
+  static constexpr uint32_t oDO = oQ + kTile;
+  static constexpr uint32_t oK = oDO + kTile;
+  static constexpr uint32_t oV = oK + NS * kTile;
+  static constexpr uint32_t oBar = oV + NS * kTile;
+  static constexpr uint32_t kDynamic = oBar + 256 + 1024;
+};
+
+struct Bars {
+  uint64_t qdo_full;
+  uint64_t k_full[NS], v_full[NS], k_empty[NS], v_empty[NS];
+  uint64_t s_full[2], ds_ready[2];
+  uint64_t dp_full, dp_free, mma_final;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+       const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo, const Params p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::oBar);
+  volatile int* abort_flag = &bars->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int per_tile = p.P_sel * p.b * p.hq;
+  const int tile = p.ntiles - 1 - int(blockIdx.x / per_tile);
+  int rem = int(blockIdx.x % per_tile);
+  const int h = rem % p.hq;
+  rem /= p.hq;
+  const int bb = rem % p.b;
+  const int r = p.rank0 + rem / p.b;
+  const int rb = r * p.b + bb;
+  const int g = h / p.G;
+  const int64_t t0 = int64_t(tile) * BM;
+  const int64_t last_row = (t0 + BM - 1 < p.n - 1) ? (t0 + BM - 1) : (p.n - 1);
+  const int32_t* ss = p.segstart + int64_t(bb) * p.n;
+  const int64_t seg_lo = ss[t0];
+  const int64_t seg_hi = ss[last_row];
+  const int kv_first = int(seg_lo / BN);
+  const int nkv = int(last_row / BN) - kv_first + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->qdo_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->ds_ready[s], 256);
+    }
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->dp_free, 256);
+    mbar_init(&bars->mma_final, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  auto tS = [&](int b) { return tmem + 128u * uint32_t(b); };
+  const uint32_t tDP = tmem + 256, tDQ = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&mk);
+      tma_prefetch_desc(&mv);
+      mbar_arrive_expect_tx(&bars->qdo_full, 2 * L::kTile);
+      for (int dc = 0; dc < D / 64; ++dc) {
+        tma_load_4d(&mq, &bars->qdo_full, smem + L::oQ + dc * BM * 128, dc * 64, h, int(t0), rb);
+        tma_load_4d(&mdo, &bars->qdo_full, smem + L::oDO + dc * BM * 128, dc * 64, h, int(t0), rb);
+      }
+      int issued = 0;
+      for (int it = 0; it < nkv; ++it) {
+        const int st = it % NS, rnd = it / NS;
+        const int k0 = (kv_first + it) * BN;
+        if (rnd > 0 && !mbar_wait(&bars->k_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
+        mbar_arrive_expect_tx(&bars->k_full[st], L::kTile);
+        for (int dc = 0; dc < D / 64; ++dc)
+          tma_load_4d(&mk, &bars->k_full[st], smem + L::oK + st * L::kTile + dc * BN * 128, dc * 64, g, k0, rb);
+        if (rnd > 0 && !mbar_wait(&bars->v_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) {
+          issued = it * 2 + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
+        for (int dc = 0; dc < D / 64; ++dc)
+          tma_load_4d(&mv, &bars->v_full[st], smem + L::oV + st * L::kTile + dc * BN * 128, dc * 64, g, k0, rb);
+        issued = it * 2 + 2;
+      }
+      if (*abort_flag) {
+        mbar_wait(&bars->qdo_full, 0, nullptr, nullptr, p.limit_ns);
+        for (int x = max(0, issued - 2 * NS); x < issued; ++x) {
+          const int it = x / 2, st = it % NS, rnd = it / NS;
+          mbar_wait((x & 1) ? &bars->v_full[st] : &bars->k_full[st], rnd & 1, nullptr, nullptr, p.limit_ns);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16(BM, BN, false, false);
+      const uint32_t id_q = idesc_bf16(BM, D, false, true);
+      const uint32_t q_addr = smem_u32(smem + L::oQ), do_addr = smem_u32(smem + L::oDO);
+      bool ok = mbar_wait(&bars->qdo_full, 0, abort_flag, p.status, p.limit_ns);
       tc_fence_after();
-      uint32_t a0[32], a1[32];
-      tmem_ld32(tDQ + lane_off, a0);
-      tmem_ld32(tDQ + lane_off + 32, a1);
+      auto issue_dq = [&](int jt) -> bool {
+        const int b = jt & 1, st = jt % NS;
+        if (!mbar_wait(&bars->ds_ready[b], (jt >> 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + L::oK + st * L::kTile);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // dS of keys [16kk, 16kk+16): the first 64 keys' bf16 pairs sit in S
+          // columns [0,32), the last 64 keys' in [64,96) (one half per warpgroup).
+          const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
+          umma_ts(tDQ, tS(b) + a_col, sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), id_q,
+                  (jt > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->k_empty[st]);
+        return true;
+      };
+      for (int it = 0; ok && it < nkv; ++it) {
+        const int st = it % NS, rnd = it / NS, b = it & 1;
+        if (!mbar_wait(&bars->k_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + L::oK + st * L::kTile);
+        const uint32_t v_addr = smem_u32(smem + L::oV + st * L::kTile);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          umma_ss(tS(b), sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), id_s, kk > 0);
+        }
+        umma_commit(&bars->s_full[b]);
+        if (it >= 1 && !mbar_wait(&bars->dp_free, (it - 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait(&bars->v_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          umma_ss(tDP, sdesc_sw128(do_addr + off, 16, 1024), sdesc_sw128(v_addr + off, 16, 1024), id_s, kk > 0);
+        }
+        umma_commit(&bars->dp_full);
+        umma_commit(&bars->v_empty[st]);
+        if (it >= 1 && !issue_dq(it - 1)) { ok = false; break; }
+      }
+      if (ok) issue_dq(nkv - 1);
+      umma_commit(&bars->mma_final);
+    }
+  } else if (warp >= 4) {
+    const int wg = (warp - 4) >> 2;                 // column half handled by this warpgroup
+    const int row = ((warp - 4) & 3) * 32 + lane;
+    const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
+    const int64_t i = t0 + row;
+    const bool valid = i < p.n;
+    const int64_t s_i = valid ? ss[i] : seg_hi;
+    float2 st2 = make_float2(0.f, 0.f);
+    if (valid) st2 = p.stats[(int64_t(rb) * p.hq + h) * p.n_pad + i];
+    bool ok = true;
+    for (int it = 0; it < nkv; ++it) {
+      const int b = it & 1;
+      const int64_t k0 = int64_t(kv_first + it) * BN + 64 * wg;
+      if (!mbar_wait(&bars->s_full[b], (it >> 1) & 1, abort_flag, p.status, p.limit_ns) ||
+          !mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s0[32], s1[32], d0[32], d1[32];
+      tmem_ld32(tS(b) + lane_off + 64 * wg, s0);
+      tmem_ld32(tS(b) + lane_off + 64 * wg + 32, s1);
+      tmem_ld32(tDP + lane_off + 64 * wg, d0);
+      tmem_ld32(tDP + lane_off + 64 * wg + 32, d1);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars->dq_free);
-      if (dd < D) {
-        float* base = p.dq_acc + ((int64_t(rb) * p.n + q0) * p.hq + h) * D + dd;
-        const int64_t stride = int64_t(p.hq) * D;
-        const int nvalid = int(p.n - q0 < BQ ? p.n - q0 : BQ);
+      mbar_arrive(&bars->dp_free);
+      const bool need_mask = (k0 + 63 > t0) || (k0 < seg_hi) || !valid || (t0 + BM > p.n);
+      uint32_t w[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (c < nvalid) atomicAdd(base + c * stride, __uint_as_float(a0[c]) * p.scale);
-          if (c + 32 < nvalid) atomicAdd(base + (c + 32) * stride, __uint_as_float(a1[c]) * p.scale);
+      for (int c = 0; c < 32; ++c) {
+        const uint32_t sa = c < 16 ? s0[2 * c] : s1[2 * c - 32];
+        const uint32_t sb = c < 16 ? s0[2 * c + 1] : s1[2 * c - 31];
+        const uint32_t da = c < 16 ? d0[2 * c] : d1[2 * c - 32];
+        const uint32_t db = c < 16 ? d0[2 * c + 1] : d1[2 * c - 31];
+        float pa = ex2_approx(__uint_as_float(sa) * p.scale_log2 - st2.x);
+        float pb = ex2_approx(__uint_as_float(sb) * p.scale_log2 - st2.x);
+        if (need_mask) {
+          const int64_t key = k0 + 2 * c;
+          if (!valid || key < s_i || key > i) pa = 0.f;
+          if (!valid || key + 1 < s_i || key + 1 > i) pb = 0.f;
+        }
+        w[c] = pack_bf16x2(pa * (__uint_as_float(da) - st2.y), pb * (__uint_as_float(db) - st2.y));
+      }
+      tmem_st32(tS(b) + lane_off + 64 * wg, w);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_ready[b]);
+    }
+    if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
+      tc_fence_after();
+      const int64_t orow = (int64_t(rb) * p.n + i) * p.hq + h;
+      for (int c = 64 * wg; c < D; c += 128) {
+        // warpgroup wg stores head-dim columns [64 wg, 64 wg + 64) (D = 64: wg 0 only)
+#pragma unroll
+        for (int c2 = 0; c2 < 64; c2 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tDQ + lane_off + c + c2, o);
+          tmem_ld_wait();
+          if (valid) {
+            if (p.g_f32) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.dq) + orow * D + c + c2);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(o[4 * e]) * p.scale, __uint_as_float(o[4 * e + 1]) * p.scale,
+                                     __uint_as_float(o[4 * e + 2]) * p.scale, __uint_as_float(o[4 * e + 3]) * p.scale);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dq) + orow * D + c + c2);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_uint4(
+                    pack_bf16x2(__uint_as_float(o[8 * e]) * p.scale, __uint_as_float(o[8 * e + 1]) * p.scale),
+                    pack_bf16x2(__uint_as_float(o[8 * e + 2]) * p.scale, __uint_as_float(o[8 * e + 3]) * p.scale),
+                    pack_bf16x2(__uint_as_float(o[8 * e + 4]) * p.scale, __uint_as_float(o[8 * e + 5]) * p.scale),
+                    pack_bf16x2(__uint_as_float(o[8 * e + 6]) * p.scale, __uint_as_float(o[8 * e + 7]) * p.scale));
+            }
+          }
         }
       }
     }
@@ -375,68 +621,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   }
 }
 
-// D_i = dO_i . O_i for every (rank, row, head) of the selected ranks, and the
-// fp32 dQ accumulator rows zeroed.  One warp per (row, head).
-template <int D, bool kOF32>
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const uint16_t* __restrict__ dO,
-                                                      float* __restrict__ delta, float* __restrict__ dq_acc,
-                                                      int64_t rb0, int64_t rows_per_rb, int64_t total_rows, int64_t n,
-                                                      int32_t hq) {
-  const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= total_rows) return;
-  const int64_t rb = rb0 + w / rows_per_rb;
-  const int64_t rem = w % rows_per_rb;      // (token, head) with head fastest
-  const int64_t i = rem / hq;
-  const int64_t h = rem % hq;
-  const int64_t row = rb * rows_per_rb + rem;   // [P*b][n][hq] flattened
-  constexpr int E = D / 32;                      // elements per lane (2 or 4)
-  float acc = 0.f;
-  const uint16_t* dp = dO + row * D + lane * E;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const float dv = __uint_as_float(uint32_t(dp[e]) << 16);
-    float ov;
-    if (kOF32)
-      ov = static_cast<const float*>(o)[row * D + lane * E + e];
-    else
-      ov = __uint_as_float(uint32_t(static_cast<const uint16_t*>(o)[row * D + lane * E + e]) << 16);
-    acc = fmaf(dv, ov, acc);
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) delta[(rb * hq + h) * n + i] = acc;
-#pragma unroll
-  for (int e = 0; e < E; ++e) dq_acc[row * D + lane * E + e] = 0.f;
-}
-
-// dQ (bf16) from the fp32 accumulator of the selected ranks.
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq,
-                                                       int64_t nvec) {
-  for (int64_t v = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec; v += int64_t(gridDim.x) * blockDim.x) {
-    const float4 a = acc[v];
-    dq[v] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
-  }
-}
-
-template <int D>
-cudaError_t launch_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mdo,
-                        const Params& p, int64_t grid, cudaStream_t s) {
-  auto kern = attn_bwd_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::kDynamic);
-  if (e != cudaSuccess) return e;
-  kern<<<unsigned(grid), kThreads, Layout<D>::kDynamic, s>>>(mq, mk, mv, mdo, p);
-  return cudaGetLastError();
-}
+}  // namespace dq
 
 }  // namespace bwd
 
-// Backward workspace: the segment tables (as the forward), then D
-// ([P][b][hq][n] fp32), then, for bf16 gradients, the fp32 dQ accumulator.
-static size_t bwd_ws_delta_off(const uly_shape* s) { return seg_workspace_bytes(s->b, s->n); }
-static size_t bwd_ws_delta_bytes(const uly_shape* s) {
-  return (size_t(s->P) * size_t(s->b) * size_t(s->h_q / s->P) * size_t(s->n) * 4 + 255) & ~size_t(255);
-}
+// Backward workspace: the segment tables (as the forward), then the padded
+// row-statistics table [P][b][hq][n_pad] x {LSE*log2e, D} (n_pad = n rounded
+// up to 64).
+static int64_t bwd_n_pad(int64_t n) { return (n + 63) / 64 * 64; }
+static size_t bwd_ws_stats_off(const uly_shape* s) { return seg_workspace_bytes(s->b, s->n); }
 
 }  // namespace uly
 
@@ -444,9 +637,7 @@ using namespace uly;
 
 extern "C" size_t ulysses_attn_bwd_workspace(const uly_shape* s, uly_dtype g_dtype) {
   if (check_shape(s) != ULY_OK || !dtype_ok(g_dtype)) return 0;
-  size_t need = bwd_ws_delta_off(s) + bwd_ws_delta_bytes(s);
-  if (g_dtype == ULY_BF16) need += size_t(s->b) * size_t(s->n) * size_t(s->h_q) * size_t(s->d) * 4;
-  return need;
+  return bwd_ws_stats_off(s) + size_t(s->b) * size_t(s->h_q) * size_t(bwd_n_pad(s->n)) * 8;
 }
 
 extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* v_head, const void* o_head,
@@ -480,9 +671,10 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
     if (overlaps(outs[a], outsz[a], ws, ws_bytes)) return ULY_ERR_INVALID_ARG;
   }
 
-  CUtensorMap mq, mk, mv, mdo;
-  if (!make_head_map(&mq, q_head, Pb, s.n, hq, s.d, bwd::BQ) || !make_head_map(&mdo, do_head, Pb, s.n, hq, s.d, bwd::BQ) ||
-      !make_head_map(&mk, k_head, Pb, s.n, hkv, s.d, bwd::BKV) || !make_head_map(&mv, v_head, Pb, s.n, hkv, s.d, bwd::BKV))
+  CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128;
+  if (!make_head_map(&mq64, q_head, Pb, s.n, hq, s.d, 64) || !make_head_map(&mdo64, do_head, Pb, s.n, hq, s.d, 64) ||
+      !make_head_map(&mk128, k_head, Pb, s.n, hkv, s.d, 128) || !make_head_map(&mv128, v_head, Pb, s.n, hkv, s.d, 128) ||
+      !make_head_map(&mq128, q_head, Pb, s.n, hq, s.d, 128) || !make_head_map(&mdo128, do_head, Pb, s.n, hq, s.d, 128))
     return ULY_ERR_CUDA;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -490,9 +682,8 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
   const size_t tab = (size_t(s.b) * size_t(s.n) * 4 + 255) & ~size_t(255);
   int32_t* segstart = reinterpret_cast<int32_t*>(wsb + 256);
   int32_t* segend = reinterpret_cast<int32_t*>(wsb + 256 + tab);
-  float* delta = reinterpret_cast<float*>(wsb + bwd_ws_delta_off(&s));
-  float* dq_acc = g_dtype == ULY_F32 ? static_cast<float*>(dq_head)
-                                     : reinterpret_cast<float*>(wsb + bwd_ws_delta_off(&s) + bwd_ws_delta_bytes(&s));
+  float2* stats = reinterpret_cast<float2*>(wsb + bwd_ws_stats_off(&s));
+  const int64_t n_pad = bwd_n_pad(s.n);
 
   cudaError_t e = launch_segments(position_ids, segstart, segend, s.b, s.n, cs);
   if (e != cudaSuccess) return ULY_ERR_CUDA;
@@ -500,57 +691,92 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
   const int64_t P_sel = rank < 0 ? s.P : 1;
   const int64_t rank0 = rank < 0 ? 0 : rank;
   const int64_t rb0 = rank0 * s.b, nrb = P_sel * s.b;
-  const int64_t rows_per_rb = s.n * hq;
-  const int64_t total_rows = nrb * rows_per_rb;
   {
-    const int64_t blocks = (total_rows * 32 + 255) / 256;
+    const int64_t total = nrb * n_pad * hq;
+    const int64_t blocks = (total * 32 + 255) / 256;
     if (blocks > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
     const bool of32 = o_dtype == ULY_F32;
+    const uint16_t* dop = static_cast<const uint16_t*>(do_head);
+    const unsigned nb = unsigned(blocks);
     if (s.d == 128) {
-      if (of32) bwd::bwd_pre_kernel<128, true><<<unsigned(blocks), 256, 0, cs>>>(o_head, static_cast<const uint16_t*>(do_head), delta, dq_acc, rb0, rows_per_rb, total_rows, s.n, int32_t(hq));
-      else bwd::bwd_pre_kernel<128, false><<<unsigned(blocks), 256, 0, cs>>>(o_head, static_cast<const uint16_t*>(do_head), delta, dq_acc, rb0, rows_per_rb, total_rows, s.n, int32_t(hq));
+      if (of32) bwd::bwd_pre_kernel<128, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
+      else bwd::bwd_pre_kernel<128, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
     } else {
-      if (of32) bwd::bwd_pre_kernel<64, true><<<unsigned(blocks), 256, 0, cs>>>(o_head, static_cast<const uint16_t*>(do_head), delta, dq_acc, rb0, rows_per_rb, total_rows, s.n, int32_t(hq));
-      else bwd::bwd_pre_kernel<64, false><<<unsigned(blocks), 256, 0, cs>>>(o_head, static_cast<const uint16_t*>(do_head), delta, dq_acc, rb0, rows_per_rb, total_rows, s.n, int32_t(hq));
+      if (of32) bwd::bwd_pre_kernel<64, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
+      else bwd::bwd_pre_kernel<64, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
     }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return ULY_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
 
-  bwd::Params p;
-  p.segstart = segstart;
-  p.segend = segend;
-  p.lse = lse;
-  p.delta = delta;
-  p.dq_acc = dq_acc;
-  p.dk = dk_head;
-  p.dv = dv_head;
-  p.status = reinterpret_cast<int*>(wsb);
-  p.n = s.n;
-  p.b = int32_t(s.b);
-  p.P_sel = int32_t(P_sel);
-  p.rank0 = int32_t(rank0);
-  p.hq = int32_t(hq);
-  p.hkv = int32_t(hkv);
-  p.G = int32_t(s.h_q / s.h_kv);
-  p.nkt = int32_t((s.n + bwd::BKV - 1) / bwd::BKV);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(float(s.d));
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.g_f32 = g_dtype == ULY_F32;
-  p.limit_ns = 2000000000ull;
-  const int64_t grid = int64_t(p.nkt) * P_sel * s.b * hkv;
-  if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
-  e = s.d == 128 ? bwd::launch_main<128>(mq, mk, mv, mdo, p, grid, cs) : bwd::launch_main<64>(mq, mk, mv, mdo, p, grid, cs);
-  if (e != cudaSuccess) return ULY_ERR_CUDA;
-
-  if (g_dtype == ULY_BF16) {
-    const int64_t first = rb0 * rows_per_rb * s.d, count = total_rows * s.d;
-    const int64_t nvec = count / 4;
-    bwd::bwd_post_kernel<<<1184, 256, 0, cs>>>(reinterpret_cast<const float4*>(dq_acc + first),
-                                               reinterpret_cast<uint2*>(static_cast<uint16_t*>(dq_head) + first), nvec);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return ULY_ERR_CUDA;
+  // ---- dK, dV
+  {
+    bwd::dkdv::Params p;
+    p.segend = segend;
+    p.stats = stats;
+    p.dk = dk_head;
+    p.dv = dv_head;
+    p.status = reinterpret_cast<int*>(wsb);
+    p.n = s.n;
+    p.n_pad = n_pad;
+    p.b = int32_t(s.b);
+    p.P_sel = int32_t(P_sel);
+    p.rank0 = int32_t(rank0);
+    p.hq = int32_t(hq);
+    p.hkv = int32_t(hkv);
+    p.G = int32_t(s.h_q / s.h_kv);
+    p.scale = scale;
+    p.scale_log2 = scale * bwd::kLog2e;
+    p.g_f32 = g_dtype == ULY_F32;
+    p.limit_ns = 2000000000ull;
+    const int64_t grid = (s.n + bwd::dkdv::BKV - 1) / bwd::dkdv::BKV * P_sel * s.b * hkv;
+    if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
+    if (s.d == 128) {
+      auto kern = bwd::dkdv::kernel<128>;
+      const uint32_t sm = bwd::dkdv::Layout<128>::kDynamic;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
+      kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq64, mk128, mv128, mdo64, p);
+    } else {
+      auto kern = bwd::dkdv::kernel<64>;
+      const uint32_t sm = bwd::dkdv::Layout<64>::kDynamic;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
+      kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq64, mk128, mv128, mdo64, p);
+    }
+    if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
+  }
+  // ---- dQ
+  {
+    bwd::dq::Params p;
+    p.segstart = segstart;
+    p.stats = stats;
+    p.dq = dq_head;
+    p.status = reinterpret_cast<int*>(wsb);
+    p.n = s.n;
+    p.n_pad = n_pad;
+    p.b = int32_t(s.b);
+    p.P_sel = int32_t(P_sel);
+    p.rank0 = int32_t(rank0);
+    p.hq = int32_t(hq);
+    p.G = int32_t(s.h_q / s.h_kv);
+    p.ntiles = int32_t((s.n + bwd::dq::BM - 1) / bwd::dq::BM);
+    p.scale = scale;
+    p.scale_log2 = scale * bwd::kLog2e;
+    p.g_f32 = g_dtype == ULY_F32;
+    p.limit_ns = 2000000000ull;
+    const int64_t grid = int64_t(p.ntiles) * P_sel * s.b * hq;
+    if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
+    if (s.d == 128) {
+      auto kern = bwd::dq::kernel<128>;
+      const uint32_t sm = bwd::dq::Layout<128>::kDynamic;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
+      kern<<<unsigned(grid), bwd::dq::kThreads, sm, cs>>>(mq128, mk128, mv128, mdo128, p);
+    } else {
+      auto kern = bwd::dq::kernel<64>;
+      const uint32_t sm = bwd::dq::Layout<64>::kDynamic;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
+      kern<<<unsigned(grid), bwd::dq::kThreads, sm, cs>>>(mq128, mk128, mv128, mdo128, p);
+    }
+    if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
   return ULY_OK;
 }
