@@ -144,6 +144,35 @@ uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* 
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ulysses_attn_fwd_noalloc -- ulysses_attn_fwd without a caller workspace.
+ * The pages have no counterpart for this call; it exists for callers that
+ * cannot allocate device memory themselves: code that runs under a framework
+ * whose allocator owns all device memory and forbids raw allocations on the
+ * hot path, or a service that reserves its memory once at start-up and must
+ * not allocate per request.  Same arguments and results as ulysses_attn_fwd,
+ * minus ws / ws_bytes.
+ *   Scratch: a fixed 4 MiB + 256 B device array inside the library, one per
+ *   GPU that loads the library, held until the process exits.  It covers
+ *   b * n <= 524288 tokens; larger shapes return ULY_ERR_WORKSPACE and
+ *   enqueue nothing.  The call allocates nothing (no cudaMalloc, no
+ *   allocating library routine).
+ *   First call per device: looks up the scratch's device address
+ *   (cudaGetSymbolAddress) with that device current and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: every call on a device uses the same scratch and it keeps the
+ *   last call's contents (nothing in it needs to start at zero).  Calls whose
+ *   work overlaps on the GPU (e.g. on two concurrently running streams) race
+ *   on it and give wrong results: serialise them.
+ *   A pipeline timeout inside the kernel is not reported by this call (there
+ *   is no workspace to read the status word from); use ulysses_attn_fwd
+ *   where that report is needed.
+ */
+uly_status ulysses_attn_fwd_noalloc(const void* q_head, const void* k_head, const void* v_head,
+                                    const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                                    float softmax_scale, void* o_head, uly_dtype o_dtype, float* lse,
+                                    void* stream);
+
+/*
  * ulysses_workspace_status -- synchronizes `stream`, then reads and clears
  * the status word kept at the start of an attention workspace.  *code gets
  * ULY_OK, or ULY_ERR_TIMEOUT when a kernel gave up waiting on one of its own

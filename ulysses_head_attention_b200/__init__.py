@@ -29,7 +29,8 @@ STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED",
                 4: "ULY_ERR_WORKSPACE", 5: "ULY_ERR_TIMEOUT"}
 # Every symbol include/ulysses.h declares.
 EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
-           "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_workspace_status", "ulysses_status_string")
+           "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_fwd_noalloc", "ulysses_workspace_status",
+           "ulysses_status_string")
 
 
 class UlyShape(ctypes.Structure):
@@ -45,7 +46,7 @@ class UlyssesError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m ulysses_head_attention_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python ulysses_head_attention_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
     shp = ctypes.POINTER(UlyShape)
@@ -56,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "ulysses_attn_fwd": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp, sz, vp], i32),
         "ulysses_attn_bwd_workspace": ([shp, i32], sz),
         "ulysses_attn_bwd": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i32, f32, vp, vp, vp, i32, vp, sz, vp], i32),
+        "ulysses_attn_fwd_noalloc": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp], i32),
         "ulysses_workspace_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "ulysses_status_string": ([i32], ctypes.c_char_p),
     }
@@ -156,6 +158,24 @@ def ulysses_attn_fwd(q_head, k_head, v_head, position_ids, o_head, lse, ws, rank
                                 _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
                                 _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
            "ulysses_attn_fwd")
+
+
+def ulysses_attn_fwd_noalloc(q_head, k_head, v_head, position_ids, o_head, lse, rank: int = -1,
+                             softmax_scale: float = 0.0, stream=None) -> None:
+    """ulysses_attn_fwd without a workspace, for callers that cannot allocate
+    device memory: the library's fixed per-GPU scratch (b*n <= 524288 tokens)
+    is used instead.  Calls that overlap on the GPU race on that scratch."""
+    shape = _attn_shape(q_head, k_head)
+    for t, nm in ((k_head, "k_head"), (v_head, "v_head"), (q_head, "q_head")):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{nm} must be bfloat16")
+    if position_ids.dtype != torch.int64:
+        raise TypeError("position_ids must be int64")
+    _check(lib.ulysses_attn_fwd_noalloc(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
+                                        _dev(position_ids, "position_ids"), ctypes.byref(shape), rank,
+                                        softmax_scale, _dev(o_head, "o_head"), _dtype_code(o_head),
+                                        _dev(lse, "lse"), _stream(stream)),
+           "ulysses_attn_fwd_noalloc")
 
 
 def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse, do_head, position_ids, dq_head, dk_head, dv_head, ws,

@@ -1,6 +1,9 @@
 """Build libulysses.so (all CUDA sources under csrc/) for sm_100a, in-tree.
 
-    python -m ulysses_head_attention_b200.build [--force]
+    python ulysses_head_attention_b200/build.py [--force]
+
+(Run by path: importing the package itself loads the library, which may be
+missing or stale before a build.)
 
 Each .cu file is compiled in parallel with nvcc, then linked into one shared
 library next to this file.  Rebuilds only when a source or header is newer

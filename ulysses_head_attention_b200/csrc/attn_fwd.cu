@@ -21,6 +21,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <mutex>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -423,4 +424,63 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
   p.limit_ns = 2000000000ull;
   e = s.d == 128 ? fwd::launch<128>(mq, mk, mv, p, grid, cs) : fwd::launch<64>(mq, mk, mv, p, grid, cs);
   return cuda_status(e);
+}
+
+// ---------------------------------------------------------------------------
+// Forward with library-owned scratch (ulysses_attn_fwd_noalloc).
+//
+// For callers that may not allocate device memory themselves.  The scratch
+// the forward needs (status word + the two per-token segment tables) lives
+// in a fixed file-scope device array instead of a caller workspace.  Host
+// code never hands the array's name to a kernel: in host code that name is
+// only a stand-in, so the device address is looked up with
+// cudaGetSymbolAddress, once per device, the first time this entry point
+// runs on that device.
+// ---------------------------------------------------------------------------
+namespace uly {
+namespace {
+
+constexpr int64_t kNoAllocMaxTokens = int64_t(1) << 19;                     // b * n limit
+constexpr size_t kNoAllocScratchBytes = 256 + 2 * size_t(kNoAllocMaxTokens) * 4;   // 4 MiB + 256 B
+
+static __device__ __align__(256) uint8_t g_fwd_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_fwd_scratch on the current device; set up on first use.
+uly_status scratch_on_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ULY_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fwd_scratch) != cudaSuccess || p == nullptr) return ULY_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return ULY_OK;
+}
+
+}  // namespace
+}  // namespace uly
+
+extern "C" uly_status ulysses_attn_fwd_noalloc(const void* q_head, const void* k_head, const void* v_head,
+                                               const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                                               float softmax_scale, void* o_head, uly_dtype o_dtype, float* lse,
+                                               void* stream) {
+  if (!shape) return ULY_ERR_INVALID_ARG;
+  const uly_status sst = check_shape(shape);
+  if (sst != ULY_OK) return sst;
+  // Sizes beyond the fixed scratch are refused before anything is enqueued.
+  if (ulysses_attn_fwd_workspace(shape) > kNoAllocScratchBytes) return ULY_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const uly_status st = scratch_on_current_device(&scratch);
+  if (st != ULY_OK) return st;
+  // Nothing in the scratch has to start at zero: every call rewrites both
+  // segment tables before reading them, and the status word is only written
+  // (on a pipeline timeout), never read, on this path.
+  return ulysses_attn_fwd(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, o_head, o_dtype, lse,
+                          scratch, kNoAllocScratchBytes, stream);
 }
