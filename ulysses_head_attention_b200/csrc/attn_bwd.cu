@@ -14,14 +14,17 @@
 //   dQ_i  = scale sum_j dS_ij k_j
 //
 // Three kernels, no atomics (results are bitwise reproducible):
-//  * bwd_pre:   D_i and LSE_i*log2(e) per (rank, head, row), written as
-//               interleaved pairs into a padded workspace table.
+//  * bwd_pre:   -LSE_i*log2(e) and -D_i per (rank, head, row), written into
+//               a padded workspace table of 64-row blocks, each holding the
+//               block's 64 values of -LSE*log2e followed by its 64 values of
+//               -D (negated so they feed packed fused multiply-adds).
 //  * bwd_dkdv:  one CTA per (rank, batch row, kv head, 128-key tile),
 //               heaviest first.  Loops over the G query heads of the kv head
 //               and the 64-row query tiles that can see the key tile:
 //                 warp 0      TMA producer (K, V once; Q, dO, row stats ring)
 //                 warp 1      TMEM owner, single-thread MMA issuer
-//                 warps 4..7  thread = key row: P^T, dS^T from S^T, dP^T
+//                 warps 4..11 thread = key row, two warpgroups each taking
+//                             32 of the 64 query columns: P^T, dS^T from S^T, dP^T
 //               S^T = K Q^T and dP^T = V dO^T (M=128 keys, N=64) are double
 //               buffered in TMEM; P^T and dS^T go back to TMEM as bf16 over
 //               them and feed dV += P^T dO, dK += dS^T Q as A-from-TMEM MMAs
@@ -50,10 +53,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ============================================================================
 // bwd_pre: D = rowsum(dO * O) and LSE*log2(e), one warp per (rank, row, head)
 // ============================================================================
-// stats layout: [P*b][hq][n_pad] x float2 {LSE*log2e, D}; rows n..n_pad-1 zero.
+// stats layout: [P*b][hq][n_pad/64] blocks of {64 x -LSE*log2e, 64 x -D};
+// rows n..n_pad-1 are zero.
+__device__ __forceinline__ int64_t stats_index(int64_t rbh, int64_t n_pad, int64_t i) {
+  return (rbh * (n_pad / 64) + i / 64) * 128 + (i & 63);
+}
+
 template <int D, bool kOF32>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const uint16_t* __restrict__ dO,
-                                                      const float* __restrict__ lse, float2* __restrict__ stats,
+                                                      const float* __restrict__ lse, float* __restrict__ stats,
                                                       int64_t rb0, int64_t n, int64_t n_pad, int32_t hq,
                                                       int64_t total) {
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -64,9 +72,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
   const int64_t rem = w % per_rb;
   const int64_t i = rem / hq;          // token (head fastest: consecutive warps read adjacent rows)
   const int64_t h = rem % hq;
-  const int64_t sidx = (rb * hq + h) * n_pad + i;
+  const int64_t sidx = stats_index(rb * hq + h, n_pad, i);
   if (i >= n) {
-    if (lane == 0) stats[sidx] = make_float2(0.f, 0.f);
+    if (lane == 0) {
+      stats[sidx] = 0.f;
+      stats[sidx + 64] = 0.f;
+    }
     return;
   }
   const int64_t row = (rb * n + i) * hq + h;
@@ -82,7 +93,10 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) stats[sidx] = make_float2(lse[(rb * hq + h) * n + i] * kLog2e, acc);
+  if (lane == 0) {
+    stats[sidx] = -lse[(rb * hq + h) * n + i] * kLog2e;
+    stats[sidx + 64] = -acc;
+  }
 }
 
 // ============================================================================
@@ -93,11 +107,11 @@ namespace dkdv {
 constexpr int BKV = 128;
 constexpr int BQ = 64;
 constexpr int NS = 3;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 
 struct Params {
   const int32_t* segend;
-  const float2* stats;   // [P*b][hq][n_pad]
+  const float* stats;    // see stats_index
   void* dk;              // [P*b][n][hkv][D]
   void* dv;
   int* status;
@@ -133,7 +147,7 @@ struct Bars {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
        const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo, const Params p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -167,7 +181,7 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_ready[s], 128);
+      mbar_init(&bars->p_ready[s], 256);
     }
     mbar_init(&bars->mma_final, 1);
     bars->abort_flag = 0;
@@ -205,7 +219,7 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
           tma_load_4d(&mq, &bars->q_full[st], smem + L::oQ + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
           tma_load_4d(&mdo, &bars->q_full[st], smem + L::oDO + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
         }
-        bulk_load(smem + L::oSt + st * L::kSt, p.stats + (int64_t(rb) * p.hq + h) * p.n_pad + q0, L::kSt,
+        bulk_load(smem + L::oSt + st * L::kSt, p.stats + stats_index(int64_t(rb) * p.hq + h, p.n_pad, q0), L::kSt,
                   &bars->q_full[st]);
         issued = it + 1;
       }
@@ -230,9 +244,13 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
         const uint32_t do_addr = smem_u32(smem + L::oDO + st * L::kQ);
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
+          // P^T / dS^T bf16 pairs of query columns [16kk, 16kk+16): the first
+          // 32 columns sit in TMEM columns [0,16), the last 32 in [32,48)
+          // (one block per softmax warpgroup).
+          const uint32_t a_col = kk < 2 ? kk * 8 : 32 + (kk - 2) * 8;
           const uint32_t acc = (jt > 0 || kk > 0) ? 1u : 0u;
-          umma_ts(tDV, tS(b) + kk * 8, sdesc_sw128(do_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
-          umma_ts(tDK, tDP(b) + kk * 8, sdesc_sw128(q_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
+          umma_ts(tDV, tS(b) + a_col, sdesc_sw128(do_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
+          umma_ts(tDK, tDP(b) + a_col, sdesc_sw128(q_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
         }
         umma_commit(&bars->q_empty[st]);
         return true;
@@ -257,45 +275,54 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
       umma_commit(&bars->mma_final);
     }
   } else if (warp >= 4) {
-    const int row = (warp - 4) * 32 + lane;
-    const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
+    const int wg = (warp - 4) >> 2;                  // query columns [32 wg, 32 wg + 32) of each tile
+    const int row = ((warp - 4) & 3) * 32 + lane;    // key row within the tile
+    const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t kj = k0 + row;
     const int64_t kj_end = kj < p.n ? int64_t(se[kj]) : kj;   // query rows [kj, kj_end) see key kj
+    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < niter; ++it) {
       const int b = it & 1, st = it % NS;
-      const int64_t q0 = int64_t(qt_first + it % nqt) * BQ;
+      const int64_t qb = int64_t(qt_first + it % nqt) * BQ + 32 * wg;   // first query column of this warpgroup
       if (!mbar_wait(&bars->q_full[st], (it / NS) & 1, abort_flag, p.status, p.limit_ns) ||
           !mbar_wait(&bars->s_full[b], (it >> 1) & 1, abort_flag, p.status, p.limit_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float4* stt = reinterpret_cast<const float4*>(smem + L::oSt + st * L::kSt);
-      const bool need_mask = (q0 < k0 + BKV - 1) || (q0 + BQ > seg_end_min) || (q0 + BQ > p.n);
+      const float* stt = reinterpret_cast<const float*>(smem + L::oSt + st * L::kSt) + 32 * wg;
+      // visible query columns c of this warpgroup: lo <= c < hi
+      const int64_t lo64 = kj - qb, hi64 = kj_end - qb;
+      const bool need_mask = lo64 > 0 || hi64 < 32;
+      const int lo = int(lo64 < 0 ? 0 : (lo64 > 32 ? 32 : lo64));
+      const int hi = int(hi64 < 0 ? 0 : (hi64 > 32 ? 32 : hi64));
+      uint32_t s[32], dp[32];
+      tmem_ld32(tS(b) + lane_off + 32 * wg, s);
+      tmem_ld32(tDP(b) + lane_off + 32 * wg, dp);
+      tmem_ld_wait();
+      uint32_t pw[16], dw[16];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(tS(b) + lane_off + 32 * half, s);
-        tmem_ld32(tDP(b) + lane_off + 32 * half, dp);
-        tmem_ld_wait();
-        uint32_t pw[16], dw[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float4 sv = stt[16 * half + c];    // {lse2, D} of columns 2c, 2c+1 of this half
-          float pr0 = ex2_approx(__uint_as_float(s[2 * c]) * p.scale_log2 - sv.x);
-          float pr1 = ex2_approx(__uint_as_float(s[2 * c + 1]) * p.scale_log2 - sv.z);
-          if (need_mask) {
-            const int64_t qa = q0 + 32 * half + 2 * c;
-            if (qa < kj || qa >= kj_end) pr0 = 0.f;
-            if (qa + 1 < kj || qa + 1 >= kj_end) pr1 = 0.f;
-          }
-          pw[c] = pack_bf16x2(pr0, pr1);
-          dw[c] = pack_bf16x2(pr0 * (__uint_as_float(dp[2 * c]) - sv.y), pr1 * (__uint_as_float(dp[2 * c + 1]) - sv.w));
+      for (int c = 0; c < 16; ++c) {
+        const float2 nl = *reinterpret_cast<const float2*>(stt + 2 * c);        // -LSE*log2e
+        const float2 nd = *reinterpret_cast<const float2*>(stt + 64 + 2 * c);   // -D
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2,
+                         f2_pack(nl.x, nl.y)), x0, x1);
+        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        if (need_mask) {
+          if (unsigned(2 * c - lo) >= unsigned(hi - lo)) p0 = 0.f;
+          if (unsigned(2 * c + 1 - lo) >= unsigned(hi - lo)) p1 = 0.f;
         }
-        tmem_st16(tS(b) + lane_off + 16 * half, pw);
-        tmem_st16(tDP(b) + lane_off + 16 * half, dw);
+        const uint64_t pp = f2_pack(p0, p1);
+        float d0, d1;
+        f2_unpack(f2_mul(pp, f2_add(f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])),
+                                    f2_pack(nd.x, nd.y))), d0, d1);
+        pw[c] = pack_bf16x2(p0, p1);
+        dw[c] = pack_bf16x2(d0, d1);
       }
+      tmem_st16(tS(b) + lane_off + 32 * wg, pw);
+      tmem_st16(tDP(b) + lane_off + 32 * wg, dw);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->p_ready[b]);
@@ -304,8 +331,8 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
       tc_fence_after();
       const bool valid = kj < p.n;
       const int64_t orow = (int64_t(rb) * p.n + kj) * p.hkv + g;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
+      {
+        const int which = wg;   // warpgroup 0 stores dK, warpgroup 1 stores dV
         const uint32_t base = which == 0 ? tDK : tDV;
         const float mul = which == 0 ? p.scale : 1.f;
         void* out = which == 0 ? p.dk : p.dv;
@@ -359,7 +386,7 @@ constexpr int kThreads = 384;
 
 struct Params {
   const int32_t* segstart;
-  const float2* stats;
+  const float* stats;    // see stats_index
   void* dq;              // [P*b][n][hq][D]
   int* status;
   int64_t n, n_pad;
@@ -391,7 +418,7 @@ struct Bars {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
        const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo, const Params p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -537,12 +564,17 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
     const int64_t i = t0 + row;
     const bool valid = i < p.n;
     const int64_t s_i = valid ? ss[i] : seg_hi;
-    float2 st2 = make_float2(0.f, 0.f);
-    if (valid) st2 = p.stats[(int64_t(rb) * p.hq + h) * p.n_pad + i];
+    float nl = 0.f, nd = 0.f;   // -LSE*log2e, -D of this row
+    if (valid) {
+      const int64_t si = stats_index(int64_t(rb) * p.hq + h, p.n_pad, i);
+      nl = p.stats[si];
+      nd = p.stats[si + 64];
+    }
+    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(nl, nl), nd2 = f2_pack(nd, nd);
     bool ok = true;
     for (int it = 0; it < nkv; ++it) {
       const int b = it & 1;
-      const int64_t k0 = int64_t(kv_first + it) * BN + 64 * wg;
+      const int64_t k0 = int64_t(kv_first + it) * BN + 64 * wg;   // first key column of this warpgroup
       if (!mbar_wait(&bars->s_full[b], (it >> 1) & 1, abort_flag, p.status, p.limit_ns) ||
           !mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
         ok = false;
@@ -557,7 +589,11 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->dp_free);
-      const bool need_mask = (k0 + 63 > t0) || (k0 < seg_hi) || !valid || (t0 + BM > p.n);
+      // visible key columns c of this warpgroup: lo <= c < hi (keys s_i .. i)
+      const int64_t lo64 = s_i - k0, hi64 = valid ? i + 1 - k0 : lo64;
+      const bool need_mask = lo64 > 0 || hi64 < 64;
+      const int lo = int(lo64 < 0 ? 0 : (lo64 > 64 ? 64 : lo64));
+      const int hi = int(hi64 < lo ? lo : (hi64 > 64 ? 64 : hi64));
       uint32_t w[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
@@ -565,14 +601,16 @@ kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorM
         const uint32_t sb = c < 16 ? s0[2 * c + 1] : s1[2 * c - 31];
         const uint32_t da = c < 16 ? d0[2 * c] : d1[2 * c - 32];
         const uint32_t db = c < 16 ? d0[2 * c + 1] : d1[2 * c - 31];
-        float pa = ex2_approx(__uint_as_float(sa) * p.scale_log2 - st2.x);
-        float pb = ex2_approx(__uint_as_float(sb) * p.scale_log2 - st2.x);
+        float xa, xb;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sa), __uint_as_float(sb)), sl2, nl2), xa, xb);
+        float pa = ex2_approx(xa), pb = ex2_approx(xb);
         if (need_mask) {
-          const int64_t key = k0 + 2 * c;
-          if (!valid || key < s_i || key > i) pa = 0.f;
-          if (!valid || key + 1 < s_i || key + 1 > i) pb = 0.f;
+          if (unsigned(2 * c - lo) >= unsigned(hi - lo)) pa = 0.f;
+          if (unsigned(2 * c + 1 - lo) >= unsigned(hi - lo)) pb = 0.f;
         }
-        w[c] = pack_bf16x2(pa * (__uint_as_float(da) - st2.y), pb * (__uint_as_float(db) - st2.y));
+        float ga, gb;
+        f2_unpack(f2_mul(f2_pack(pa, pb), f2_add(f2_pack(__uint_as_float(da), __uint_as_float(db)), nd2)), ga, gb);
+        w[c] = pack_bf16x2(ga, gb);
       }
       tmem_st32(tS(b) + lane_off + 64 * wg, w);
       tmem_st_wait();
@@ -682,7 +720,7 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
   const size_t tab = (size_t(s.b) * size_t(s.n) * 4 + 255) & ~size_t(255);
   int32_t* segstart = reinterpret_cast<int32_t*>(wsb + 256);
   int32_t* segend = reinterpret_cast<int32_t*>(wsb + 256 + tab);
-  float2* stats = reinterpret_cast<float2*>(wsb + bwd_ws_stats_off(&s));
+  float* stats = reinterpret_cast<float*>(wsb + bwd_ws_stats_off(&s));
   const int64_t n_pad = bwd_n_pad(s.n);
 
   cudaError_t e = launch_segments(position_ids, segstart, segend, s.b, s.n, cs);
@@ -732,12 +770,12 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
     const int64_t grid = (s.n + bwd::dkdv::BKV - 1) / bwd::dkdv::BKV * P_sel * s.b * hkv;
     if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
     if (s.d == 128) {
-      auto kern = bwd::dkdv::kernel<128>;
+      auto kern = bwd::dkdv::attn_bwd_dkdv_kernel<128>;
       const uint32_t sm = bwd::dkdv::Layout<128>::kDynamic;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
       kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq64, mk128, mv128, mdo64, p);
     } else {
-      auto kern = bwd::dkdv::kernel<64>;
+      auto kern = bwd::dkdv::attn_bwd_dkdv_kernel<64>;
       const uint32_t sm = bwd::dkdv::Layout<64>::kDynamic;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
       kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq64, mk128, mv128, mdo64, p);
@@ -766,12 +804,12 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
     const int64_t grid = int64_t(p.ntiles) * P_sel * s.b * hq;
     if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
     if (s.d == 128) {
-      auto kern = bwd::dq::kernel<128>;
+      auto kern = bwd::dq::attn_bwd_dq_kernel<128>;
       const uint32_t sm = bwd::dq::Layout<128>::kDynamic;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
       kern<<<unsigned(grid), bwd::dq::kThreads, sm, cs>>>(mq128, mk128, mv128, mdo128, p);
     } else {
-      auto kern = bwd::dq::kernel<64>;
+      auto kern = bwd::dq::attn_bwd_dq_kernel<64>;
       const uint32_t sm = bwd::dq::Layout<64>::kDynamic;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
       kern<<<unsigned(grid), bwd::dq::kThreads, sm, cs>>>(mq128, mk128, mv128, mdo128, p);

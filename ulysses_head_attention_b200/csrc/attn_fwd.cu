@@ -35,6 +35,7 @@ constexpr int BN = 128;        // keys per tile
 constexpr int NS = 2;          // K/V stages
 constexpr int kThreads = 256;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
+constexpr int kMufuPairs = 48;              // of the 64 column pairs per row, the rest use exp2_poly
 
 struct Params {
   const int32_t* segstart;   // [b][n]
@@ -208,7 +209,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     const int64_t i = t0 + row;
     const bool valid = i < p.n;
     const int64_t s_i = valid ? ss[i] : seg_hi;
-    float m_used = -INFINITY, l = 0.f;
+    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+    float m_used = -INFINITY, l = 0.f;   // running max (log2 units, scaled) and row sum
     bool ok = true;
     for (int it = 0; it < nkv; ++it) {
       const int sb = it & 1;
@@ -221,25 +223,35 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       tmem_ld32((tS0 + 128u * sb) + lane_off + 64, a2);
       tmem_ld32((tS0 + 128u * sb) + lane_off + 96, a3);
       tmem_ld_wait();
-      float x[BN];
+      float x[BN];   // raw scores q.k
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(a0[c]) * p.scale_log2;
-        x[32 + c] = __uint_as_float(a1[c]) * p.scale_log2;
-        x[64 + c] = __uint_as_float(a2[c]) * p.scale_log2;
-        x[96 + c] = __uint_as_float(a3[c]) * p.scale_log2;
+        x[c] = __uint_as_float(a0[c]);
+        x[32 + c] = __uint_as_float(a1[c]);
+        x[64 + c] = __uint_as_float(a2[c]);
+        x[96 + c] = __uint_as_float(a3[c]);
       }
-      const bool need_mask = (k0 + BN - 1 > t0) || (k0 < seg_hi);
-      if (need_mask) {
+      // visible key columns: lo <= c < hi (keys s_i .. i)
+      const int64_t lo64 = s_i - k0, hi64 = valid ? i + 1 - k0 : lo64;
+      if (lo64 > 0 || hi64 < BN) {
+        const int lo = int(lo64 < 0 ? 0 : (lo64 > BN ? BN : lo64));
+        const int hi = int(hi64 < lo ? lo : (hi64 > BN ? BN : hi64));
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int64_t key = k0 + c;
-          if (key < s_i || key > i) x[c] = -INFINITY;
-        }
+        for (int c = 0; c < BN; ++c)
+          if (unsigned(c - lo) >= unsigned(hi - lo)) x[c] = -INFINITY;
       }
-      float mx = x[0];
+      // row max of the raw scores (scale > 0), four independent chains
+      float m0 = x[0], m1 = x[1], m2 = x[2], m3 = x[3];
 #pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, x[c]);
+      for (int c = 4; c + 8 <= BN; c += 8) {
+        m0 = fmax3(m0, x[c], x[c + 1]);
+        m1 = fmax3(m1, x[c + 2], x[c + 3]);
+        m2 = fmax3(m2, x[c + 4], x[c + 5]);
+        m3 = fmax3(m3, x[c + 6], x[c + 7]);
+      }
+      m0 = fmax3(m0, x[BN - 4], x[BN - 3]);
+      m1 = fmax3(m1, x[BN - 2], x[BN - 1]);
+      const float mx = fmaxf(fmax3(m0, m1, m2), m3) * p.scale_log2;
       const float m_new = fmaxf(m_used, mx);
       const bool grow = m_new > m_used + kRescaleThreshold;   // also true when m_used is -inf and m_new finite
       float factor = 1.f;
@@ -267,15 +279,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         }
       }
       const float ms = (m_used == -INFINITY) ? 0.f : m_used;
+      const uint64_t nms2 = f2_pack(-ms, -ms);
+      // P = 2^(scale*x - m): column pairs [0, kMufuPairs) on the MUFU unit,
+      // the rest on the FMA pipe (exp2_poly), so both pipes share the load.
       uint32_t pk0[32], pk1[32];
+      uint64_t sum0 = f2_pack(0.f, 0.f), sum1 = sum0, sum2 = sum0, sum3 = sum0;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float e0 = ex2_approx(x[2 * c] - ms), e1 = ex2_approx(x[2 * c + 1] - ms);
-        const float e2 = ex2_approx(x[64 + 2 * c] - ms), e3 = ex2_approx(x[64 + 2 * c + 1] - ms);
-        l += (e0 + e1) + (e2 + e3);
-        pk0[c] = pack_bf16x2(e0, e1);
-        pk1[c] = pack_bf16x2(e2, e3);
+      for (int c2 = 0; c2 < BN / 2; ++c2) {
+        float e0, e1;
+        f2_unpack(f2_fma(f2_pack(x[2 * c2], x[2 * c2 + 1]), sl2, nms2), e0, e1);
+        if (c2 < kMufuPairs) {
+          e0 = ex2_approx(e0);
+          e1 = ex2_approx(e1);
+        } else {
+          e0 = exp2_poly(e0);
+          e1 = exp2_poly(e1);
+        }
+        const uint64_t ee = f2_pack(e0, e1);
+        if ((c2 & 3) == 0) sum0 = f2_add(sum0, ee);
+        else if ((c2 & 3) == 1) sum1 = f2_add(sum1, ee);
+        else if ((c2 & 3) == 2) sum2 = f2_add(sum2, ee);
+        else sum3 = f2_add(sum3, ee);
+        if (c2 < 32) pk0[c2] = pack_bf16x2(e0, e1);
+        else pk1[c2 - 32] = pack_bf16x2(e0, e1);
       }
+      float sa, sb2;
+      f2_unpack(f2_add(f2_add(sum0, sum1), f2_add(sum2, sum3)), sa, sb2);
+      l += sa + sb2;
       tmem_st32((tS0 + 128u * sb) + lane_off + 0, pk0);
       tmem_st32((tS0 + 128u * sb) + lane_off + 32, pk1);
       tmem_st_wait();

@@ -259,6 +259,57 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// ----------------------------------------------------------------------------
+// Packed fp32 pairs (Blackwell f32x2 FMA-pipe instructions)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA/ALU pipes, for x <= 126 (arguments here are <= 8).
+// Range reduction 2^x = 2^n * 2^f with n = round(x), f in [-1/2, 1/2]: adding
+// 1.5 * 2^23 rounds x to an integer held in the low mantissa bits, and those
+// bits shifted into the exponent field scale p(f) by 2^n.  p is the degree-3
+// polynomial minimising the maximum relative error of 2^f on [-1/2, 1/2]
+// (Lawson's iteratively reweighted least squares; fit_exp2_poly.py next to
+// this file derives the coefficients): max relative error 7.5e-5 in fp32.
+// x is clamped at -125, so anything smaller returns about 2^-125 instead of 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float q = fmaf(0.05517167f, f, 0.24261114f);
+  q = fmaf(q, f, 0.69326097f);
+  q = fmaf(q, f, 0.99992806f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ int elect_one_lane() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace uly
