@@ -32,7 +32,8 @@
 //               TMEM: dK [0,128) dV [128,256) S^T_b [256+128b, +64)
 //               dP^T_b [320+128b, +64).
 //  * bwd_dq:    one CTA per (rank, batch row, query head, 128-row tile),
-//               heaviest first; the forward's structure.  S = Q K^T into a
+//               heaviest first; the forward's structure (K and V rings fed
+//               by separate producer warps).  S = Q K^T into a
 //               double-buffered TMEM tile, dP = dO V^T, two softmax
 //               warpgroups (64 columns each) turn them into dS (bf16, over S)
 //               and dQ += dS K accumulates in TMEM.
@@ -473,38 +474,37 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
   auto tS = [&](int b) { return tmem + 128u * uint32_t(b); };
   const uint32_t tDP = tmem + 256, tDQ = tmem + 384;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 2) {
+    // producers: warp 0 loads Q, dO and the K ring, warp 2 the V ring, so a
+    // K load never waits behind a V stage that is still being read
     if (lane == 0) {
-      tma_prefetch_desc(&mk);
-      tma_prefetch_desc(&mv);
-      mbar_arrive_expect_tx(&bars->qdo_full, 2 * L::kTile);
-      for (int dc = 0; dc < D / 64; ++dc) {
-        tma_load_4d(&mq, &bars->qdo_full, smem + L::oQ + dc * BM * 128, dc * 64, h, int(t0), rb);
-        tma_load_4d(&mdo, &bars->qdo_full, smem + L::oDO + dc * BM * 128, dc * 64, h, int(t0), rb);
+      const bool is_k = warp == 0;
+      const CUtensorMap* map = is_k ? &mk : &mv;
+      uint64_t* full = is_k ? bars->k_full : bars->v_full;
+      uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
+      const uint32_t base = is_k ? L::oK : L::oV;
+      tma_prefetch_desc(map);
+      if (is_k) {
+        mbar_arrive_expect_tx(&bars->qdo_full, 2 * L::kTile);
+        for (int dc = 0; dc < D / 64; ++dc) {
+          tma_load_4d(&mq, &bars->qdo_full, smem + L::oQ + dc * BM * 128, dc * 64, h, int(t0), rb);
+          tma_load_4d(&mdo, &bars->qdo_full, smem + L::oDO + dc * BM * 128, dc * 64, h, int(t0), rb);
+        }
       }
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
         const int st = it % NS, rnd = it / NS;
         const int k0 = (kv_first + it) * BN;
-        if (rnd > 0 && !mbar_wait(&bars->k_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
-        mbar_arrive_expect_tx(&bars->k_full[st], L::kTile);
+        if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
+        mbar_arrive_expect_tx(&full[st], L::kTile);
         for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(&mk, &bars->k_full[st], smem + L::oK + st * L::kTile + dc * BN * 128, dc * 64, g, k0, rb);
-        if (rnd > 0 && !mbar_wait(&bars->v_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) {
-          issued = it * 2 + 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&bars->v_full[st], L::kTile);
-        for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(&mv, &bars->v_full[st], smem + L::oV + st * L::kTile + dc * BN * 128, dc * 64, g, k0, rb);
-        issued = it * 2 + 2;
+          tma_load_4d(map, &full[st], smem + base + st * L::kTile + dc * BN * 128, dc * 64, g, k0, rb);
+        issued = it + 1;
       }
       if (*abort_flag) {
-        mbar_wait(&bars->qdo_full, 0, nullptr, nullptr, p.limit_ns);
-        for (int x = max(0, issued - 2 * NS); x < issued; ++x) {
-          const int it = x / 2, st = it % NS, rnd = it / NS;
-          mbar_wait((x & 1) ? &bars->v_full[st] : &bars->k_full[st], rnd & 1, nullptr, nullptr, p.limit_ns);
-        }
+        if (is_k) mbar_wait(&bars->qdo_full, 0, nullptr, nullptr, p.limit_ns);
+        for (int x = max(0, issued - NS); x < issued; ++x)
+          mbar_wait(&full[x % NS], (x / NS) & 1, nullptr, nullptr, p.limit_ns);
       }
     }
   } else if (warp == 1) {

@@ -7,17 +7,29 @@
 // guide "Sequence parallelism", "ALST/Ulysses SP backend configuration":
 // samples packed into one row must not attend to one another.
 //
-// Kernel structure (one CTA per (rank, batch row, query head, 128-row tile),
-// heaviest tiles first):
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
-//   warp 1      TMEM owner and single-thread tcgen05 MMA issuer
-//   warps 4..7  softmax: thread = query row; reads S from TMEM, writes
-//               P (bf16) back over S for the PV MMA, rescales O lazily
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D).
-// Keys a tile cannot see are never loaded: the key-tile range starts at the
-// tile holding the sample start of the tile's first row and ends at the
-// diagonal tile; per-element masks run only on tiles that straddle the
-// diagonal or a sample start.
+// Kernel structure: one CTA per (rank, batch row, query head, pair of
+// adjacent 128-row query tiles), heaviest pairs first.  Both query tiles
+// share every K/V tile the CTA loads, which halves the L2 -> shared-memory
+// traffic per flop (every CTA streams its head's whole visible K/V prefix).
+//   warp 0       TMA producer: Q tiles once, then K tiles into a 2-stage ring
+//   warp 2       TMA producer: V tiles into a 2-stage ring
+//   warp 1       TMEM owner and single-thread tcgen05 MMA issuer
+//   warps 4..7   softmax of query tile 0, thread = query row
+//   warps 8..11  softmax of query tile 1
+// Per key tile j the MMAs are issued as PV_0(j-1), S_0(j), PV_1(j-1), S_1(j)
+// (S_q = Q_q K^T, PV_q: O_q += P_q V), each pair as one burst after all of
+// its waits (a wait by the issuing thread stalls MMA issue for a few hundred
+// cycles, so waits are batched).  While one warpgroup turns S into P the
+// tensor core works on the other tile, and S_q(j) completing implies
+// PV_q(j-1) completed, so the lazy O rescale needs no extra wait.  The
+// softmax writes P (bf16) back over S; PV reads it as the A operand from TMEM.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+// The producer/MMA warpgroup hands registers to the two softmax warpgroups
+// (setmaxnreg): 72 + 2 x 216 = 3 x 168 registers per thread slot.
+// Keys a tile cannot see are never loaded: a tile's key range starts at the
+// key tile holding the sample start of its first row and ends at its
+// diagonal; per-element masks run only on tiles that straddle the diagonal
+// or a sample start.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -33,9 +45,9 @@ namespace fwd {
 constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // keys per tile
 constexpr int NS = 2;          // K/V stages
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
-constexpr int kMufuPairs = 48;              // of the 64 column pairs per row, the rest use exp2_poly
+constexpr int kMufuPairs = 40;              // of the 64 column pairs per row, the rest use exp2_poly
 
 struct Params {
   const int32_t* segstart;   // [b][n]
@@ -43,7 +55,7 @@ struct Params {
   void* o;                   // [P][b][n][hq][D]
   int* status;
   int64_t n;
-  int32_t b, P_sel, rank0, hq, G, ntiles;
+  int32_t b, P_sel, rank0, hq, G, ntiles, npairs;
   float scale_log2;
   int32_t o_f32;
   uint64_t limit_ns;
@@ -52,8 +64,8 @@ struct Params {
 template <int D>
 struct Layout {
   static constexpr uint32_t kTileBytes = BM * D * 2;   // a Q, K or V tile
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTileBytes;
+  static constexpr uint32_t kQ = 0;                     // two query tiles
+  static constexpr uint32_t kK = kQ + 2 * kTileBytes;
   static constexpr uint32_t kV = kK + NS * kTileBytes;
   static constexpr uint32_t kBar = kV + NS * kTileBytes;
   static constexpr uint32_t kBytes = kBar + 256;
@@ -64,10 +76,33 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[NS], v_full[NS], k_empty[NS], v_empty[NS];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_done, o_final;
+  uint64_t o_final[2];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+__device__ __forceinline__ void regs_dec72() { asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory"); }
+__device__ __forceinline__ void regs_inc216() { asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory"); }
+
+// Key-tile range [first, last] of query tile `tile`, and the largest sample
+// start among its rows.
+struct TileRange {
+  int first, last;
+  int64_t t0, seg_hi;
+  bool valid;
+};
+
+__device__ __forceinline__ TileRange tile_range(const int32_t* ss, int64_t n, int tile, int ntiles) {
+  TileRange tr;
+  tr.valid = tile < ntiles;
+  const int tl = tr.valid ? tile : ntiles - 1;
+  tr.t0 = int64_t(tl) * BM;
+  const int64_t last_row = (tr.t0 + BM - 1 < n - 1) ? (tr.t0 + BM - 1) : (n - 1);
+  tr.first = int(int64_t(ss[tr.t0]) / BN);
+  tr.last = int(last_row / BN);
+  tr.seg_hi = ss[last_row];
+  return tr;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -80,23 +115,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item: heaviest (last) query tiles first
-  const int per_tile = p.P_sel * p.b * p.hq;
-  const int tile = p.ntiles - 1 - int(blockIdx.x / per_tile);
-  int rem = int(blockIdx.x % per_tile);
+  // ---- work item: heaviest (last) pairs of query tiles first
+  const int per_pair = p.P_sel * p.b * p.hq;
+  const int pair = p.npairs - 1 - int(blockIdx.x / per_pair);
+  int rem = int(blockIdx.x % per_pair);
   const int j = rem % p.hq;
   rem /= p.hq;
   const int bb = rem % p.b;
   const int r = p.rank0 + rem / p.b;
   const int rb = r * p.b + bb;
   const int g = j / p.G;
-  const int64_t t0 = int64_t(tile) * BM;
-  const int64_t last_row = (t0 + BM - 1 < p.n - 1) ? (t0 + BM - 1) : (p.n - 1);
   const int32_t* ss = p.segstart + int64_t(bb) * p.n;
-  const int64_t seg_lo = ss[t0];
-  const int64_t seg_hi = ss[last_row];
-  const int kv_first = int(seg_lo / BN);
-  const int nkv = int(last_row / BN) - kv_first + 1;
+  const TileRange tr0 = tile_range(ss, p.n, 2 * pair, p.ntiles);
+  const TileRange tr1 = tile_range(ss, p.n, 2 * pair + 1, p.ntiles);
+  const int j_lo = tr0.first;                               // tile 1 starts no earlier
+  const int j_hi = tr1.valid ? tr1.last : tr0.last;
+  const int nkv = j_hi - j_lo + 1;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -109,9 +143,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->o_final[s], 1);
     }
-    mbar_init(&bars->o_done, 1);
-    mbar_init(&bars->o_final, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -123,131 +156,149 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tS0 = tmem;   // S buffer sb lives at tS0 + 128 * sb
-  const uint32_t tO = tmem + 256;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&mq);
-      tma_prefetch_desc(&mk);
-      tma_prefetch_desc(&mv);
-      mbar_arrive_expect_tx(&bars->q_full, L::kTileBytes);
-      for (int dc = 0; dc < D / 64; ++dc)
-        tma_load_4d(&mq, &bars->q_full, smem + L::kQ + dc * BM * 128, dc * 64, j, int(t0), rb);
+  if (warp < 4) {
+    regs_dec72();
+    if ((warp == 0 || warp == 2) && lane == 0) {
+      // ---------------------------------------------------------- producers
+      const bool is_k = warp == 0;
+      const CUtensorMap* map = is_k ? &mk : &mv;
+      uint64_t* full = is_k ? bars->k_full : bars->v_full;
+      uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
+      const uint32_t base = is_k ? L::kK : L::kV;
+      tma_prefetch_desc(map);
+      if (is_k) {
+        tma_prefetch_desc(&mq);
+        mbar_arrive_expect_tx(&bars->q_full, (tr1.valid ? 2 : 1) * L::kTileBytes);
+        for (int q = 0; q < (tr1.valid ? 2 : 1); ++q)
+          for (int dc = 0; dc < D / 64; ++dc)
+            tma_load_4d(&mq, &bars->q_full, smem + L::kQ + q * L::kTileBytes + dc * BM * 128, dc * 64, j,
+                        int((q ? tr1 : tr0).t0), rb);
+      }
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
         const int st = it % NS, rnd = it / NS;
-        const int k0 = (kv_first + it) * BN;
-        if (rnd > 0 && !mbar_wait(&bars->k_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
-        mbar_arrive_expect_tx(&bars->k_full[st], L::kTileBytes);
+        const int k0 = (j_lo + it) * BN;
+        if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
+        mbar_arrive_expect_tx(&full[st], L::kTileBytes);
         for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(&mk, &bars->k_full[st], smem + L::kK + st * L::kTileBytes + dc * BN * 128, dc * 64, g, k0, rb);
-        if (rnd > 0 && !mbar_wait(&bars->v_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) {
-          issued = it * 2 + 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&bars->v_full[st], L::kTileBytes);
-        for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(&mv, &bars->v_full[st], smem + L::kV + st * L::kTileBytes + dc * BN * 128, dc * 64, g, k0, rb);
-        issued = it * 2 + 2;
+          tma_load_4d(map, &full[st], smem + base + st * L::kTileBytes + dc * BN * 128, dc * 64, g, k0, rb);
+        issued = it + 1;
       }
       // Error path only: let every copy this thread started land before exit.
       if (*abort_flag) {
-        mbar_wait(&bars->q_full, 0, nullptr, nullptr, p.limit_ns);
-        for (int x = max(0, issued - 2 * NS); x < issued; ++x) {
-          const int it = x / 2, st = it % NS, rnd = it / NS;
-          mbar_wait((x & 1) ? &bars->v_full[st] : &bars->k_full[st], rnd & 1, nullptr, nullptr, p.limit_ns);
-        }
+        if (is_k) mbar_wait(&bars->q_full, 0, nullptr, nullptr, p.limit_ns);
+        for (int x = max(0, issued - NS); x < issued; ++x)
+          mbar_wait(&full[x % NS], (x / NS) & 1, nullptr, nullptr, p.limit_ns);
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       const uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
       const uint32_t idesc_o = idesc_bf16(BM, D, false, true);
-      const uint32_t q_addr = smem_u32(smem + L::kQ);
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, p.status, p.limit_ns);
-      tc_fence_after();
-      auto issue_pv = [&](int jt) -> bool {
-        const int sb = jt & 1, st = jt % NS, rnd = jt / NS;
-        if (!mbar_wait(&bars->p_full[sb], (jt >> 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
-        if (!mbar_wait(&bars->v_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + L::kV + st * L::kTileBytes);
+      int npv[2] = {0, 0};
+      for (int it = 0; ok && it <= nkv; ++it) {
+        const int jj = j_lo + it;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(v_addr + kk * 2048, BN * 128, 1024);
-          umma_ts(tO, (tS0 + 128u * sb) + kk * 8, bdesc, idesc_o, (jt > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&bars->o_done);
-        umma_commit(&bars->v_empty[st]);
-        return true;
-      };
-      for (int it = 0; ok && it < nkv; ++it) {
-        const int st = it % NS, rnd = it / NS, sb = it & 1;
-        if (!mbar_wait(&bars->k_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + L::kK + st * L::kTileBytes);
+        for (int q = 0; q < 2; ++q) {
+          const TileRange& tr = q ? tr1 : tr0;
+          const uint32_t tS = tmem + 128u * q, tO = tmem + 256u + 128u * q;
+          const bool do_pv = it >= 1 && tr.valid && jj - 1 >= tr.first && jj - 1 <= tr.last;
+          const bool do_s = it < nkv && tr.valid && jj >= tr.first && jj <= tr.last;
+          // All waits of this step first, then its MMAs in one burst: a wait by
+          // the issuing thread stalls MMA issue for a few hundred cycles, so
+          // the stage waits ride along with tile 0's P wait.
+          if (do_pv && !mbar_wait(&bars->p_full[q], npv[q] & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+          if (q == 0) {
+            if (it >= 1 && !mbar_wait(&bars->v_full[(it - 1) % NS], ((it - 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+              ok = false;
+              break;
+            }
+            if (it < nkv && !mbar_wait(&bars->k_full[it % NS], (it / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+              ok = false;
+              break;
+            }
+          }
+          tc_fence_after();
+          // PV_q of the previous key tile (its P sits in S_q: must precede S_q(jj))
+          // Descriptors: base once, then + compile-time offsets (16-byte units)
+          // so the issue loop is a few instructions per MMA.
+          if (do_pv) {
+            const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::kV + ((it - 1) % NS) * L::kTileBytes), BN * 128, 1024);
+            umma_ts(tO, tS, v_desc, idesc_o, npv[q] > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          umma_ss((tS0 + 128u * sb), sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc_s,
-                  kk > 0 ? 1u : 0u);
+            for (int kk = 1; kk < BN / 16; ++kk)
+              umma_ts(tO, tS + kk * 8, v_desc + uint64_t(kk * 2048 / 16), idesc_o, 1u);
+            ++npv[q];
+          }
+          if (do_s) {
+            const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::kQ + q * L::kTileBytes), 16, 1024);
+            const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::kK + (it % NS) * L::kTileBytes), 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = uint64_t(((kk >> 2) * (BM * 128) + (kk & 3) * 32) / 16);
+              umma_ss(tS, q_desc + off, k_desc + off, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars->s_full[q]);
+          }
         }
-        umma_commit(&bars->s_full[sb]);
-        umma_commit(&bars->k_empty[st]);
-        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
+        if (!ok) break;
+        if (it >= 1) umma_commit(&bars->v_empty[(it - 1) % NS]);
+        if (it < nkv) umma_commit(&bars->k_empty[it % NS]);
       }
-      if (ok) issue_pv(nkv - 1);
-      umma_commit(&bars->o_final);
+      umma_commit(&bars->o_final[0]);
+      umma_commit(&bars->o_final[1]);
     }
-  } else if (warp >= 4) {
+  } else {
+    regs_inc216();
     // ------------------------------------------------------------ softmax
-    const int row = (warp - 4) * 32 + lane;
-    const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
-    const int64_t i = t0 + row;
-    const bool valid = i < p.n;
-    const int64_t s_i = valid ? ss[i] : seg_hi;
+    const int q = (warp - 4) >> 2;                     // query tile of this warpgroup
+    const TileRange tr = q ? tr1 : tr0;
+    const uint32_t tS = tmem + 128u * q, tO = tmem + 256u + 128u * q;
+    const int row = ((warp - 4) & 3) * 32 + lane;
+    const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
+    const int64_t i = tr.t0 + row;
+    const bool valid = tr.valid && i < p.n;
+    const int64_t s_i = valid ? ss[i] : tr.seg_hi;
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     float m_used = -INFINITY, l = 0.f;   // running max (log2 units, scaled) and row sum
     bool ok = true;
-    for (int it = 0; it < nkv; ++it) {
-      const int sb = it & 1;
-      const int64_t k0 = int64_t(kv_first + it) * BN;
-      if (!mbar_wait(&bars->s_full[sb], (it >> 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+    const int ntile = tr.valid ? tr.last - tr.first + 1 : 0;
+    for (int c = 0; c < ntile; ++c) {
+      const int64_t k0 = int64_t(tr.first + c) * BN;
+      if (!mbar_wait(&bars->s_full[q], c & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
       tc_fence_after();
       uint32_t a0[32], a1[32], a2[32], a3[32];
-      tmem_ld32((tS0 + 128u * sb) + lane_off + 0, a0);
-      tmem_ld32((tS0 + 128u * sb) + lane_off + 32, a1);
-      tmem_ld32((tS0 + 128u * sb) + lane_off + 64, a2);
-      tmem_ld32((tS0 + 128u * sb) + lane_off + 96, a3);
+      tmem_ld32(tS + lane_off + 0, a0);
+      tmem_ld32(tS + lane_off + 32, a1);
+      tmem_ld32(tS + lane_off + 64, a2);
+      tmem_ld32(tS + lane_off + 96, a3);
       tmem_ld_wait();
       float x[BN];   // raw scores q.k
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(a0[c]);
-        x[32 + c] = __uint_as_float(a1[c]);
-        x[64 + c] = __uint_as_float(a2[c]);
-        x[96 + c] = __uint_as_float(a3[c]);
+      for (int e = 0; e < 32; ++e) {
+        x[e] = __uint_as_float(a0[e]);
+        x[32 + e] = __uint_as_float(a1[e]);
+        x[64 + e] = __uint_as_float(a2[e]);
+        x[96 + e] = __uint_as_float(a3[e]);
       }
-      // visible key columns: lo <= c < hi (keys s_i .. i)
+      // visible key columns: lo <= col < hi (keys s_i .. i)
       const int64_t lo64 = s_i - k0, hi64 = valid ? i + 1 - k0 : lo64;
       if (lo64 > 0 || hi64 < BN) {
         const int lo = int(lo64 < 0 ? 0 : (lo64 > BN ? BN : lo64));
         const int hi = int(hi64 < lo ? lo : (hi64 > BN ? BN : hi64));
 #pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (unsigned(c - lo) >= unsigned(hi - lo)) x[c] = -INFINITY;
+        for (int e = 0; e < BN; ++e)
+          if (unsigned(e - lo) >= unsigned(hi - lo)) x[e] = -INFINITY;
       }
       // row max of the raw scores (scale > 0), four independent chains
       float m0 = x[0], m1 = x[1], m2 = x[2], m3 = x[3];
 #pragma unroll
-      for (int c = 4; c + 8 <= BN; c += 8) {
-        m0 = fmax3(m0, x[c], x[c + 1]);
-        m1 = fmax3(m1, x[c + 2], x[c + 3]);
-        m2 = fmax3(m2, x[c + 4], x[c + 5]);
-        m3 = fmax3(m3, x[c + 6], x[c + 7]);
+      for (int e = 4; e + 8 <= BN; e += 8) {
+        m0 = fmax3(m0, x[e], x[e + 1]);
+        m1 = fmax3(m1, x[e + 2], x[e + 3]);
+        m2 = fmax3(m2, x[e + 4], x[e + 5]);
+        m3 = fmax3(m3, x[e + 6], x[e + 7]);
       }
       m0 = fmax3(m0, x[BN - 4], x[BN - 3]);
       m1 = fmax3(m1, x[BN - 2], x[BN - 1]);
@@ -259,61 +310,60 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         factor = ex2_approx(m_used - m_new);   // 0 when m_used is -inf
         l *= factor;
       }
-      // O already holds contributions only if an earlier tile had a finite max.
+      // O_q holds contributions only if an earlier tile had a finite max; all
+      // of them are complete (S_q of this tile was issued after them).
       const bool rescale_o = grow && m_used != -INFINITY;
       if (grow) m_used = m_new;
       if (__any_sync(0xffffffffu, rescale_o)) {
-        if (!mbar_wait(&bars->o_done, (it - 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; }
-        __syncwarp();
-        if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-        tc_fence_after();
         const float f = rescale_o ? factor : 1.f;
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        for (int e0 = 0; e0 < D; e0 += 32) {
           uint32_t o[32];
-          tmem_ld32(tO + lane_off + c, o);
+          tmem_ld32(tO + lane_off + e0, o);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-          tmem_st32(tO + lane_off + c, o);
+          tmem_st32(tO + lane_off + e0, o);
         }
       }
       const float ms = (m_used == -INFINITY) ? 0.f : m_used;
       const uint64_t nms2 = f2_pack(-ms, -ms);
       // P = 2^(scale*x - m): column pairs [0, kMufuPairs) on the MUFU unit,
       // the rest on the FMA pipe (exp2_poly), so both pipes share the load.
-      uint32_t pk0[32], pk1[32];
       uint64_t sum0 = f2_pack(0.f, 0.f), sum1 = sum0, sum2 = sum0, sum3 = sum0;
 #pragma unroll
-      for (int c2 = 0; c2 < BN / 2; ++c2) {
-        float e0, e1;
-        f2_unpack(f2_fma(f2_pack(x[2 * c2], x[2 * c2 + 1]), sl2, nms2), e0, e1);
-        if (c2 < kMufuPairs) {
-          e0 = ex2_approx(e0);
-          e1 = ex2_approx(e1);
-        } else {
-          e0 = exp2_poly(e0);
-          e1 = exp2_poly(e1);
+      for (int half = 0; half < 2; ++half) {   // 64 columns at a time: P stored before the next half
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int c2 = 32 * half + c;
+          float e0, e1;
+          f2_unpack(f2_fma(f2_pack(x[2 * c2], x[2 * c2 + 1]), sl2, nms2), e0, e1);
+          if (c2 < kMufuPairs) {
+            e0 = ex2_approx(e0);
+            e1 = ex2_approx(e1);
+          } else {
+            e0 = exp2_poly(e0);
+            e1 = exp2_poly(e1);
+          }
+          const uint64_t ee = f2_pack(e0, e1);
+          if ((c & 3) == 0) sum0 = f2_add(sum0, ee);
+          else if ((c & 3) == 1) sum1 = f2_add(sum1, ee);
+          else if ((c & 3) == 2) sum2 = f2_add(sum2, ee);
+          else sum3 = f2_add(sum3, ee);
+          pk[c] = pack_bf16x2(e0, e1);
         }
-        const uint64_t ee = f2_pack(e0, e1);
-        if ((c2 & 3) == 0) sum0 = f2_add(sum0, ee);
-        else if ((c2 & 3) == 1) sum1 = f2_add(sum1, ee);
-        else if ((c2 & 3) == 2) sum2 = f2_add(sum2, ee);
-        else sum3 = f2_add(sum3, ee);
-        if (c2 < 32) pk0[c2] = pack_bf16x2(e0, e1);
-        else pk1[c2 - 32] = pack_bf16x2(e0, e1);
+        tmem_st32(tS + lane_off + 32 * half, pk);
       }
-      float sa, sb2;
-      f2_unpack(f2_add(f2_add(sum0, sum1), f2_add(sum2, sum3)), sa, sb2);
-      l += sa + sb2;
-      tmem_st32((tS0 + 128u * sb) + lane_off + 0, pk0);
-      tmem_st32((tS0 + 128u * sb) + lane_off + 32, pk1);
+      float sa, sb;
+      f2_unpack(f2_add(f2_add(sum0, sum1), f2_add(sum2, sum3)), sa, sb);
+      l += sa + sb;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[sb]);
+      mbar_arrive(&bars->p_full[q]);
     }
     // ---- epilogue: O / l and LSE
-    if (mbar_wait(&bars->o_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
+    if (ntile > 0 && mbar_wait(&bars->o_final[q], 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const int64_t orow = (int64_t(rb) * p.n + i) * p.hq + j;
@@ -347,8 +397,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     }
   }
 
-  // ---- teardown: every MMA has completed once o_final fired (or the wait gave up)
-  if (warp == 1 && lane == 0) mbar_wait(&bars->o_final, 0, nullptr, nullptr, p.limit_ns);
+  // ---- teardown: every MMA has completed once both o_final fired (or the waits gave up)
+  if (warp == 1 && lane == 0) {
+    mbar_wait(&bars->o_final[0], 0, nullptr, nullptr, p.limit_ns);
+    mbar_wait(&bars->o_final[1], 0, nullptr, nullptr, p.limit_ns);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -412,8 +465,9 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
   const uly_shape& s = *shape;
   const int64_t hq = s.h_q / s.P, hkv = s.h_kv / s.P, Pb = int64_t(s.P) * s.b;
   const int64_t ntiles = (s.n + fwd::BM - 1) / fwd::BM;
+  const int64_t npairs = (ntiles + 1) / 2;
   const int64_t P_sel = rank < 0 ? s.P : 1;
-  const int64_t grid = ntiles * P_sel * s.b * hq;
+  const int64_t grid = npairs * P_sel * s.b * hq;
   if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
   // Outputs must not overlap inputs.
   const size_t qbytes = size_t(Pb * s.n * hq * s.d) * 2, kvbytes = size_t(Pb * s.n * hkv * s.d) * 2;
@@ -448,6 +502,7 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
   p.hq = int32_t(hq);
   p.G = int32_t(s.h_q / s.h_kv);
   p.ntiles = int32_t(ntiles);
+  p.npairs = int32_t(npairs);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(float(s.d));
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_f32 = o_dtype == ULY_F32;

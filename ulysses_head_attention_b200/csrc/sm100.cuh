@@ -39,14 +39,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// is parked by the hardware (up to kSuspendHintNs) and woken when the phase
+// completes, instead of re-issuing polls that steal issue slots from the
+// math warps sharing its SM sub-partition.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -57,9 +63,9 @@ enum : int {
   kDevTimeout = 1,
 };
 
-// Bounded wait on an mbarrier phase.  Spins on try_wait; every 1024 polls it
-// checks the CTA-wide abort flag (set by any warp that gave up) and the
-// elapsed time.  Returns false when it gave up: the caller must stop its
+// Bounded wait on an mbarrier phase.  Repeats the (suspending) try_wait;
+// every 16 tries it checks the CTA-wide abort flag (set by any warp that gave
+// up) and the elapsed time.  Returns false when it gave up: the caller must stop its
 // loop, and the kernel reports kDevTimeout through the status word.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* status, uint64_t limit_ns) {
@@ -67,7 +73,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 1023u) == 0) {
+    if ((it & 15u) == 0) {
       if (abort_flag && *abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         if (abort_flag) *abort_flag = 1;
