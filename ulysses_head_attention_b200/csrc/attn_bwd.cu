@@ -20,17 +20,17 @@
 //               -D (negated so they feed packed fused multiply-adds).
 //  * bwd_dkdv:  one CTA per (rank, batch row, kv head, 128-key tile),
 //               heaviest first.  Loops over the G query heads of the kv head
-//               and the 64-row query tiles that can see the key tile:
+//               and the 128-row query tiles that can see the key tile:
 //                 warp 0      TMA producer (K, V once; Q, dO, row stats ring)
 //                 warp 1      TMEM owner, single-thread MMA issuer
 //                 warps 4..11 thread = key row, two warpgroups each taking
-//                             32 of the 64 query columns: P^T, dS^T from S^T, dP^T
-//               S^T = K Q^T and dP^T = V dO^T (M=128 keys, N=64) are double
-//               buffered in TMEM; P^T and dS^T go back to TMEM as bf16 over
-//               them and feed dV += P^T dO, dK += dS^T Q as A-from-TMEM MMAs
-//               accumulating in TMEM across the whole group.
-//               TMEM: dK [0,128) dV [128,256) S^T_b [256+128b, +64)
-//               dP^T_b [320+128b, +64).
+//                             64 of the 128 query columns: P^T, dS^T from S^T, dP^T
+//               S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128: the
+//               shape runs the tensor core at full rate, N = 64 does not) go
+//               to TMEM; P^T and dS^T go back over them as bf16 and feed
+//               dV += P^T dO, dK += dS^T Q as A-from-TMEM MMAs accumulating
+//               in TMEM across the whole group.
+//               TMEM: dK [0,128) dV [128,256) S^T [256,384) dP^T [384,512).
 //  * bwd_dq:    one CTA per (rank, batch row, query head, 128-row tile),
 //               heaviest first; the forward's structure (K and V rings fed
 //               by separate producer warps).  S = Q K^T into a
@@ -54,7 +54,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ============================================================================
 // bwd_pre: D = rowsum(dO * O) and LSE*log2(e), one warp per (rank, row, head)
 // ============================================================================
-// stats layout: [P*b][hq][n_pad/64] blocks of {64 x -LSE*log2e, 64 x -D};
+// stats layout: [P*b][hq][n_pad/64] blocks of {64 x -LSE*log2e, 64 x -D}
+// (n_pad a multiple of 128, so a 128-row query tile is two whole blocks);
 // rows n..n_pad-1 are zero.
 __device__ __forceinline__ int64_t stats_index(int64_t rbh, int64_t n_pad, int64_t i) {
   return (rbh * (n_pad / 64) + i / 64) * 128 + (i & 63);
@@ -105,9 +106,9 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
 // ============================================================================
 namespace dkdv {
 
-constexpr int BKV = 128;
-constexpr int BQ = 64;
-constexpr int NS = 3;
+constexpr int BKV = 128;   // keys per CTA
+constexpr int BQ = 128;    // query rows per inner tile (N = 128 MMAs)
+constexpr int NS = 2;      // Q / dO / row-statistics stages
 constexpr int kThreads = 384;
 
 struct Params {
@@ -127,7 +128,7 @@ template <int D>
 struct Layout {
   static constexpr uint32_t kKV = BKV * D * 2;
   static constexpr uint32_t kQ = BQ * D * 2;
-  static constexpr uint32_t kSt = BQ * 8;
+  static constexpr uint32_t kSt = BQ * 8;                // two 64-row blocks of {-LSE*log2e, -D}
   static constexpr uint32_t oK = 0;
   static constexpr uint32_t oV = oK + kKV;
   static constexpr uint32_t oQ = oV + kKV;
@@ -140,16 +141,26 @@ struct Layout {
 struct Bars {
   uint64_t kv_full;
   uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full[2], p_ready[2];
+  uint64_t s_full, dp_full, p_ready, ds_ready;
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// Key-stationary dK/dV.  Per (query head, 128-row query tile):
+//   S^T = K Q^T, dP^T = V dO^T   (M = 128 keys, N = 128 queries)
+//   softmax warpgroups: P^T, dS^T back over S^T / dP^T as bf16
+//   dV += P^T dO, dK += dS^T Q   (A from TMEM, N = D)
+// TMEM: dK [0,128) dV [128,256) S^T [256,384) dP^T [384,512), single
+// buffered.  Issue order S(0) dP(0) | dV(0) S(1) dK(0) dP(1) | dV(1) S(2) ...:
+// each region is rewritten only after the MMA that reads its bf16 copy was
+// issued (the pipe runs one thread's MMAs in order), and the exponentials of
+// tile i+1 overlap dK(i) and dP(i+1) on the tensor core.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-       const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo, const Params p) {
+                     const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+                     const Params p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,10 +180,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   const int64_t last_key = (k0 + BKV - 1 < p.n - 1) ? (k0 + BKV - 1) : (p.n - 1);
   const int32_t* se = p.segend + int64_t(bb) * p.n;
   const int64_t q_end = se[last_key];      // query rows that see this key tile: [k0, q_end)
-  const int64_t seg_end_min = se[k0];
   const int qt_first = int(k0 / BQ);
   const int nqt = int((q_end + BQ - 1) / BQ) - qt_first;
-  const int niter = nqt * p.G;
+  const int niter = nqt * p.G;             // (query head, query tile) pairs, head-major
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -180,10 +190,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_ready[s], 256);
-    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->p_ready, 256);
+    mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->mma_final, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -196,9 +206,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tDK = tmem, tDV = tmem + 128;
-  auto tS = [&](int b) { return tmem + 256u + 128u * uint32_t(b); };
-  auto tDP = [&](int b) { return tmem + 320u + 128u * uint32_t(b); };
+  const uint32_t tDK = tmem, tDV = tmem + 128, tS = tmem + 256, tDP = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -234,49 +242,66 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16(BKV, BQ, false, false);
       const uint32_t id_g = idesc_bf16(BKV, D, false, true);
-      const uint32_t k_addr = smem_u32(smem + L::oK), v_addr = smem_u32(smem + L::oV);
-      bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns);
-      tc_fence_after();
-      auto issue_grads = [&](int jt) -> bool {
-        const int b = jt & 1, st = jt % NS;
-        if (!mbar_wait(&bars->p_ready[b], (jt >> 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + L::oQ + st * L::kQ);
-        const uint32_t do_addr = smem_u32(smem + L::oDO + st * L::kQ);
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          // P^T / dS^T bf16 pairs of query columns [16kk, 16kk+16): the first
-          // 32 columns sit in TMEM columns [0,16), the last 32 in [32,48)
-          // (one block per softmax warpgroup).
-          const uint32_t a_col = kk < 2 ? kk * 8 : 32 + (kk - 2) * 8;
-          const uint32_t acc = (jt > 0 || kk > 0) ? 1u : 0u;
-          umma_ts(tDV, tS(b) + a_col, sdesc_sw128(do_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
-          umma_ts(tDK, tDP(b) + a_col, sdesc_sw128(q_addr + kk * 2048, BQ * 128, 1024), id_g, acc);
-        }
-        umma_commit(&bars->q_empty[st]);
-        return true;
-      };
-      for (int it = 0; ok && it < niter; ++it) {
-        const int st = it % NS, rnd = it / NS, b = it & 1;
-        if (!mbar_wait(&bars->q_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(smem + L::oQ + st * L::kQ);
-        const uint32_t do_addr = smem_u32(smem + L::oDO + st * L::kQ);
+      const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::oK), 16, 1024);
+      const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::oV), 16, 1024);
+      auto issue_s = [&](int it) {   // S^T = K Q^T into [256, 384)
+        const uint64_t qd = sdesc_sw128(smem_u32(smem + L::oQ + (it % NS) * L::kQ), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * (BKV * 128) + (kk & 3) * 32;
-          const uint32_t qa = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          umma_ss(tS(b), sdesc_sw128(k_addr + ka, 16, 1024), sdesc_sw128(q_addr + qa, 16, 1024), id_s, kk > 0);
-          umma_ss(tDP(b), sdesc_sw128(v_addr + ka, 16, 1024), sdesc_sw128(do_addr + qa, 16, 1024), id_s, kk > 0);
+          const uint64_t ka = uint64_t(((kk >> 2) * (BKV * 128) + (kk & 3) * 32) / 16);
+          const uint64_t qa = uint64_t(((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16);
+          umma_ss(tS, k_desc + ka, qd + qa, id_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full[b]);
-        if (it >= 1 && !issue_grads(it - 1)) { ok = false; break; }
+        umma_commit(&bars->s_full);
+      };
+      auto issue_dp = [&](int it) {   // dP^T = V dO^T into [384, 512)
+        const uint64_t dod = sdesc_sw128(smem_u32(smem + L::oDO + (it % NS) * L::kQ), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ka = uint64_t(((kk >> 2) * (BKV * 128) + (kk & 3) * 32) / 16);
+          const uint64_t qa = uint64_t(((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16);
+          umma_ss(tDP, v_desc + ka, dod + qa, id_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->dp_full);
+      };
+      // P^T / dS^T bf16 pairs of query columns [16kk, 16kk+16): the first 64
+      // columns sit in TMEM columns [0,32) of their region, the last 64 in
+      // [64,96) (one block per softmax warpgroup).  B = dO / Q, MN-major.
+      auto issue_grad = [&](int it, uint32_t acc_tmem, uint32_t a_tmem, uint8_t* b_smem) {
+        const uint64_t bd = sdesc_sw128(smem_u32(b_smem + (it % NS) * L::kQ), BQ * 128, 1024);
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
+          umma_ts(acc_tmem, a_tmem + a_col, bd + uint64_t(kk * 2048 / 16), id_g, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns) && niter > 0 &&
+                mbar_wait(&bars->q_full[0], 0, abort_flag, p.status, p.limit_ns);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
       }
-      if (ok && niter > 0) issue_grads(niter - 1);
+      for (int it = 0; ok && it < niter; ++it) {
+        const bool more = it + 1 < niter;
+        if (more && !mbar_wait(&bars->q_full[(it + 1) % NS], ((it + 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&bars->p_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        issue_grad(it, tDV, tS, smem + L::oDO);          // dV += P^T dO
+        if (more) issue_s(it + 1);
+        if (!mbar_wait(&bars->ds_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        tc_fence_after();
+        issue_grad(it, tDK, tDP, smem + L::oQ);          // dK += dS^T Q
+        umma_commit(&bars->q_empty[it % NS]);
+        if (more) issue_dp(it + 1);
+      }
       umma_commit(&bars->mma_final);
     }
   } else if (warp >= 4) {
-    const int wg = (warp - 4) >> 2;                  // query columns [32 wg, 32 wg + 32) of each tile
+    const int wg = (warp - 4) >> 2;                  // query columns [64 wg, 64 wg + 64) of each tile
     const int row = ((warp - 4) & 3) * 32 + lane;    // key row within the tile
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t kj = k0 + row;
@@ -284,49 +309,75 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < niter; ++it) {
-      const int b = it & 1, st = it % NS;
-      const int64_t qb = int64_t(qt_first + it % nqt) * BQ + 32 * wg;   // first query column of this warpgroup
+      const int st = it % NS;
+      const int64_t q0 = int64_t(qt_first + it % nqt) * BQ;
       if (!mbar_wait(&bars->q_full[st], (it / NS) & 1, abort_flag, p.status, p.limit_ns) ||
-          !mbar_wait(&bars->s_full[b], (it >> 1) & 1, abort_flag, p.status, p.limit_ns)) {
+          !mbar_wait(&bars->s_full, it & 1, abort_flag, p.status, p.limit_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float* stt = reinterpret_cast<const float*>(smem + L::oSt + st * L::kSt) + 32 * wg;
-      // visible query columns c of this warpgroup: lo <= c < hi
-      const int64_t lo64 = kj - qb, hi64 = kj_end - qb;
-      const bool need_mask = lo64 > 0 || hi64 < 32;
-      const int lo = int(lo64 < 0 ? 0 : (lo64 > 32 ? 32 : lo64));
-      const int hi = int(hi64 < 0 ? 0 : (hi64 > 32 ? 32 : hi64));
-      uint32_t s[32], dp[32];
-      tmem_ld32(tS(b) + lane_off + 32 * wg, s);
-      tmem_ld32(tDP(b) + lane_off + 32 * wg, dp);
-      tmem_ld_wait();
-      uint32_t pw[16], dw[16];
+      // this warpgroup's 64 columns are statistics block wg: {64 x -LSE*log2e, 64 x -D}
+      const float* stt = reinterpret_cast<const float*>(smem + L::oSt + st * L::kSt) + 128 * wg;
+      float pr[64];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float2 nl = *reinterpret_cast<const float2*>(stt + 2 * c);        // -LSE*log2e
-        const float2 nd = *reinterpret_cast<const float2*>(stt + 64 + 2 * c);   // -D
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sl2,
-                         f2_pack(nl.x, nl.y)), x0, x1);
-        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-        if (need_mask) {
-          if (unsigned(2 * c - lo) >= unsigned(hi - lo)) p0 = 0.f;
-          if (unsigned(2 * c + 1 - lo) >= unsigned(hi - lo)) p1 = 0.f;
+      for (int ch = 0; ch < 2; ++ch) {
+        const int64_t qb = q0 + 64 * wg + 32 * ch;   // first query column of this chunk
+        const int64_t lo64 = kj - qb, hi64 = kj_end - qb;
+        const bool need_mask = lo64 > 0 || hi64 < 32;
+        const int lo = int(lo64 < 0 ? 0 : (lo64 > 32 ? 32 : lo64));
+        const int hi = int(hi64 < lo ? lo : (hi64 > 32 ? 32 : hi64));
+        uint32_t sv[32];
+        tmem_ld32(tS + lane_off + 64 * wg + 32 * ch, sv);
+        tmem_ld_wait();
+        uint32_t pw[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float2 nl = *reinterpret_cast<const float2*>(stt + 32 * ch + 2 * c);   // -LSE*log2e
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2,
+                           f2_pack(nl.x, nl.y)), x0, x1);
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (need_mask) {
+            if (unsigned(2 * c - lo) >= unsigned(hi - lo)) p0 = 0.f;
+            if (unsigned(2 * c + 1 - lo) >= unsigned(hi - lo)) p1 = 0.f;
+          }
+          pr[32 * ch + 2 * c] = p0;
+          pr[32 * ch + 2 * c + 1] = p1;
+          pw[c] = pack_bf16x2(p0, p1);
         }
-        const uint64_t pp = f2_pack(p0, p1);
-        float d0, d1;
-        f2_unpack(f2_mul(pp, f2_add(f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])),
-                                    f2_pack(nd.x, nd.y))), d0, d1);
-        pw[c] = pack_bf16x2(p0, p1);
-        dw[c] = pack_bf16x2(d0, d1);
+        // packed pairs of this chunk go to columns [64 wg + 16 ch, +16): inside
+        // this warpgroup's own, already read, column range
+        tmem_st16(tS + lane_off + 64 * wg + 16 * ch, pw);
       }
-      tmem_st16(tS(b) + lane_off + 32 * wg, pw);
-      tmem_st16(tDP(b) + lane_off + 32 * wg, dw);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready[b]);
+      mbar_arrive(&bars->p_ready);
+      if (!mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t dp[32];
+        tmem_ld32(tDP + lane_off + 64 * wg + 32 * ch, dp);
+        tmem_ld_wait();
+        uint32_t dw[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float2 nd = *reinterpret_cast<const float2*>(stt + 64 + 32 * ch + 2 * c);   // -D
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(pr[32 * ch + 2 * c], pr[32 * ch + 2 * c + 1]),
+                           f2_add(f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])),
+                                  f2_pack(nd.x, nd.y))), d0, d1);
+          dw[c] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tDP + lane_off + 64 * wg + 16 * ch, dw);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_ready);
     }
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
@@ -664,9 +715,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
 }  // namespace bwd
 
 // Backward workspace: the segment tables (as the forward), then the padded
-// row-statistics table [P][b][hq][n_pad] x {LSE*log2e, D} (n_pad = n rounded
-// up to 64).
-static int64_t bwd_n_pad(int64_t n) { return (n + 63) / 64 * 64; }
+// row-statistics table (see stats_index; n_pad = n rounded up to 128).
+static int64_t bwd_n_pad(int64_t n) { return (n + 127) / 128 * 128; }
 static size_t bwd_ws_stats_off(const uly_shape* s) { return seg_workspace_bytes(s->b, s->n); }
 
 }  // namespace uly
@@ -709,9 +759,8 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
     if (overlaps(outs[a], outsz[a], ws, ws_bytes)) return ULY_ERR_INVALID_ARG;
   }
 
-  CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128;
-  if (!make_head_map(&mq64, q_head, Pb, s.n, hq, s.d, 64) || !make_head_map(&mdo64, do_head, Pb, s.n, hq, s.d, 64) ||
-      !make_head_map(&mk128, k_head, Pb, s.n, hkv, s.d, 128) || !make_head_map(&mv128, v_head, Pb, s.n, hkv, s.d, 128) ||
+  CUtensorMap mk128, mv128, mq128, mdo128;
+  if (!make_head_map(&mk128, k_head, Pb, s.n, hkv, s.d, 128) || !make_head_map(&mv128, v_head, Pb, s.n, hkv, s.d, 128) ||
       !make_head_map(&mq128, q_head, Pb, s.n, hq, s.d, 128) || !make_head_map(&mdo128, do_head, Pb, s.n, hq, s.d, 128))
     return ULY_ERR_CUDA;
 
@@ -773,12 +822,12 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
       auto kern = bwd::dkdv::attn_bwd_dkdv_kernel<128>;
       const uint32_t sm = bwd::dkdv::Layout<128>::kDynamic;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
-      kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq64, mk128, mv128, mdo64, p);
+      kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq128, mk128, mv128, mdo128, p);
     } else {
       auto kern = bwd::dkdv::attn_bwd_dkdv_kernel<64>;
       const uint32_t sm = bwd::dkdv::Layout<64>::kDynamic;
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) != cudaSuccess) return ULY_ERR_CUDA;
-      kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq64, mk128, mv128, mdo64, p);
+      kern<<<unsigned(grid), bwd::dkdv::kThreads, sm, cs>>>(mq128, mk128, mv128, mdo128, p);
     }
     if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
