@@ -239,7 +239,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {   // whole warp; the elected lane issues
       const uint32_t id_s = idesc_bf16(BKV, BQ, false, false);
       const uint32_t id_g = idesc_bf16(BKV, D, false, true);
       const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::oK), 16, 1024);
@@ -250,9 +250,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ka = uint64_t(((kk >> 2) * (BKV * 128) + (kk & 3) * 32) / 16);
           const uint64_t qa = uint64_t(((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16);
-          umma_ss(tS, k_desc + ka, qd + qa, id_s, kk > 0 ? 1u : 0u);
+          umma_ss_warp(tS, k_desc + ka, qd + qa, id_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->s_full);
+        umma_commit_warp(&bars->s_full);
       };
       auto issue_dp = [&](int it) {   // dP^T = V dO^T into [384, 512)
         const uint64_t dod = sdesc_sw128(smem_u32(smem + L::oDO + (it % NS) * L::kQ), 16, 1024);
@@ -260,9 +260,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ka = uint64_t(((kk >> 2) * (BKV * 128) + (kk & 3) * 32) / 16);
           const uint64_t qa = uint64_t(((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16);
-          umma_ss(tDP, v_desc + ka, dod + qa, id_s, kk > 0 ? 1u : 0u);
+          umma_ss_warp(tDP, v_desc + ka, dod + qa, id_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars->dp_full);
+        umma_commit_warp(&bars->dp_full);
       };
       // P^T / dS^T bf16 pairs of query columns [16kk, 16kk+16): the first 64
       // columns sit in TMEM columns [0,32) of their region, the last 64 in
@@ -272,11 +272,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
-          umma_ts(acc_tmem, a_tmem + a_col, bd + uint64_t(kk * 2048 / 16), id_g, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_warp(acc_tmem, a_tmem + a_col, bd + uint64_t(kk * 2048 / 16), id_g, (it > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns) && niter > 0 &&
-                mbar_wait(&bars->q_full[0], 0, abort_flag, p.status, p.limit_ns);
+      bool ok = mbar_wait_warp(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns) && niter > 0 &&
+                mbar_wait_warp(&bars->q_full[0], 0, abort_flag, p.status, p.limit_ns);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -284,21 +284,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       }
       for (int it = 0; ok && it < niter; ++it) {
         const bool more = it + 1 < niter;
-        if (more && !mbar_wait(&bars->q_full[(it + 1) % NS], ((it + 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+        if (more && !mbar_wait_warp(&bars->q_full[(it + 1) % NS], ((it + 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(&bars->p_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->p_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
         issue_grad(it, tDV, tS, smem + L::oDO);          // dV += P^T dO
         if (more) issue_s(it + 1);
-        if (!mbar_wait(&bars->ds_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->ds_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
         issue_grad(it, tDK, tDP, smem + L::oQ);          // dK += dS^T Q
-        umma_commit(&bars->q_empty[it % NS]);
+        umma_commit_warp(&bars->q_empty[it % NS]);
         if (more) issue_dp(it + 1);
       }
-      umma_commit(&bars->mma_final);
+      umma_commit_warp(&bars->mma_final);
     }
   } else if (warp >= 4) {
     const int wg = (warp - 4) >> 2;                  // query columns [64 wg, 64 wg + 64) of each tile
@@ -559,15 +559,15 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {   // whole warp; the elected lane issues
       const uint32_t id_s = idesc_bf16(BM, BN, false, false);
       const uint32_t id_q = idesc_bf16(BM, D, false, true);
       const uint32_t q_addr = smem_u32(smem + L::oQ), do_addr = smem_u32(smem + L::oDO);
-      bool ok = mbar_wait(&bars->qdo_full, 0, abort_flag, p.status, p.limit_ns);
+      bool ok = mbar_wait_warp(&bars->qdo_full, 0, abort_flag, p.status, p.limit_ns);
       tc_fence_after();
       auto issue_dq = [&](int jt) -> bool {
         const int b = jt & 1, st = jt % NS;
-        if (!mbar_wait(&bars->ds_ready[b], (jt >> 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
+        if (!mbar_wait_warp(&bars->ds_ready[b], (jt >> 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + L::oK + st * L::kTile);
 #pragma unroll
@@ -575,38 +575,38 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
           // dS of keys [16kk, 16kk+16): the first 64 keys' bf16 pairs sit in S
           // columns [0,32), the last 64 keys' in [64,96) (one half per warpgroup).
           const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
-          umma_ts(tDQ, tS(b) + a_col, sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), id_q,
+          umma_ts_warp(tDQ, tS(b) + a_col, sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), id_q,
                   (jt > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars->k_empty[st]);
+        umma_commit_warp(&bars->k_empty[st]);
         return true;
       };
       for (int it = 0; ok && it < nkv; ++it) {
         const int st = it % NS, rnd = it / NS, b = it & 1;
-        if (!mbar_wait(&bars->k_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->k_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + L::oK + st * L::kTile);
         const uint32_t v_addr = smem_u32(smem + L::oV + st * L::kTile);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          umma_ss(tS(b), sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), id_s, kk > 0);
+          umma_ss_warp(tS(b), sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), id_s, kk > 0);
         }
-        umma_commit(&bars->s_full[b]);
-        if (it >= 1 && !mbar_wait(&bars->dp_free, (it - 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-        if (!mbar_wait(&bars->v_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        umma_commit_warp(&bars->s_full[b]);
+        if (it >= 1 && !mbar_wait_warp(&bars->dp_free, (it - 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->v_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          umma_ss(tDP, sdesc_sw128(do_addr + off, 16, 1024), sdesc_sw128(v_addr + off, 16, 1024), id_s, kk > 0);
+          umma_ss_warp(tDP, sdesc_sw128(do_addr + off, 16, 1024), sdesc_sw128(v_addr + off, 16, 1024), id_s, kk > 0);
         }
-        umma_commit(&bars->dp_full);
-        umma_commit(&bars->v_empty[st]);
+        umma_commit_warp(&bars->dp_full);
+        umma_commit_warp(&bars->v_empty[st]);
         if (it >= 1 && !issue_dq(it - 1)) { ok = false; break; }
       }
       if (ok) issue_dq(nkv - 1);
-      umma_commit(&bars->mma_final);
+      umma_commit_warp(&bars->mma_final);
     }
   } else if (warp >= 4) {
     const int wg = (warp - 4) >> 2;                 // column half handled by this warpgroup

@@ -191,11 +191,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         for (int x = max(0, issued - NS); x < issued; ++x)
           mbar_wait(&full[x % NS], (x / NS) & 1, nullptr, nullptr, p.limit_ns);
       }
-    } else if (warp == 1 && lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer (whole warp, elected lane issues)
       const uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
       const uint32_t idesc_o = idesc_bf16(BM, D, false, true);
-      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, p.status, p.limit_ns);
+      bool ok = mbar_wait_warp(&bars->q_full, 0, abort_flag, p.status, p.limit_ns);
       int npv[2] = {0, 0};
       for (int it = 0; ok && it <= nkv; ++it) {
         const int jj = j_lo + it;
@@ -205,16 +205,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           const uint32_t tS = tmem + 128u * q, tO = tmem + 256u + 128u * q;
           const bool do_pv = it >= 1 && tr.valid && jj - 1 >= tr.first && jj - 1 <= tr.last;
           const bool do_s = it < nkv && tr.valid && jj >= tr.first && jj <= tr.last;
-          // All waits of this step first, then its MMAs in one burst: a wait by
-          // the issuing thread stalls MMA issue for a few hundred cycles, so
-          // the stage waits ride along with tile 0's P wait.
-          if (do_pv && !mbar_wait(&bars->p_full[q], npv[q] & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+          // All waits of this step first, then its MMAs in one burst: a wait
+          // in the issuing warp leaves the tensor pipe short of work, so the
+          // stage waits ride along with tile 0's P wait.
+          if (do_pv && !mbar_wait_warp(&bars->p_full[q], npv[q] & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
           if (q == 0) {
-            if (it >= 1 && !mbar_wait(&bars->v_full[(it - 1) % NS], ((it - 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+            if (it >= 1 && !mbar_wait_warp(&bars->v_full[(it - 1) % NS], ((it - 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
               ok = false;
               break;
             }
-            if (it < nkv && !mbar_wait(&bars->k_full[it % NS], (it / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+            if (it < nkv && !mbar_wait_warp(&bars->k_full[it % NS], (it / NS) & 1, abort_flag, p.status, p.limit_ns)) {
               ok = false;
               break;
             }
@@ -225,10 +225,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           // so the issue loop is a few instructions per MMA.
           if (do_pv) {
             const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::kV + ((it - 1) % NS) * L::kTileBytes), BN * 128, 1024);
-            umma_ts(tO, tS, v_desc, idesc_o, npv[q] > 0 ? 1u : 0u);
+            umma_ts_warp(tO, tS, v_desc, idesc_o, npv[q] > 0 ? 1u : 0u);
 #pragma unroll
             for (int kk = 1; kk < BN / 16; ++kk)
-              umma_ts(tO, tS + kk * 8, v_desc + uint64_t(kk * 2048 / 16), idesc_o, 1u);
+              umma_ts_warp(tO, tS + kk * 8, v_desc + uint64_t(kk * 2048 / 16), idesc_o, 1u);
             ++npv[q];
           }
           if (do_s) {
@@ -237,17 +237,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t off = uint64_t(((kk >> 2) * (BM * 128) + (kk & 3) * 32) / 16);
-              umma_ss(tS, q_desc + off, k_desc + off, idesc_s, kk > 0 ? 1u : 0u);
+              umma_ss_warp(tS, q_desc + off, k_desc + off, idesc_s, kk > 0 ? 1u : 0u);
             }
-            umma_commit(&bars->s_full[q]);
+            umma_commit_warp(&bars->s_full[q]);
           }
         }
         if (!ok) break;
-        if (it >= 1) umma_commit(&bars->v_empty[(it - 1) % NS]);
-        if (it < nkv) umma_commit(&bars->k_empty[it % NS]);
+        if (it >= 1) umma_commit_warp(&bars->v_empty[(it - 1) % NS]);
+        if (it < nkv) umma_commit_warp(&bars->k_empty[it % NS]);
       }
-      umma_commit(&bars->o_final[0]);
-      umma_commit(&bars->o_final[1]);
+      umma_commit_warp(&bars->o_final[0]);
+      umma_commit_warp(&bars->o_final[1]);
     }
   } else {
     regs_inc216();
