@@ -33,7 +33,9 @@
 //               TMEM: dK [0,128) dV [128,256) S^T [256,384) dP^T [384,512).
 //  * bwd_dq:    one CTA per (rank, batch row, query head, 128-row tile),
 //               heaviest first; the forward's structure (K and V rings fed
-//               by separate producer warps).  S = Q K^T into a
+//               by separate producer warps; the K ring is three deep because
+//               dQ reads a K tile one step after S did, so a two-deep ring
+//               would leave no time to load the next one).  S = Q K^T into a
 //               double-buffered TMEM tile, dP = dO V^T, two softmax
 //               warpgroups (64 columns each) turn them into dS (bf16, over S)
 //               and dQ += dS K accumulates in TMEM.
@@ -136,6 +138,7 @@ struct Layout {
   static constexpr uint32_t oSt = oDO + NS * kQ;
   static constexpr uint32_t oBar = oSt + NS * kSt;
   static constexpr uint32_t kDynamic = oBar + 256 + 1024;
+  static_assert(kDynamic <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
 };
 
 struct Bars {
@@ -433,7 +436,8 @@ namespace dq {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int NS = 2;
+constexpr int NSK = 3;   // K ring: a K tile is read by S and, one step later, by dQ
+constexpr int NSV = 2;   // V ring: read by dP only
 constexpr int kThreads = 384;
 
 struct Params {
@@ -454,14 +458,15 @@ struct Layout {
   static constexpr uint32_t oQ = 0;
   static constexpr uint32_t oDO = oQ + kTile;
   static constexpr uint32_t oK = oDO + kTile;
-  static constexpr uint32_t oV = oK + NS * kTile;
-  static constexpr uint32_t oBar = oV + NS * kTile;
+  static constexpr uint32_t oV = oK + NSK * kTile;
+  static constexpr uint32_t oBar = oV + NSV * kTile;
   static constexpr uint32_t kDynamic = oBar + 256 + 1024;
+  static_assert(kDynamic <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
 };
 
 struct Bars {
   uint64_t qdo_full;
-  uint64_t k_full[NS], v_full[NS], k_empty[NS], v_empty[NS];
+  uint64_t k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV];
   uint64_t s_full[2], ds_ready[2];
   uint64_t dp_full, dp_free, mma_final;
   uint32_t tmem_base;
@@ -498,10 +503,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qdo_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
+      mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -534,6 +541,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       uint64_t* full = is_k ? bars->k_full : bars->v_full;
       uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
       const uint32_t base = is_k ? L::oK : L::oV;
+      const int ns = is_k ? NSK : NSV;
       tma_prefetch_desc(map);
       if (is_k) {
         mbar_arrive_expect_tx(&bars->qdo_full, 2 * L::kTile);
@@ -544,7 +552,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       }
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
-        const int st = it % NS, rnd = it / NS;
+        const int st = it % ns, rnd = it / ns;
         const int k0 = (kv_first + it) * BN;
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         mbar_arrive_expect_tx(&full[st], L::kTile);
@@ -554,8 +562,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       }
       if (*abort_flag) {
         if (is_k) mbar_wait(&bars->qdo_full, 0, nullptr, nullptr, p.limit_ns);
-        for (int x = max(0, issued - NS); x < issued; ++x)
-          mbar_wait(&full[x % NS], (x / NS) & 1, nullptr, nullptr, p.limit_ns);
+        for (int x = max(0, issued - ns); x < issued; ++x)
+          mbar_wait(&full[x % ns], (x / ns) & 1, nullptr, nullptr, p.limit_ns);
       }
     }
   } else if (warp == 1) {
@@ -566,7 +574,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       bool ok = mbar_wait_warp(&bars->qdo_full, 0, abort_flag, p.status, p.limit_ns);
       tc_fence_after();
       auto issue_dq = [&](int jt) -> bool {
-        const int b = jt & 1, st = jt % NS;
+        const int b = jt & 1, st = jt % NSK;
         if (!mbar_wait_warp(&bars->ds_ready[b], (jt >> 1) & 1, abort_flag, p.status, p.limit_ns)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(smem + L::oK + st * L::kTile);
@@ -582,11 +590,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         return true;
       };
       for (int it = 0; ok && it < nkv; ++it) {
-        const int st = it % NS, rnd = it / NS, b = it & 1;
-        if (!mbar_wait_warp(&bars->k_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        const int sk = it % NSK, sv = it % NSV, b = it & 1;
+        if (!mbar_wait_warp(&bars->k_full[sk], (it / NSK) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + L::oK + st * L::kTile);
-        const uint32_t v_addr = smem_u32(smem + L::oV + st * L::kTile);
+        const uint32_t k_addr = smem_u32(smem + L::oK + sk * L::kTile);
+        const uint32_t v_addr = smem_u32(smem + L::oV + sv * L::kTile);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
@@ -594,7 +602,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         }
         umma_commit_warp(&bars->s_full[b]);
         if (it >= 1 && !mbar_wait_warp(&bars->dp_free, (it - 1) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-        if (!mbar_wait_warp(&bars->v_full[st], rnd & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->v_full[sv], (it / NSV) & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -602,7 +610,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
           umma_ss_warp(tDP, sdesc_sw128(do_addr + off, 16, 1024), sdesc_sw128(v_addr + off, 16, 1024), id_s, kk > 0);
         }
         umma_commit_warp(&bars->dp_full);
-        umma_commit_warp(&bars->v_empty[st]);
+        umma_commit_warp(&bars->v_empty[sv]);
         if (it >= 1 && !issue_dq(it - 1)) { ok = false; break; }
       }
       if (ok) issue_dq(nkv - 1);
