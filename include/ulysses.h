@@ -175,8 +175,10 @@ uly_status ulysses_attn_fwd_noalloc(const void* q_head, const void* k_head, cons
 /*
  * ulysses_workspace_status -- synchronizes `stream`, then reads and clears
  * the status word kept at the start of an attention workspace.  *code gets
- * ULY_OK, or ULY_ERR_TIMEOUT when a kernel gave up waiting on one of its own
- * pipeline stages (its outputs are then invalid).
+ * ULY_OK, ULY_ERR_TIMEOUT when a kernel gave up waiting on one of its own
+ * pipeline stages, or ULY_ERR_CUDA when a kernel found its dynamic shared
+ * memory too poorly aligned to lay out its tiles and did nothing (in both
+ * error cases the outputs are invalid).
  */
 uly_status ulysses_workspace_status(void* ws, void* stream, int32_t* code);
 

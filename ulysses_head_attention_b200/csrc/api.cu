@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace uly {
 
@@ -58,6 +59,6 @@ extern "C" uly_status ulysses_workspace_status(void* ws, void* stream, int32_t* 
   if (cudaStreamSynchronize(s) != cudaSuccess) return ULY_ERR_CUDA;
   if (cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return ULY_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return ULY_ERR_CUDA;
-  *code = word == 0 ? ULY_OK : ULY_ERR_TIMEOUT;
+  *code = word == 0 ? ULY_OK : word == uly::kDevSmemAlign ? ULY_ERR_CUDA : ULY_ERR_TIMEOUT;
   return ULY_OK;
 }

@@ -110,8 +110,13 @@ namespace dkdv {
 
 constexpr int BKV = 128;   // keys per CTA
 constexpr int BQ = 128;    // query rows per inner tile (N = 128 MMAs)
-constexpr int NS = 2;      // Q / dO / row-statistics stages
+// A Q tile is read by S at the start of step i - 1 and by dK at the end of
+// step i, so its ring is three deep (two would expose the whole load
+// latency every step); dO and the row statistics live one step less.
+constexpr int NSQ = 3;     // Q stages
+constexpr int NSO = 2;     // dO + row-statistics stages
 constexpr int kThreads = 384;
+constexpr uint32_t kSmemOptin = 232448;   // per-CTA dynamic shared memory limit (227 KB)
 
 struct Params {
   const int32_t* segend;
@@ -134,31 +139,39 @@ struct Layout {
   static constexpr uint32_t oK = 0;
   static constexpr uint32_t oV = oK + kKV;
   static constexpr uint32_t oQ = oV + kKV;
-  static constexpr uint32_t oDO = oQ + NS * kQ;
-  static constexpr uint32_t oSt = oDO + NS * kQ;
-  static constexpr uint32_t oBar = oSt + NS * kSt;
-  static constexpr uint32_t kDynamic = oBar + 256 + 1024;
-  static_assert(kDynamic <= 227 * 1024, "dynamic shared memory above the per-CTA limit");
+  static constexpr uint32_t oDO = oQ + NSQ * kQ;
+  static constexpr uint32_t oSt = oDO + NSO * kQ;
+  static constexpr uint32_t oBar = oSt + NSO * kSt;
+  static constexpr uint32_t kUsed = oBar + 256;
+  // room to round the base up to 1024 bytes; at D = 128 the limit leaves
+  // 768, and the kernel checks the base it actually got
+  static constexpr uint32_t kDynamic = kUsed + 1024 < kSmemOptin ? kUsed + 1024 : kSmemOptin;
+  static constexpr uint32_t kSlack = kDynamic - kUsed;
+  static_assert(kUsed + 256 <= kDynamic, "dynamic shared memory above the per-CTA limit");
 };
 
 struct Bars {
   uint64_t kv_full;
-  uint64_t q_full[NS], q_empty[NS];
-  uint64_t s_full, dp_full, p_ready, ds_ready;
+  uint64_t q_full[NSQ], q_empty[NSQ], do_full[NSO], do_empty[NSO];
+  uint64_t s_full, dp_full, x_free, pd_ready;
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block outgrew its slot");
 
-// Key-stationary dK/dV.  Per (query head, 128-row query tile):
-//   S^T = K Q^T, dP^T = V dO^T   (M = 128 keys, N = 128 queries)
-//   softmax warpgroups: P^T, dS^T back over S^T / dP^T as bf16
-//   dV += P^T dO, dK += dS^T Q   (A from TMEM, N = D)
-// TMEM: dK [0,128) dV [128,256) S^T [256,384) dP^T [384,512), single
-// buffered.  Issue order S(0) dP(0) | dV(0) S(1) dK(0) dP(1) | dV(1) S(2) ...:
-// each region is rewritten only after the MMA that reads its bf16 copy was
-// issued (the pipe runs one thread's MMAs in order), and the exponentials of
-// tile i+1 overlap dK(i) and dP(i+1) on the tensor core.
+// Key-stationary dK/dV.  Per (query head, 128-row query tile) i:
+//   S^T = K Q^T -> X, dP^T = V dO^T -> Y   (M = 128 keys, N = 128 queries)
+//   softmax warpgroups: read S^T (then X is free), P^T = exp(...) in
+//   registers; once dP^T is in, P^T and dS^T go back to Y as bf16, packed
+//   side by side in the columns each chunk has just read
+//   dV += P^T dO, dK += dS^T Q   (A from Y, N = D)
+// TMEM: dK [0,128) dV [128,256) X [256,384) Y [384,512).  Issue order
+//   S(0) dP(0) | S(1) dV(0) dK(0) dP(1) | S(2) dV(1) dK(1) dP(2) | ...
+// S(i+1) only waits for the softmax to have read S^T(i), so the
+// exponentials of tile i+1 run while dV(i), dK(i) and dP(i+1) do; a region
+// is rewritten only after the MMAs that read it were issued (the pipe runs
+// one warp's MMAs in order).
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
@@ -167,6 +180,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if (uint32_t(smem - smem_raw) > L::kSlack) {   // uniform across the CTA: nothing has started yet
+    if (threadIdx.x == 0) atomicExch(p.status, kDevSmemAlign);
+    return;
+  }
   Bars* bars = reinterpret_cast<Bars*>(smem + L::oBar);
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -189,14 +206,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSQ; ++s) {
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
     }
+    for (int s = 0; s < NSO; ++s) {
+      mbar_init(&bars->do_full[s], 1);
+      mbar_init(&bars->do_empty[s], 1);
+    }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_ready, 256);
-    mbar_init(&bars->ds_ready, 256);
+    mbar_init(&bars->x_free, 256);
+    mbar_init(&bars->pd_ready, 256);
     mbar_init(&bars->mma_final, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -209,36 +230,47 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tDK = tmem, tDV = tmem + 128, tS = tmem + 256, tDP = tmem + 384;
+  const uint32_t tDK = tmem, tDV = tmem + 128, tX = tmem + 256, tY = tmem + 384;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 2) {
+    // producers: warp 0 loads K, V and the Q ring, warp 2 the dO + statistics
+    // ring, so neither ring's loads wait behind the other's free slots
     if (lane == 0) {
-      tma_prefetch_desc(&mq);
-      tma_prefetch_desc(&mdo);
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKV);
-      for (int dc = 0; dc < D / 64; ++dc) {
-        tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0), rb);
-        tma_load_4d(&mv, &bars->kv_full, smem + L::oV + dc * BKV * 128, dc * 64, g, int(k0), rb);
+      const bool is_q = warp == 0;
+      const int ns = is_q ? NSQ : NSO;
+      uint64_t* full = is_q ? bars->q_full : bars->do_full;
+      uint64_t* empty = is_q ? bars->q_empty : bars->do_empty;
+      tma_prefetch_desc(is_q ? &mq : &mdo);
+      if (is_q) {
+        mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKV);
+        for (int dc = 0; dc < D / 64; ++dc) {
+          tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0), rb);
+          tma_load_4d(&mv, &bars->kv_full, smem + L::oV + dc * BKV * 128, dc * 64, g, int(k0), rb);
+        }
       }
       int issued = 0;
       for (int it = 0; it < niter; ++it) {
-        const int st = it % NS, rnd = it / NS;
+        const int st = it % ns, rnd = it / ns;
         const int h = g * p.G + it / nqt;
         const int q0 = (qt_first + it % nqt) * BQ;
-        if (rnd > 0 && !mbar_wait(&bars->q_empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
-        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kQ + L::kSt);
-        for (int dc = 0; dc < D / 64; ++dc) {
-          tma_load_4d(&mq, &bars->q_full[st], smem + L::oQ + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
-          tma_load_4d(&mdo, &bars->q_full[st], smem + L::oDO + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
+        if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
+        if (is_q) {
+          mbar_arrive_expect_tx(&full[st], L::kQ);
+          for (int dc = 0; dc < D / 64; ++dc)
+            tma_load_4d(&mq, &full[st], smem + L::oQ + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
+        } else {
+          mbar_arrive_expect_tx(&full[st], L::kQ + L::kSt);
+          for (int dc = 0; dc < D / 64; ++dc)
+            tma_load_4d(&mdo, &full[st], smem + L::oDO + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
+          bulk_load(smem + L::oSt + st * L::kSt, p.stats + stats_index(int64_t(rb) * p.hq + h, p.n_pad, q0), L::kSt,
+                    &full[st]);
         }
-        bulk_load(smem + L::oSt + st * L::kSt, p.stats + stats_index(int64_t(rb) * p.hq + h, p.n_pad, q0), L::kSt,
-                  &bars->q_full[st]);
         issued = it + 1;
       }
-      if (*abort_flag) {
-        mbar_wait(&bars->kv_full, 0, nullptr, nullptr, p.limit_ns);
-        for (int x = max(0, issued - NS); x < issued; ++x)
-          mbar_wait(&bars->q_full[x % NS], (x / NS) & 1, nullptr, nullptr, p.limit_ns);
+      if (*abort_flag) {   // error path only: let every copy this thread started land
+        if (is_q) mbar_wait(&bars->kv_full, 0, nullptr, nullptr, p.limit_ns);
+        for (int x = max(0, issued - ns); x < issued; ++x)
+          mbar_wait(&full[x % ns], (x / ns) & 1, nullptr, nullptr, p.limit_ns);
       }
     }
   } else if (warp == 1) {
@@ -247,39 +279,41 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       const uint32_t id_g = idesc_bf16(BKV, D, false, true);
       const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::oK), 16, 1024);
       const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::oV), 16, 1024);
-      auto issue_s = [&](int it) {   // S^T = K Q^T into [256, 384)
-        const uint64_t qd = sdesc_sw128(smem_u32(smem + L::oQ + (it % NS) * L::kQ), 16, 1024);
+      auto issue_s = [&](int it) {   // S^T = K Q^T into X
+        const uint64_t qd = sdesc_sw128(smem_u32(smem + L::oQ + (it % NSQ) * L::kQ), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ka = uint64_t(((kk >> 2) * (BKV * 128) + (kk & 3) * 32) / 16);
           const uint64_t qa = uint64_t(((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16);
-          umma_ss_warp(tS, k_desc + ka, qd + qa, id_s, kk > 0 ? 1u : 0u);
+          umma_ss_warp(tX, k_desc + ka, qd + qa, id_s, kk > 0 ? 1u : 0u);
         }
         umma_commit_warp(&bars->s_full);
       };
-      auto issue_dp = [&](int it) {   // dP^T = V dO^T into [384, 512)
-        const uint64_t dod = sdesc_sw128(smem_u32(smem + L::oDO + (it % NS) * L::kQ), 16, 1024);
+      auto issue_dp = [&](int it) {   // dP^T = V dO^T into Y
+        const uint64_t dod = sdesc_sw128(smem_u32(smem + L::oDO + (it % NSO) * L::kQ), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ka = uint64_t(((kk >> 2) * (BKV * 128) + (kk & 3) * 32) / 16);
           const uint64_t qa = uint64_t(((kk >> 2) * (BQ * 128) + (kk & 3) * 32) / 16);
-          umma_ss_warp(tDP, v_desc + ka, dod + qa, id_s, kk > 0 ? 1u : 0u);
+          umma_ss_warp(tY, v_desc + ka, dod + qa, id_s, kk > 0 ? 1u : 0u);
         }
         umma_commit_warp(&bars->dp_full);
       };
-      // P^T / dS^T bf16 pairs of query columns [16kk, 16kk+16): the first 64
-      // columns sit in TMEM columns [0,32) of their region, the last 64 in
-      // [64,96) (one block per softmax warpgroup).  B = dO / Q, MN-major.
+      // The bf16 pairs of query columns [16kk, 16kk+16) sit in Y columns
+      // 32 (kk/2) + 8 (kk%2) for P^T, 16 further on for dS^T: each 32-query
+      // chunk is packed as 16 columns of P^T then 16 of dS^T.  B = dO / Q,
+      // MN-major.
       auto issue_grad = [&](int it, uint32_t acc_tmem, uint32_t a_tmem, uint8_t* b_smem) {
-        const uint64_t bd = sdesc_sw128(smem_u32(b_smem + (it % NS) * L::kQ), BQ * 128, 1024);
+        const uint64_t bd = sdesc_sw128(smem_u32(b_smem), BQ * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
+          const uint32_t a_col = 32 * (kk >> 1) + 8 * (kk & 1);
           umma_ts_warp(acc_tmem, a_tmem + a_col, bd + uint64_t(kk * 2048 / 16), id_g, (it > 0 || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait_warp(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns) && niter > 0 &&
-                mbar_wait_warp(&bars->q_full[0], 0, abort_flag, p.status, p.limit_ns);
+                mbar_wait_warp(&bars->q_full[0], 0, abort_flag, p.status, p.limit_ns) &&
+                mbar_wait_warp(&bars->do_full[0], 0, abort_flag, p.status, p.limit_ns);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -287,19 +321,29 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       }
       for (int it = 0; ok && it < niter; ++it) {
         const bool more = it + 1 < niter;
-        if (more && !mbar_wait_warp(&bars->q_full[(it + 1) % NS], ((it + 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
-          ok = false;
-          break;
+        if (more) {
+          if (!mbar_wait_warp(&bars->x_free, it & 1, abort_flag, p.status, p.limit_ns) ||
+              !mbar_wait_warp(&bars->q_full[(it + 1) % NSQ], ((it + 1) / NSQ) & 1, abort_flag, p.status, p.limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(it + 1);
         }
-        if (!mbar_wait_warp(&bars->p_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->pd_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
-        issue_grad(it, tDV, tS, smem + L::oDO);          // dV += P^T dO
-        if (more) issue_s(it + 1);
-        if (!mbar_wait_warp(&bars->ds_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
-        tc_fence_after();
-        issue_grad(it, tDK, tDP, smem + L::oQ);          // dK += dS^T Q
-        umma_commit_warp(&bars->q_empty[it % NS]);
-        if (more) issue_dp(it + 1);
+        issue_grad(it, tDV, tY, smem + L::oDO + (it % NSO) * L::kQ);        // dV += P^T dO
+        umma_commit_warp(&bars->do_empty[it % NSO]);
+        issue_grad(it, tDK, tY + 16, smem + L::oQ + (it % NSQ) * L::kQ);    // dK += dS^T Q
+        umma_commit_warp(&bars->q_empty[it % NSQ]);
+        if (more) {
+          if (!mbar_wait_warp(&bars->do_full[(it + 1) % NSO], ((it + 1) / NSO) & 1, abort_flag, p.status, p.limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dp(it + 1);
+        }
       }
       umma_commit_warp(&bars->mma_final);
     }
@@ -312,9 +356,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < niter; ++it) {
-      const int st = it % NS;
+      const int st = it % NSO;
       const int64_t q0 = int64_t(qt_first + it % nqt) * BQ;
-      if (!mbar_wait(&bars->q_full[st], (it / NS) & 1, abort_flag, p.status, p.limit_ns) ||
+      if (!mbar_wait(&bars->do_full[st], (it / NSO) & 1, abort_flag, p.status, p.limit_ns) ||
           !mbar_wait(&bars->s_full, it & 1, abort_flag, p.status, p.limit_ns)) {
         ok = false;
         break;
@@ -331,15 +375,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         const int lo = int(lo64 < 0 ? 0 : (lo64 > 32 ? 32 : lo64));
         const int hi = int(hi64 < lo ? lo : (hi64 > 32 ? 32 : hi64));
         uint32_t sv[32];
-        tmem_ld32(tS + lane_off + 64 * wg + 32 * ch, sv);
+        tmem_ld32(tX + lane_off + 64 * wg + 32 * ch, sv);
+        float2 nl[16];   // -LSE*log2e, fetched while the TMEM load is in flight
+#pragma unroll
+        for (int c = 0; c < 16; ++c) nl[c] = *reinterpret_cast<const float2*>(stt + 32 * ch + 2 * c);
         tmem_ld_wait();
-        uint32_t pw[16];
+        if (ch == 1) {   // every S^T column of this thread is in registers: X may be rewritten
+          tc_fence_before();
+          mbar_arrive(&bars->x_free);
+        }
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float2 nl = *reinterpret_cast<const float2*>(stt + 32 * ch + 2 * c);   // -LSE*log2e
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2,
-                           f2_pack(nl.x, nl.y)), x0, x1);
+                           f2_pack(nl[c].x, nl[c].y)), x0, x1);
           float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           if (need_mask) {
             if (unsigned(2 * c - lo) >= unsigned(hi - lo)) p0 = 0.f;
@@ -347,15 +396,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           }
           pr[32 * ch + 2 * c] = p0;
           pr[32 * ch + 2 * c + 1] = p1;
-          pw[c] = pack_bf16x2(p0, p1);
         }
-        // packed pairs of this chunk go to columns [64 wg + 16 ch, +16): inside
-        // this warpgroup's own, already read, column range
-        tmem_st16(tS + lane_off + 64 * wg + 16 * ch, pw);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->p_ready);
       if (!mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
         ok = false;
         break;
@@ -364,23 +406,28 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t dp[32];
-        tmem_ld32(tDP + lane_off + 64 * wg + 32 * ch, dp);
+        tmem_ld32(tY + lane_off + 64 * wg + 32 * ch, dp);
+        float2 nd[16];   // -D
+#pragma unroll
+        for (int c = 0; c < 16; ++c) nd[c] = *reinterpret_cast<const float2*>(stt + 64 + 32 * ch + 2 * c);
         tmem_ld_wait();
-        uint32_t dw[16];
+        uint32_t pw[16], dw[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float2 nd = *reinterpret_cast<const float2*>(stt + 64 + 32 * ch + 2 * c);   // -D
+          const float p0 = pr[32 * ch + 2 * c], p1 = pr[32 * ch + 2 * c + 1];
           float d0, d1;
-          f2_unpack(f2_mul(f2_pack(pr[32 * ch + 2 * c], pr[32 * ch + 2 * c + 1]),
-                           f2_add(f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])),
-                                  f2_pack(nd.x, nd.y))), d0, d1);
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])),
+                                                   f2_pack(nd[c].x, nd[c].y))), d0, d1);
+          pw[c] = pack_bf16x2(p0, p1);
           dw[c] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(tDP + lane_off + 64 * wg + 16 * ch, dw);
+        // the 32 columns this chunk has just read: 16 of P^T, then 16 of dS^T
+        tmem_st16(tY + lane_off + 64 * wg + 32 * ch, pw);
+        tmem_st16(tY + lane_off + 64 * wg + 32 * ch + 16, dw);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->ds_ready);
+      mbar_arrive(&bars->pd_ready);
     }
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();

@@ -57,10 +57,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Error words written to the caller's status slot when a wait gives up.
+// Error words written to the caller's status slot: a wait gave up, or a
+// kernel found its dynamic shared memory too poorly aligned for its tiles.
 enum : int {
   kDevOk = 0,
   kDevTimeout = 1,
+  kDevSmemAlign = 2,
 };
 
 // Bounded wait on an mbarrier phase.  Repeats the (suspending) try_wait;
