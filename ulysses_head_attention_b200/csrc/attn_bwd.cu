@@ -117,6 +117,11 @@ constexpr int NSQ = 3;     // Q stages
 constexpr int NSO = 2;     // dO + row-statistics stages
 constexpr int kThreads = 384;
 constexpr uint32_t kSmemOptin = 232448;   // per-CTA dynamic shared memory limit (227 KB)
+#ifndef DKDV_REGS_LO
+#define DKDV_REGS_LO 72
+#define DKDV_REGS_HI 216
+#endif
+constexpr int kRegsLo = DKDV_REGS_LO, kRegsHi = DKDV_REGS_HI;
 
 struct Params {
   const int32_t* segend;
@@ -232,6 +237,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   const uint32_t tmem = bars->tmem_base;
   const uint32_t tDK = tmem, tDV = tmem + 128, tX = tmem + 256, tY = tmem + 384;
 
+
+  if (warp < 4) {
+  regs_split<kRegsLo, kRegsHi>(false);   // producers, MMA issuer, idle warp 3
   if (warp == 0 || warp == 2) {
     // producers: warp 0 loads K, V and the Q ring, warp 2 the dO + statistics
     // ring, so neither ring's loads wait behind the other's free slots
@@ -347,7 +355,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       }
       umma_commit_warp(&bars->mma_final);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    regs_split<kRegsLo, kRegsHi>(true);   // softmax warpgroups and epilogue
     const int wg = (warp - 4) >> 2;                  // query columns [64 wg, 64 wg + 64) of each tile
     const int row = ((warp - 4) & 3) * 32 + lane;    // key row within the tile
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
@@ -366,36 +376,37 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       tc_fence_after();
       // this warpgroup's 64 columns are statistics block wg: {64 x -LSE*log2e, 64 x -D}
       const float* stt = reinterpret_cast<const float*>(smem + L::oSt + st * L::kSt) + 128 * wg;
+      // visible query columns c of this warpgroup: lo <= c < hi (queries kj .. kj_end-1)
+      const int64_t qb = q0 + 64 * wg;
+      const int64_t lo64 = kj - qb, hi64 = kj_end - qb;
+      const bool need_mask = lo64 > 0 || hi64 < 64;
+      const int lo = int(lo64 < 0 ? 0 : (lo64 > 64 ? 64 : lo64));
+      const int hi = int(hi64 < lo ? lo : (hi64 > 64 ? 64 : hi64));
       float pr[64];
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int64_t qb = q0 + 64 * wg + 32 * ch;   // first query column of this chunk
-        const int64_t lo64 = kj - qb, hi64 = kj_end - qb;
-        const bool need_mask = lo64 > 0 || hi64 < 32;
-        const int lo = int(lo64 < 0 ? 0 : (lo64 > 32 ? 32 : lo64));
-        const int hi = int(hi64 < lo ? lo : (hi64 > 32 ? 32 : hi64));
-        uint32_t sv[32];
-        tmem_ld32(tX + lane_off + 64 * wg + 32 * ch, sv);
-        float2 nl[16];   // -LSE*log2e, fetched while the TMEM load is in flight
-#pragma unroll
-        for (int c = 0; c < 16; ++c) nl[c] = *reinterpret_cast<const float2*>(stt + 32 * ch + 2 * c);
+      uint32_t pw[32];
+      {
+        // both S^T chunks in one round trip, then X may be rewritten
+        uint32_t sv0[32], sv1[32];
+        tmem_ld32(tX + lane_off + 64 * wg, sv0);
+        tmem_ld32(tX + lane_off + 64 * wg + 32, sv1);
         tmem_ld_wait();
-        if (ch == 1) {   // every S^T column of this thread is in registers: X may be rewritten
-          tc_fence_before();
-          mbar_arrive(&bars->x_free);
-        }
+        tc_fence_before();
+        mbar_arrive(&bars->x_free);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 32; ++c) {
+          const int j = 2 * c;
+          const uint32_t s0 = c < 16 ? sv0[j] : sv1[j - 32], s1 = c < 16 ? sv0[j + 1] : sv1[j - 31];
+          const float2 nl = *reinterpret_cast<const float2*>(stt + j);   // -LSE*log2e
           float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), sl2,
-                           f2_pack(nl[c].x, nl[c].y)), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s0), __uint_as_float(s1)), sl2, f2_pack(nl.x, nl.y)), x0, x1);
           float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           if (need_mask) {
-            if (unsigned(2 * c - lo) >= unsigned(hi - lo)) p0 = 0.f;
-            if (unsigned(2 * c + 1 - lo) >= unsigned(hi - lo)) p1 = 0.f;
+            if (unsigned(j - lo) >= unsigned(hi - lo)) p0 = 0.f;
+            if (unsigned(j + 1 - lo) >= unsigned(hi - lo)) p1 = 0.f;
           }
-          pr[32 * ch + 2 * c] = p0;
-          pr[32 * ch + 2 * c + 1] = p1;
+          pr[j] = p0;
+          pr[j + 1] = p1;
+          pw[c] = pack_bf16x2(p0, p1);
         }
       }
       if (!mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
@@ -403,27 +414,30 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t dp[32];
-        tmem_ld32(tY + lane_off + 64 * wg + 32 * ch, dp);
-        float2 nd[16];   // -D
-#pragma unroll
-        for (int c = 0; c < 16; ++c) nd[c] = *reinterpret_cast<const float2*>(stt + 64 + 32 * ch + 2 * c);
+      {
+        uint32_t dp0[32], dp1[32];
+        tmem_ld32(tY + lane_off + 64 * wg, dp0);
+        tmem_ld32(tY + lane_off + 64 * wg + 32, dp1);
         tmem_ld_wait();
-        uint32_t pw[16], dw[16];
+        // each 32-query chunk goes back over the 32 columns it came from:
+        // 16 columns of P^T, then 16 of dS^T
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float p0 = pr[32 * ch + 2 * c], p1 = pr[32 * ch + 2 * c + 1];
-          float d0, d1;
-          f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dp[2 * c]), __uint_as_float(dp[2 * c + 1])),
-                                                   f2_pack(nd[c].x, nd[c].y))), d0, d1);
-          pw[c] = pack_bf16x2(p0, p1);
-          dw[c] = pack_bf16x2(d0, d1);
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t dw[16], pc[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int j = 32 * ch + 2 * c;
+            const uint32_t a0 = ch == 0 ? dp0[2 * c] : dp1[2 * c], a1 = ch == 0 ? dp0[2 * c + 1] : dp1[2 * c + 1];
+            const float2 nd = *reinterpret_cast<const float2*>(stt + 64 + j);   // -D
+            float d0, d1;
+            f2_unpack(f2_mul(f2_pack(pr[j], pr[j + 1]),
+                             f2_add(f2_pack(__uint_as_float(a0), __uint_as_float(a1)), f2_pack(nd.x, nd.y))), d0, d1);
+            dw[c] = pack_bf16x2(d0, d1);
+            pc[c] = pw[16 * ch + c];
+          }
+          tmem_st16(tY + lane_off + 64 * wg + 32 * ch, pc);
+          tmem_st16(tY + lane_off + 64 * wg + 32 * ch + 16, dw);
         }
-        // the 32 columns this chunk has just read: 16 of P^T, then 16 of dS^T
-        tmem_st16(tY + lane_off + 64 * wg + 32 * ch, pw);
-        tmem_st16(tY + lane_off + 64 * wg + 32 * ch + 16, dw);
       }
       tmem_st_wait();
       tc_fence_before();

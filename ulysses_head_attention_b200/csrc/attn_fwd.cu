@@ -81,8 +81,6 @@ struct Bars {
   int abort_flag;
 };
 
-__device__ __forceinline__ void regs_dec72() { asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory"); }
-__device__ __forceinline__ void regs_inc216() { asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory"); }
 
 // Key-tile range [first, last] of query tile `tile`, and the largest sample
 // start among its rows.
@@ -158,7 +156,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   const uint32_t tmem = bars->tmem_base;
 
   if (warp < 4) {
-    regs_dec72();
+    regs_split<72, 216>(false);
     if ((warp == 0 || warp == 2) && lane == 0) {
       // ---------------------------------------------------------- producers
       const bool is_k = warp == 0;
@@ -250,7 +248,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       umma_commit_warp(&bars->o_final[1]);
     }
   } else {
-    regs_inc216();
+    regs_split<72, 216>(true);
     // ------------------------------------------------------------ softmax
     const int q = (warp - 4) >> 2;                     // query tile of this warpgroup
     const TileRange tr = q ? tr1 : tr0;

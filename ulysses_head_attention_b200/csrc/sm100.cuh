@@ -39,20 +39,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-// try_wait with a suspend-time hint: a thread whose phase has not completed
-// is parked by the hardware (up to kSuspendHintNs) and woken when the phase
-// completes, instead of re-issuing polls that steal issue slots from the
-// math warps sharing its SM sub-partition.
-constexpr uint32_t kSuspendHintNs = 20000;
-
+// try_wait without a suspend-time hint: the hardware's own (short) limit
+// applies before it returns false and the caller polls again.  Measured on
+// B200 the waiting warp then sees a completed phase sooner than when it is
+// parked with a long hint (about 4% per backward step).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -256,6 +254,17 @@ __device__ __forceinline__ void umma_commit_warp(uint64_t* bar) {
   asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
                "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
                ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Register split for warp-specialised kernels of 384 threads launched at
+// 168 registers: the first warpgroup (producers, MMA issuer) drops to LO,
+// the two softmax warpgroups rise to HI, with 4*32*LO + 8*32*HI <= 384*168.
+// ptxas allocates each region to its own limit.
+template <int LO, int HI>
+__device__ __forceinline__ void regs_split(bool softmax_warpgroup) {
+  static_assert(LO % 8 == 0 && HI % 8 == 0 && 128 * LO + 256 * HI <= 384 * 168, "register split over budget");
+  if (softmax_warpgroup) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(HI) : "memory");
+  else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(LO) : "memory");
 }
 
 // ----------------------------------------------------------------------------
