@@ -158,7 +158,7 @@ struct Layout {
 struct Bars {
   uint64_t kv_full;
   uint64_t q_full[NSQ], q_empty[NSQ], do_full[NSO], do_empty[NSO];
-  uint64_t s_full, dp_full, x_free, pd_ready;
+  uint64_t s_full, dp_full, x_free, p_ready, ds_ready;
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort_flag;
@@ -168,8 +168,8 @@ static_assert(sizeof(Bars) <= 256, "barrier block outgrew its slot");
 // Key-stationary dK/dV.  Per (query head, 128-row query tile) i:
 //   S^T = K Q^T -> X, dP^T = V dO^T -> Y   (M = 128 keys, N = 128 queries)
 //   softmax warpgroups: read S^T (then X is free), P^T = exp(...) in
-//   registers; once dP^T is in, P^T and dS^T go back to Y as bf16, packed
-//   side by side in the columns each chunk has just read
+//   registers; once dP^T is in, P^T goes back to Y as bf16 (dV may start),
+//   then dS^T, packed side by side in the columns each chunk has just read
 //   dV += P^T dO, dK += dS^T Q   (A from Y, N = D)
 // TMEM: dK [0,128) dV [128,256) X [256,384) Y [384,512).  Issue order
 //   S(0) dP(0) | S(1) dV(0) dK(0) dP(1) | S(2) dV(1) dK(1) dP(2) | ...
@@ -222,7 +222,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
     mbar_init(&bars->x_free, 256);
-    mbar_init(&bars->pd_ready, 256);
+    mbar_init(&bars->p_ready, 256);
+    mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->mma_final, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -338,10 +339,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           tc_fence_after();
           issue_s(it + 1);
         }
-        if (!mbar_wait_warp(&bars->pd_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars->p_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
         issue_grad(it, tDV, tY, smem + L::oDO + (it % NSO) * L::kQ);        // dV += P^T dO
         umma_commit_warp(&bars->do_empty[it % NSO]);
+        if (!mbar_wait_warp(&bars->ds_ready, it & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
+        tc_fence_after();
         issue_grad(it, tDK, tY + 16, smem + L::oQ + (it % NSQ) * L::kQ);    // dK += dS^T Q
         umma_commit_warp(&bars->q_empty[it % NSQ]);
         if (more) {
@@ -420,10 +423,23 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         tmem_ld32(tY + lane_off + 64 * wg + 32, dp1);
         tmem_ld_wait();
         // each 32-query chunk goes back over the 32 columns it came from:
-        // 16 columns of P^T, then 16 of dS^T
+        // 16 columns of P^T, then 16 of dS^T.  P^T first, so dV can start
+        // while dS is computed.
+        {
+          uint32_t pc[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pc[c] = pw[c];
+          tmem_st16(tY + lane_off + 64 * wg, pc);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) pc[c] = pw[16 + c];
+          tmem_st16(tY + lane_off + 64 * wg + 32, pc);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
-          uint32_t dw[16], pc[16];
+          uint32_t dw[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int j = 32 * ch + 2 * c;
@@ -433,15 +449,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
             f2_unpack(f2_mul(f2_pack(pr[j], pr[j + 1]),
                              f2_add(f2_pack(__uint_as_float(a0), __uint_as_float(a1)), f2_pack(nd.x, nd.y))), d0, d1);
             dw[c] = pack_bf16x2(d0, d1);
-            pc[c] = pw[16 * ch + c];
           }
-          tmem_st16(tY + lane_off + 64 * wg + 32 * ch, pc);
           tmem_st16(tY + lane_off + 64 * wg + 32 * ch + 16, dw);
         }
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->pd_ready);
+      mbar_arrive(&bars->ds_ready);
     }
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
