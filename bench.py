@@ -37,6 +37,55 @@ METRIC = "causal attn TFLOP/s fwd & fwd+bwd (% bf16 peak); re-layout GB/s (% HBM
 DEFAULT_WORKLOAD = "llama8b_p4_n32k"
 
 
+# DRAM traffic per launch of the dominant kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum; the capture's command and
+# figures are in the profile named).  It applies only while the kernel's
+# sources hash to the value recorded with it; otherwise traffic is null.
+KERNEL_SOURCES = ("ulysses_head_attention_b200/csrc/attn_bwd.cu", "ulysses_head_attention_b200/csrc/sm100.cuh",
+                  "ulysses_head_attention_b200/csrc/common.cuh")
+TRAFFIC = {}   # kernel name -> {"sources_sha256": ..., "bytes_per_launch": ..., "profile": ...}
+
+
+def sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str):
+    rec = TRAFFIC.get(kernel)
+    if rec is None or rec["sources_sha256"] != sources_sha256():
+        return None
+    return rec["bytes_per_launch"]
+
+
+# ----------------------------------------------------------------------------- multi-rank plumbing
+def max_over_ranks(val: float, world: int, device=None) -> float:
+    """Max of `val` over all ranks of the default process group (identity at world 1).
+    NCCL groups need `device` (the rank's GPU); gloo groups take the CPU default."""
+    if world == 1:
+        return float(val)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(val)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job rate: every rank runs its own copy of the step (weak scaling),
+    and the step time is the slowest rank's."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
+def reports(rank: int) -> bool:
+    """Only rank 0 prints the JSON line."""
+    return rank == 0
+
+
 def pairs_of(lengths):
     return sum(L * (L + 1) // 2 for row in lengths for L in row)
 
@@ -133,7 +182,7 @@ def oracle_sample(w, x, rows: int, heads: int):
 
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if not reports(rank):   # the oracle runs on rank 0 only; other ranks exit without work
         return 0
     x = synthetic.make_inputs(w)
     rows, heads = 512, 2
@@ -206,12 +255,13 @@ def run_ours(args, w):
     ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, uly.ULY_F32), dev)
     stream = torch.cuda.current_stream()
     # s2h x3; fwd: segments + attn_fwd; h2s O; s2h dO; bwd: segments + bwd_pre + bwd_dkdv + bwd_dq; h2s x3
+    # (the event records inside the timed backward are not kernels)
     launches_per_step = 3 + 2 + 1 + 1 + 4 + 3
 
     relayout_bytes = 2 * sum(t.numel() * t.element_size() for t in (seq["q"], seq["k"], seq["v"], seq["do"]))
     relayout_bytes += 2 * sum(t.numel() * t.element_size() for t in (o_seq, g_seq["q"], g_seq["k"], g_seq["v"]))
 
-    def step(ev=None):
+    def step(ev=None, kev=None):
         if ev is not None:
             ev[0].record(stream)
         for k in ("q", "k", "v"):
@@ -225,8 +275,12 @@ def run_ours(args, w):
         uly.ulysses_seq_to_head(seq["do"], head["do"])
         if ev is not None:
             ev[3].record(stream)
-        uly.ulysses_attn_bwd(head["q"], head["k"], head["v"], o_head, lse, head["do"], pos,
-                             g_head["q"], g_head["k"], g_head["v"], ws_b)
+        if kev is not None:   # the same call, with events around its four kernels
+            uly.ulysses_attn_bwd_timed(head["q"], head["k"], head["v"], o_head, lse, head["do"], pos,
+                                       g_head["q"], g_head["k"], g_head["v"], ws_b, kev)
+        else:
+            uly.ulysses_attn_bwd(head["q"], head["k"], head["v"], o_head, lse, head["do"], pos,
+                                 g_head["q"], g_head["k"], g_head["v"], ws_b)
         if ev is not None:
             ev[4].record(stream)
         for k in ("q", "k", "v"):
@@ -245,15 +299,9 @@ def run_ours(args, w):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(val):
-        if world == 1:
-            return val
-        t = torch.tensor([val], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ---- device-timed region: K steps, inputs resident in HBM
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -262,23 +310,32 @@ def run_ours(args, w):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(evs[i], kevs[i])
     end.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    ms_total = max_over_ranks(start.elapsed_time(end))
+    ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
     ms_step = ms_total / args.steps
     stage = {"s2h_qkv": [], "attn_fwd": [], "h2s_o_s2h_do": [], "attn_bwd": [], "h2s_grads": []}
     for e in evs:
         for k, (a, bnd) in zip(stage, ((0, 1), (1, 2), (2, 3), (3, 4), (4, 5))):
             stage[k].append(e[a].elapsed_time(e[bnd]))
     st_ms = {k: statistics.mean(v) for k, v in stage.items()}
+    # per-kernel device time inside the backward call (events on the launching stream)
+    k_ms = {"attn_bwd_dkdv_kernel": statistics.mean(e[2].elapsed_time(e[3]) for e in kevs),
+            "attn_bwd_dq_kernel": statistics.mean(e[3].elapsed_time(e[4]) for e in kevs),
+            "bwd_pre_kernel": statistics.mean(e[1].elapsed_time(e[2]) for e in kevs)}
+    # algorithmic flops per launch: dK/dV runs S, dP, dV, dK (4 products of 2*d flops
+    # per visible pair); dQ runs S, dP, dQ (3)
+    k_flops = {"attn_bwd_dkdv_kernel": 8 * d * hq * pairs, "attn_bwd_dq_kernel": 6 * d * hq * pairs}
+    dom = max(k_flops, key=lambda kname: k_ms[kname])
+    dom_tf = k_flops[dom] / (k_ms[dom] * 1e-3) / 1e12
     for ws in (ws_f, ws_b):
         if uly.ulysses_workspace_status(ws) != 0:
             raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
 
-    value = world * (fwd_flops + bwd_flops) / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, fwd_flops + bwd_flops, ms_step)
     fwd_tf = fwd_flops / (st_ms["attn_fwd"] * 1e-3) / 1e12
     bwd_tf = bwd_flops / (st_ms["attn_bwd"] * 1e-3) / 1e12
     relayout_ms = st_ms["s2h_qkv"] + st_ms["h2s_o_s2h_do"] + st_ms["h2s_grads"]
@@ -312,8 +369,8 @@ def run_ours(args, w):
     e2.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(s2.elapsed_time(e2)) / args.steps
-    e2e_value = world * (fwd_flops + bwd_flops) / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, dev) / args.steps
+    e2e_value = whole_job_tflops(world, fwd_flops + bwd_flops, e2e_ms)
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -328,13 +385,16 @@ def run_ours(args, w):
             "attn_bwd_tflops": bwd_tf, "attn_bwd_frac": bwd_tf / peak_t,
             "attn_fwd_bwd_tflops": (fwd_flops + bwd_flops) / ((st_ms["attn_fwd"] + st_ms["attn_bwd"]) * 1e-3) / 1e12,
             "relayout_gbs": relayout_gbs, "relayout_frac": relayout_gbs / peaks["hbm_gbs"],
-            "stage_ms": st_ms, "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
+            "stage_ms": st_ms, "bwd_kernel_ms": k_ms,
+            "bwd_kernel_tflops": {kname: k_flops[kname] / (k_ms[kname] * 1e-3) / 1e12 for kname in k_flops},
+            "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
             "bwd_flops_with_recompute_convention": 10 * d * hq * pairs,
             "peaks": peaks,
         },
-        "roofline": {"bound": "tensor", "kernel": "attn_bwd: one ulysses_attn_bwd call (segments, bwd_pre, bwd_dkdv, bwd_dq kernels)",
-                     "achieved": bwd_tf, "peak": peak_t, "unit": "TFLOP/s", "frac": bwd_tf / peak_t,
-                     "peak_kind": f"bf16_tflops_sustained ({peaks['source']})", "traffic": None},
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": dom_tf / peak_t, "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                     "flops_per_launch": k_flops[dom], "ms_per_launch": k_ms[dom],
+                     "traffic": recorded_traffic(dom)},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
@@ -350,7 +410,7 @@ def run_ours(args, w):
         out["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
                                "kind": "oracle",
                                "sample": f"4 x oracle fwd+bwd of the last {rows} query rows of {heads} heads"}
-    if rank == 0:
+    if reports(rank):
         print(json.dumps(out))
     if world > 1:
         dist.destroy_process_group()

@@ -144,6 +144,25 @@ uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* 
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ulysses_attn_bwd_timed -- ulysses_attn_bwd that also records five
+ * caller-owned CUDA events on `stream` around its kernels, for measuring
+ * each kernel's device time (the pages have no counterpart; this is
+ * instrumentation).  events[0] before the sample-table kernel, events[1]
+ * before the row-statistics kernel, events[2] before the dK/dV kernel,
+ * events[3] before the dQ kernel, events[4] after it.  `events` points to
+ * five cudaEvent_t handles (as void*), created by the caller on the current
+ * device; a null array or a null handle returns ULY_ERR_INVALID_ARG and
+ * enqueues nothing.  A failed record returns ULY_ERR_CUDA.  All other
+ * arguments, results and errors are those of ulysses_attn_bwd.
+ */
+uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_head, const void* v_head,
+                                  const void* o_head, uly_dtype o_dtype, const float* lse,
+                                  const void* do_head, const int64_t* position_ids,
+                                  const uly_shape* shape, int32_t rank, float softmax_scale,
+                                  void* dq_head, void* dk_head, void* dv_head, uly_dtype g_dtype,
+                                  void* ws, size_t ws_bytes, void* stream, void* const* events);
+
+/*
  * ulysses_attn_fwd_noalloc -- ulysses_attn_fwd without a caller workspace.
  * The pages have no counterpart for this call; it exists for callers that
  * cannot allocate device memory themselves: code that runs under a framework

@@ -106,3 +106,15 @@ def test_workspace_queries_reject_bad_shapes():
     assert uly.ulysses_attn_fwd_workspace(shape(n=1001)) == 0
     assert uly.ulysses_attn_bwd_workspace(shape(P=3), 1) == 0
     assert uly.ulysses_attn_fwd_workspace(shape()) >= 256 + 2 * 4 * 1024
+
+
+def test_timed_backward_rejects_missing_events():
+    """The event array is checked before anything else: null array or null handle."""
+    import ulysses_head_attention_b200 as uly
+    s = shape()
+    G = 1 << 30
+    args = (F, F + G, F + 2 * G, F + 3 * G, 1, F + 4 * G, F + 5 * G, F + 6 * G, ctypes.byref(s), -1, 0.0,
+            F + 7 * G, F + 8 * G, F + 9 * G, 1, F + 10 * G, 1 << 24, None)
+    assert uly.lib.ulysses_attn_bwd_timed(*args, None) == INVALID
+    events = (ctypes.c_void_p * 5)(1, 2, 0, 4, 5)
+    assert uly.lib.ulysses_attn_bwd_timed(*args, events) == INVALID

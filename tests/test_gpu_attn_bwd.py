@@ -117,3 +117,36 @@ def test_bwd_column_sums(cuda_device):
         for g in range(dv.shape[3]):
             want = do[r, 0, :, g * G:(g + 1) * G].sum(axis=(0, 1))
             assert np.abs(dv[r, 0, :, g].sum(axis=0) - want).max() <= 1e-3 * max(1.0, np.abs(want).max())
+
+
+def test_bwd_timed_matches_untimed(cuda_device):
+    """The event-recording entry point computes exactly what ulysses_attn_bwd
+    does, and its five events bracket four kernels in order."""
+    uly = _uly()
+    P = 2
+    x = synthetic.custom_inputs(seed=41, b=1, n=512, h_q=4, h_kv=2, d=128, lengths=[[200, 312]], with_do=True)
+    heads = [head_layout(x[k], P) for k in ("q", "k", "v", "do")]
+    q, k, v, do = (to_dev_bf16(t, cuda_device) for t in heads)
+    pos = torch.from_numpy(x["position_ids"]).to(cuda_device)
+    shape = uly.make_shape(1, 512, 4, 2, 128, P)
+    o = torch.empty((P, 1, 512, 2, 128), dtype=torch.float32, device=cuda_device)
+    lse = torch.empty((P, 1, 2, 512), dtype=torch.float32, device=cuda_device)
+    ws_f = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(shape), cuda_device)
+    uly.ulysses_attn_fwd(q, k, v, pos, o, lse, ws_f)
+    ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, uly.ULY_F32), cuda_device)
+    outs = []
+    for timed in (False, True):
+        g = [torch.empty(t.shape, dtype=torch.float32, device=cuda_device) for t in (q, k, v)]
+        if timed:
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            uly.ulysses_attn_bwd_timed(q, k, v, o, lse, do, pos, *g, ws_b, evs)
+            torch.cuda.synchronize()
+            gaps = [evs[i].elapsed_time(evs[i + 1]) for i in range(4)]
+            assert all(t >= 0.0 for t in gaps)
+            assert gaps[2] > 0.0 and gaps[3] > 0.0
+        else:
+            uly.ulysses_attn_bwd(q, k, v, o, lse, do, pos, *g, ws_b)
+        assert uly.ulysses_workspace_status(ws_b) == 0
+        outs.append([t.cpu() for t in g])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)

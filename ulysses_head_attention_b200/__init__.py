@@ -29,8 +29,8 @@ STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED",
                 4: "ULY_ERR_WORKSPACE", 5: "ULY_ERR_TIMEOUT"}
 # Every symbol include/ulysses.h declares.
 EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
-           "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_fwd_noalloc", "ulysses_workspace_status",
-           "ulysses_status_string")
+           "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_bwd_timed", "ulysses_attn_fwd_noalloc",
+           "ulysses_workspace_status", "ulysses_status_string")
 
 
 class UlyShape(ctypes.Structure):
@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
         "ulysses_attn_fwd": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp, sz, vp], i32),
         "ulysses_attn_bwd_workspace": ([shp, i32], sz),
         "ulysses_attn_bwd": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i32, f32, vp, vp, vp, i32, vp, sz, vp], i32),
+        "ulysses_attn_bwd_timed": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i32, f32, vp, vp, vp, i32, vp, sz, vp,
+                                    ctypes.POINTER(vp)], i32),
         "ulysses_attn_fwd_noalloc": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp], i32),
         "ulysses_workspace_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "ulysses_status_string": ([i32], ctypes.c_char_p),
@@ -191,6 +193,30 @@ def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse, do_head, position_ids,
                                 _dev(dv_head, "dv_head"), _dtype_code(dq_head), _dev(ws, "ws"),
                                 ws.numel() * ws.element_size(), _stream(stream)),
            "ulysses_attn_bwd")
+
+
+def ulysses_attn_bwd_timed(q_head, k_head, v_head, o_head, lse, do_head, position_ids, dq_head, dk_head, dv_head,
+                           ws, events, rank: int = -1, softmax_scale: float = 0.0, stream=None) -> None:
+    """ulysses_attn_bwd that also records five torch.cuda.Events around its
+    kernels (before sample tables, statistics, dK/dV, dQ; after dQ)."""
+    if len(events) != 5:
+        raise ValueError("five events are needed")
+    shape = _attn_shape(q_head, k_head)
+    if dk_head.dtype != dq_head.dtype or dv_head.dtype != dq_head.dtype:
+        raise TypeError("dq/dk/dv must share one dtype")
+    handles = []
+    for ev in events:
+        if ev.cuda_event == 0:   # torch creates the handle lazily, at the first record
+            ev.record(torch.cuda.current_stream() if stream is None else stream)
+        handles.append(ev.cuda_event)
+    arr = (ctypes.c_void_p * 5)(*handles)
+    _check(lib.ulysses_attn_bwd_timed(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
+                                      _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
+                                      _dev(do_head, "do_head"), _dev(position_ids, "position_ids"),
+                                      ctypes.byref(shape), rank, softmax_scale, _dev(dq_head, "dq_head"),
+                                      _dev(dk_head, "dk_head"), _dev(dv_head, "dv_head"), _dtype_code(dq_head),
+                                      _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream), arr),
+           "ulysses_attn_bwd_timed")
 
 
 def ulysses_workspace_status(ws: torch.Tensor, stream=None) -> int:

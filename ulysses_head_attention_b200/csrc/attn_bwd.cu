@@ -811,11 +811,13 @@ extern "C" size_t ulysses_attn_bwd_workspace(const uly_shape* s, uly_dtype g_dty
   return bwd_ws_stats_off(s) + size_t(s->b) * size_t(s->h_q) * size_t(bwd_n_pad(s->n)) * 8;
 }
 
-extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* v_head, const void* o_head,
-                                       uly_dtype o_dtype, const float* lse, const void* do_head,
-                                       const int64_t* position_ids, const uly_shape* shape, int32_t rank,
-                                       float softmax_scale, void* dq_head, void* dk_head, void* dv_head,
-                                       uly_dtype g_dtype, void* ws, size_t ws_bytes, void* stream) {
+// events: null, or five caller-owned cudaEvent_t recorded on the stream
+// before the segment-table, statistics, dK/dV and dQ kernels and after dQ.
+static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const void* v_head, const void* o_head,
+                                uly_dtype o_dtype, const float* lse, const void* do_head, const int64_t* position_ids,
+                                const uly_shape* shape, int32_t rank, float softmax_scale, void* dq_head,
+                                void* dk_head, void* dv_head, uly_dtype g_dtype, void* ws, size_t ws_bytes,
+                                void* stream, void* const* events) {
   uly_status st = validate_attn(q_head, k_head, v_head, position_ids, shape, rank, ws, ws_bytes,
                                 shape ? ulysses_attn_bwd_workspace(shape, g_dtype) : 0);
   if (st != ULY_OK) return st;
@@ -855,8 +857,11 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
   float* stats = reinterpret_cast<float*>(wsb + bwd_ws_stats_off(&s));
   const int64_t n_pad = bwd_n_pad(s.n);
 
+  auto mark = [&](int i) { return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), cs) == cudaSuccess; };
+  if (!mark(0)) return ULY_ERR_CUDA;
   cudaError_t e = launch_segments(position_ids, segstart, segend, s.b, s.n, cs);
   if (e != cudaSuccess) return ULY_ERR_CUDA;
+  if (!mark(1)) return ULY_ERR_CUDA;
 
   const int64_t P_sel = rank < 0 ? s.P : 1;
   const int64_t rank0 = rank < 0 ? 0 : rank;
@@ -879,6 +884,7 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
   }
 
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(float(s.d));
+  if (!mark(2)) return ULY_ERR_CUDA;
   // ---- dK, dV
   {
     bwd::dkdv::Params p;
@@ -914,6 +920,7 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
     }
     if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
+  if (!mark(3)) return ULY_ERR_CUDA;
   // ---- dQ
   {
     bwd::dq::Params p;
@@ -948,5 +955,28 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
     }
     if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
+  if (!mark(4)) return ULY_ERR_CUDA;
   return ULY_OK;
+}
+
+extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* v_head, const void* o_head,
+                                       uly_dtype o_dtype, const float* lse, const void* do_head,
+                                       const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                                       float softmax_scale, void* dq_head, void* dk_head, void* dv_head,
+                                       uly_dtype g_dtype, void* ws, size_t ws_bytes, void* stream) {
+  return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
+                       softmax_scale, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, nullptr);
+}
+
+extern "C" uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_head, const void* v_head,
+                                             const void* o_head, uly_dtype o_dtype, const float* lse,
+                                             const void* do_head, const int64_t* position_ids,
+                                             const uly_shape* shape, int32_t rank, float softmax_scale,
+                                             void* dq_head, void* dk_head, void* dv_head, uly_dtype g_dtype,
+                                             void* ws, size_t ws_bytes, void* stream, void* const* events) {
+  if (!events) return ULY_ERR_INVALID_ARG;
+  for (int i = 0; i < 5; ++i)
+    if (!events[i]) return ULY_ERR_INVALID_ARG;
+  return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
+                       softmax_scale, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, events);
 }
