@@ -7,6 +7,7 @@ seq_to_head(dO) -> attention backward -> head_to_seq(dQ, dK, dV).
 Outputs are stored fp32 (the precision the parity tests gate).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --profile-case      # one small fwd + bwd for ncu captures
 
 `value` is the algorithmic fwd+bwd attention FLOP rate of the whole step
 (12 * d * H_q * pairs per step, pairs = sum over samples of L(L+1)/2, i.e.
@@ -41,23 +42,36 @@ DEFAULT_WORKLOAD = "llama8b_p4_n32k"
 # (dram__bytes_read.sum + dram__bytes_write.sum; the capture's command and
 # figures are in the profile named).  It applies only while the kernel's
 # sources hash to the value recorded with it; otherwise traffic is null.
-KERNEL_SOURCES = ("ulysses_head_attention_b200/csrc/attn_bwd.cu", "ulysses_head_attention_b200/csrc/sm100.cuh",
-                  "ulysses_head_attention_b200/csrc/common.cuh")
-TRAFFIC = {}   # kernel name -> {"sources_sha256": ..., "bytes_per_launch": ..., "profile": ...}
+KERNEL_SOURCES = {
+    # kernel -> (file, first line of its source region or None for the whole file, ...)
+    "attn_bwd_dkdv_kernel": (("ulysses_head_attention_b200/csrc/attn_bwd.cu", "namespace dkdv {", "}  // namespace dkdv"),
+                             ("ulysses_head_attention_b200/csrc/sm100.cuh", None, None),
+                             ("ulysses_head_attention_b200/csrc/common.cuh", None, None)),
+}
+# llama8b_p4_n32k, one launch (ncu, dram__bytes_read.sum 4.28 GB + dram__bytes_write.sum 246.83 MB,
+# as ncu printed them); see profiles/attn_bwd_dkdv_kernel.md
+TRAFFIC = {
+    "attn_bwd_dkdv_kernel": {"workload": "llama8b_p4_n32k", "bytes_per_launch": 4.28e9 + 246.83e6,
+                             "sources_sha256": "f8604d95571327241bbb0f8de753d89c5727e5512e23054c983a3c7c5fbe4b43"},
+}
 
 
-def sources_sha256() -> str:
+def sources_sha256(kernel: str) -> str:
+    """Hash of the kernel's own source region and the headers it uses."""
     import hashlib
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+    for rel, begin, end in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            text = f.read()
+        if begin is not None:
+            text = text[text.index(begin):text.index(end)]
+        h.update(text.encode())
     return h.hexdigest()
 
 
-def recorded_traffic(kernel: str):
+def recorded_traffic(kernel: str, workload: str):
     rec = TRAFFIC.get(kernel)
-    if rec is None or rec["sources_sha256"] != sources_sha256():
+    if rec is None or rec["workload"] != workload or rec["sources_sha256"] != sources_sha256(kernel):
         return None
     return rec["bytes_per_launch"]
 
@@ -394,7 +408,7 @@ def run_ours(args, w):
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": dom_tf / peak_t, "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
                      "flops_per_launch": k_flops[dom], "ms_per_launch": k_ms[dom],
-                     "traffic": recorded_traffic(dom)},
+                     "traffic": recorded_traffic(dom, w.name)},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
@@ -417,6 +431,41 @@ def run_ours(args, w):
     return 0
 
 
+# ----------------------------------------------------------------------------- profiling case
+def run_profile_case():
+    """One forward + one backward on a small case for ncu captures: P = 4,
+    b = 1, n = 16384, H_q = 32, H_kv = 8, d = 128, one causal sample,
+    virtual rank 0 only (its 8 query heads), standard-normal bf16 inputs
+    drawn on the device (seed 0).  Each tensor is above L2's size, the
+    device holds well under 1 GB.  Times nothing."""
+    import torch
+    import ulysses_head_attention_b200 as uly
+    dev = torch.device("cuda:0")
+    P, b, n, hq, hkv, d = 4, 1, 16384, 32, 8, 128
+    g = torch.Generator(device=dev).manual_seed(0)
+
+    def mk(h):
+        return torch.randn((P, b, n, h // P, d), device=dev, generator=g).to(torch.bfloat16)
+
+    q, k, v, do = mk(hq), mk(hkv), mk(hkv), mk(hq)
+    pos = torch.arange(n, device=dev).view(1, n)
+    o = torch.empty((P, b, n, hq // P, d), dtype=torch.float32, device=dev)
+    lse = torch.empty((P, b, hq // P, n), dtype=torch.float32, device=dev)
+    shape = uly.make_shape(b, n, hq, hkv, d, P)
+    wf = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(shape), dev)
+    wb = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, uly.ULY_F32), dev)
+    dq = torch.empty_like(o)
+    dk = torch.empty((P, b, n, hkv // P, d), device=dev)
+    dv = torch.empty((P, b, n, hkv // P, d), device=dev)
+    uly.ulysses_attn_fwd(q, k, v, pos, o, lse, wf, rank=0)
+    uly.ulysses_attn_bwd(q, k, v, o, lse, do, pos, dq, dk, dv, wb, rank=0)
+    torch.cuda.synchronize()
+    if uly.ulysses_workspace_status(wf) != 0 or uly.ulysses_workspace_status(wb) != 0:
+        raise RuntimeError("a kernel reported a pipeline timeout")
+    print("profile case done")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -425,7 +474,11 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="run one small forward + backward for an ncu capture, then exit (no timing, no JSON)")
     args = ap.parse_args()
+    if args.profile_case:
+        return run_profile_case()
     w = synthetic.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
