@@ -33,8 +33,11 @@
  *    void* so this header needs no CUDA header.
  *  - Calls only enqueue work on `stream` and return; results are valid once
  *    the stream has run.  Outputs are fully overwritten.  The library
- *    allocates no device memory and keeps no mutable global state; scratch
- *    space is the caller's workspace, sized by the *_workspace queries.
+ *    allocates no device memory; scratch space is the caller's workspace,
+ *    sized by the *_workspace queries.  The only mutable global state is
+ *    ulysses_attn_fwd_noalloc's fixed per-GPU scratch array (see there),
+ *    plus caches of looked-up addresses (that array's per device, and the
+ *    driver's tensor-map encoder), filled once.
  *  - Errors: every argument is checked on the host before anything is
  *    launched; a bad argument returns ULY_ERR_INVALID_ARG (or
  *    ULY_ERR_UNSUPPORTED for a valid but unimplemented size/type) and
