@@ -16,7 +16,11 @@ Pages followed (cited by title and section):
   [BLOG]     "Ulysses Sequence Parallelism: Training with Million-Token
              Contexts": "How Ulysses works" steps 1-6 (sharding, all-to-all,
              local attention, inverse all-to-all; heads are independent);
-             "Communication complexity"; the position_ids masking paragraph.
+             "Communication complexity"; the position_ids masking paragraph;
+             "Loss aggregation".
+  [ACC-SP] also: the custom training loop's weighted per-rank loss
+             aggregation (labels -100 excluded, zero-token ranks skipped,
+             division by max(total, 1)).
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against something
 other than itself (brute force, closed forms, a library routine, finite

@@ -18,6 +18,10 @@ What is computed, step by step, and where the pages define it:
   5. Backward: the gradient of the attention with respect to q, k, v
      (training through the layer, [ACC-SP] custom training loop); the
      gradient of a re-layout is the inverse re-layout.
+  6. Weighted loss aggregation across the SP ranks -- [ACC-SP] custom
+     training loop (each rank's loss weighted by its count of labels other
+     than -100; ranks without such labels skipped; divided by
+     max(total count, 1)) and [BLOG] "Loss aggregation".
 
 Readings taken where the pages are silent (each pinned by a test):
   * softmax scale = 1/sqrt(d) unless given ("standard attention");
@@ -30,6 +34,10 @@ Readings taken where the pages are silent (each pinned by a test):
   * after the first all-to-all, rank j's chunk lands at positions
     [j*n/P, (j+1)*n/P), and a rank's heads keep ascending global order;
   * LSE is the natural-log log-sum-exp of the scaled scores, per row.
+  * loss aggregation: the gradient returned is the derivative of the
+    aggregated loss with respect to each rank's loss (good_r / max(G, 1) for
+    a rank with good tokens, 0 for one without); how a framework then scales
+    gradients across ranks is outside the path.
 
 Arrays: unsharded tensors are [b][n][H][d]; seq-sharded [P][b][n/P][H][d];
 head-sharded [P][b][n][H/P][d]; LSE of head-sharded attention [P][b][H_q/P][n].
@@ -53,6 +61,7 @@ __all__ = [
     "ulysses_attn_fwd", "ulysses_attn_bwd",
     "ulysses_layer_fwd", "ulysses_layer_bwd",
     "default_scale",
+    "sp_good_tokens", "sp_loss_aggregate",
 ]
 
 
@@ -494,3 +503,43 @@ def ulysses_layer_bwd(q_seq, k_seq, v_seq, do_seq, position_ids, P: int,
                                   seq_to_head(v_seq, P), seq_to_head(do_seq, P),
                                   position_ids, P, scale)
     return head_to_seq(dQ, P), head_to_seq(dK, P), head_to_seq(dV, P)
+
+
+# --------------------------------------------------------------------------
+# Weighted SP loss aggregation
+# --------------------------------------------------------------------------
+def sp_good_tokens(shift_labels: np.ndarray, ignore_index: int = -100) -> np.ndarray:
+    """Per-rank count of labels that take part in the loss ([ACC-SP] custom
+    training loop: tokens labelled -100 are excluded).  shift_labels is
+    seq-sharded, [P][b][n/P] (int); returns int64[P]."""
+    lab = np.asarray(shift_labels)
+    P = lab.shape[0]
+    counts = np.zeros(P, dtype=np.int64)
+    for r in range(P):
+        counts[r] = int(np.count_nonzero(lab[r] != ignore_index))
+    return counts
+
+
+def sp_loss_aggregate(losses: np.ndarray, shift_labels: np.ndarray,
+                      ignore_index: int = -100) -> Tuple[float, np.ndarray, np.ndarray]:
+    """Weighted aggregation of the P per-rank losses ([ACC-SP] custom training
+    loop; [BLOG] "Loss aggregation").
+
+    total = sum over ranks r with good_r > 0 of loss_r * good_r (ranks
+    without good tokens are skipped, so a NaN loss there cannot leak in);
+    G = sum_r good_r; loss = total / max(G, 1).
+    Returns (loss, good[P], dloss/dloss_r[P])."""
+    losses = np.asarray(losses, dtype=np.float64)
+    good = sp_good_tokens(shift_labels, ignore_index)
+    P = losses.shape[0]
+    total = 0.0
+    for r in range(P):
+        if good[r] > 0:
+            total += losses[r] * float(good[r])
+    denom = float(max(int(good.sum()), 1))
+    loss = total / denom
+    grad = np.zeros(P, dtype=np.float64)
+    for r in range(P):
+        if good[r] > 0:
+            grad[r] = float(good[r]) / denom
+    return loss, good, grad
