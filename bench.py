@@ -386,6 +386,30 @@ def run_ours(args, w):
     e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, dev) / args.steps
     e2e_value = whole_job_tflops(world, fwd_flops + bwd_flops, e2e_ms)
 
+    # ---- weighted SP loss aggregation (the custom training loop's per-rank loss
+    # weighting), timed on its own: it needs a model's per-rank losses, which
+    # this path does not produce, so it is not part of the step
+    lab = synthetic.sft_shift_labels(w.wid, x["lengths"])
+    lab_sh = torch.from_numpy(np.ascontiguousarray(lab.reshape(b, P, m).transpose(1, 0, 2))).to(dev)
+    l_in = torch.from_numpy(synthetic.rank_losses(w.wid, P)).to(dev)
+    l_out, l_good, l_dl = (torch.empty(1, device=dev), torch.empty(P, dtype=torch.int64, device=dev),
+                           torch.empty(P, device=dev))
+    for _ in range(5):
+        uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
+    torch.cuda.synchronize()
+    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 50
+    s3.record(stream)
+    for _ in range(reps):
+        uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    loss_us = s3.elapsed_time(e3) * 1e3 / reps
+    loss_bytes = lab_sh.numel() * 8 + 3 * P * 8 + 4
+    loss_stat = {"us_per_call": loss_us, "bytes_per_call": loss_bytes,
+                 "gbs": loss_bytes / (loss_us * 1e-6) / 1e9, "launches_per_call": 2,
+                 "labels": "packed SFT: per sample a U[0.1, 0.6) prompt fraction and the last position are -100"}
+
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -404,6 +428,7 @@ def run_ours(args, w):
             "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
             "bwd_flops_with_recompute_convention": 10 * d * hq * pairs,
             "peaks": peaks,
+            "sp_loss_aggregate": loss_stat,
         },
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": dom_tf / peak_t, "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",

@@ -195,6 +195,35 @@ uly_status ulysses_attn_fwd_noalloc(const void* q_head, const void* k_head, cons
                                     void* stream);
 
 /*
+ * ulysses_sp_loss_aggregate -- weighted loss aggregation across the P SP
+ * ranks (Accelerate guide "Sequence parallelism", custom training loop: the
+ * differentiable weighted per-rank loss aggregation; blog "Ulysses Sequence
+ * Parallelism: Training with Million-Token Contexts", "Loss aggregation").
+ *   good[r]    = number of shift_labels of rank r that are not ignore_index
+ *                (the pages use -100);
+ *   *loss      = (sum over r with good[r] > 0 of losses[r] * good[r])
+ *                / max(sum_r good[r], 1);
+ *   dlosses[r] = d(*loss)/d(losses[r]) = good[r] / max(sum good, 1) if
+ *                good[r] > 0, else 0.
+ * A rank without valid labels is skipped, not multiplied by zero, so a NaN
+ * loss there does not reach the result.  Sums run in double precision in a
+ * fixed order (bitwise reproducible); *loss and dlosses are rounded to
+ * float once at the end.
+ *   losses        float[P], device, the per-rank losses.
+ *   shift_labels  int64 [P][b][n/P], device, seq-sharded like the inputs
+ *                 (rank r's b rows of n/P labels are contiguous).
+ *   loss          float[1], good int64[P], dlosses float[P]: device outputs,
+ *                 fully overwritten; none may overlap the inputs or each other.
+ * Errors: null pointer, P < 1 or P > 1024, b < 1, n < 1, n % P != 0,
+ * misalignment (4 bytes for float, 8 for int64) or overlap return
+ * ULY_ERR_INVALID_ARG and enqueue nothing; a failed launch ULY_ERR_CUDA.
+ * Two kernel launches on `stream`.
+ */
+uly_status ulysses_sp_loss_aggregate(const float* losses, const int64_t* shift_labels, int64_t b,
+                                     int64_t n, int32_t P, int64_t ignore_index, float* loss,
+                                     int64_t* good, float* dlosses, void* stream);
+
+/*
  * ulysses_workspace_status -- synchronizes `stream`, then reads and clears
  * the status word kept at the start of an attention workspace.  *code gets
  * ULY_OK, ULY_ERR_TIMEOUT when a kernel gave up waiting on one of its own

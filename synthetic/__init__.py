@@ -176,3 +176,31 @@ def custom_inputs(seed: int, b: int, n: int, h_q: int, h_kv: int, d: int,
     if with_do:
         out["do"] = draw(g["do"], (b, n, h_q, d))
     return out
+
+
+def sft_shift_labels(seed: int, lengths: List[List[int]], vocab: int = 128256,
+                     prompt_lo: float = 0.1, prompt_hi: float = 0.6) -> np.ndarray:
+    """shift_labels of packed SFT samples, int64 [b][n].
+
+    Per sample of length L: a prompt fraction f ~ U[prompt_lo, prompt_hi];
+    the first floor(f * L) positions and the sample's last position (it has
+    no next token) are -100, the rest are token ids ~ U[0, vocab).  Seeded
+    with SeedSequence(20261202 + 20000 + seed)."""
+    rng = np.random.default_rng(np.random.SeedSequence(SEED_BASE + 20_000 + seed))
+    rows = []
+    for ls in lengths:
+        parts = []
+        for L in ls:
+            lab = rng.integers(0, vocab, L, dtype=np.int64)
+            cut = int(np.floor(rng.uniform(prompt_lo, prompt_hi) * L))
+            lab[:cut] = -100
+            lab[L - 1] = -100
+            parts.append(lab)
+        rows.append(np.concatenate(parts))
+    return np.stack(rows)
+
+
+def rank_losses(seed: int, P: int) -> np.ndarray:
+    """P per-rank losses, float32 ~ U[0.5, 4)."""
+    rng = np.random.default_rng(np.random.SeedSequence(SEED_BASE + 30_000 + seed))
+    return rng.uniform(0.5, 4.0, P).astype(np.float32)

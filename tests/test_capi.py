@@ -118,3 +118,29 @@ def test_timed_backward_rejects_missing_events():
     assert uly.lib.ulysses_attn_bwd_timed(*args, None) == INVALID
     events = (ctypes.c_void_p * 5)(1, 2, 0, 4, 5)
     assert uly.lib.ulysses_attn_bwd_timed(*args, events) == INVALID
+
+
+@no_gpu
+@pytest.mark.parametrize("b,n,P,want", [
+    (1, 64, 0, INVALID),        # P < 1
+    (1, 64, 2048, INVALID),     # P > 1024
+    (1, 100, 8, INVALID),       # n % P
+    (0, 64, 4, INVALID),        # b < 1
+])
+def test_loss_aggregate_rejects_shapes(b, n, P, want):
+    import ulysses_head_attention_b200 as uly
+    G = 1 << 30
+    st = uly.lib.ulysses_sp_loss_aggregate(F, F + G, b, n, P, -100, F + 2 * G, F + 3 * G, F + 4 * G, None)
+    assert st == want
+
+
+@no_gpu
+def test_loss_aggregate_rejects_pointers():
+    import ulysses_head_attention_b200 as uly
+    G = 1 << 30
+    ok = [F, F + G, F + 2 * G, F + 3 * G, F + 4 * G]
+    for i, bad in ((0, 0), (1, F + G + 4), (3, F + 3 * G + 4), (4, F + G)):   # null, misaligned, overlap
+        args = list(ok)
+        args[i] = bad
+        st = uly.lib.ulysses_sp_loss_aggregate(args[0], args[1], 1, 64, 4, -100, args[2], args[3], args[4], None)
+        assert st == INVALID

@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED",
 # Every symbol include/ulysses.h declares.
 EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_bwd_timed", "ulysses_attn_fwd_noalloc",
-           "ulysses_workspace_status", "ulysses_status_string")
+           "ulysses_sp_loss_aggregate", "ulysses_workspace_status", "ulysses_status_string")
 
 
 class UlyShape(ctypes.Structure):
@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "ulysses_attn_bwd_timed": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i32, f32, vp, vp, vp, i32, vp, sz, vp,
                                     ctypes.POINTER(vp)], i32),
         "ulysses_attn_fwd_noalloc": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp], i32),
+        "ulysses_sp_loss_aggregate": ([vp, vp, i64, i64, i32, i64, vp, vp, vp, vp], i32),
         "ulysses_workspace_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "ulysses_status_string": ([i32], ctypes.c_char_p),
     }
@@ -217,6 +218,26 @@ def ulysses_attn_bwd_timed(q_head, k_head, v_head, o_head, lse, do_head, positio
                                       _dev(dk_head, "dk_head"), _dev(dv_head, "dv_head"), _dtype_code(dq_head),
                                       _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream), arr),
            "ulysses_attn_bwd_timed")
+
+
+def ulysses_sp_loss_aggregate(losses, shift_labels, loss, good, dlosses, ignore_index: int = -100,
+                              stream=None) -> None:
+    """Weighted aggregation of per-rank losses: losses float32[P], shift_labels
+    int64[P][b][n/P] (seq-sharded); writes loss float32[1], good int64[P],
+    dlosses float32[P]."""
+    if losses.dtype != torch.float32 or loss.dtype != torch.float32 or dlosses.dtype != torch.float32:
+        raise TypeError("losses, loss and dlosses must be float32")
+    if shift_labels.dtype != torch.int64 or good.dtype != torch.int64:
+        raise TypeError("shift_labels and good must be int64")
+    if shift_labels.dim() != 3:
+        raise ValueError("shift_labels must be [P][b][n/P]")
+    P, b, m = shift_labels.shape
+    if losses.numel() != P or good.numel() != P or dlosses.numel() != P or loss.numel() != 1:
+        raise ValueError("losses, good and dlosses need P elements, loss one")
+    _check(lib.ulysses_sp_loss_aggregate(_dev(losses, "losses"), _dev(shift_labels, "shift_labels"), b, m * P, P,
+                                         ignore_index, _dev(loss, "loss"), _dev(good, "good"),
+                                         _dev(dlosses, "dlosses"), _stream(stream)),
+           "ulysses_sp_loss_aggregate")
 
 
 def ulysses_workspace_status(ws: torch.Tensor, stream=None) -> int:
