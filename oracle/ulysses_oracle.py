@@ -34,6 +34,10 @@ Readings taken where the pages are silent (each pinned by a test):
   * after the first all-to-all, rank j's chunk lands at positions
     [j*n/P, (j+1)*n/P), and a rank's heads keep ascending global order;
   * LSE is the natural-log log-sum-exp of the scaled scores, per row.
+  * H_kv < P (GQA with fewer kv heads than ranks; the pages are silent): when
+    P is a multiple of H_kv, every rank r receives a copy of the one kv head
+    its query heads read, g(r) = r * H_kv // P; the gradient of that copy is
+    the sum over the ranks that hold it.
   * loss aggregation: the gradient returned is the derivative of the
     aggregated loss with respect to each rank's loss (good_r / max(G, 1) for
     a rank with good tokens, 0 for one without); how a framework then scales
@@ -53,6 +57,7 @@ import numpy as np
 __all__ = [
     "check_shape", "valid_sp_sizes",
     "shard", "unshard", "seq_to_head", "head_to_seq", "seq_to_head_window", "head_to_seq_window",
+    "kv_rank_head", "kv_seq_to_head", "kv_head_to_seq_reduce",
     "segment_ids", "segment_starts", "segment_ends", "allowed_matrix",
     "attention_brute_head", "attention_bwd_brute_head",
     "attention_fwd_head", "attention_bwd_head",
@@ -154,6 +159,52 @@ def head_to_seq(x_head: np.ndarray, P: int) -> np.ndarray:
     src_head = np.broadcast_to(g % h, (P, m, H))
     gathered = x_head[src_rank, :, src_tok, src_head]          # (P, m, H, b, d)
     return np.ascontiguousarray(gathered.transpose(0, 3, 1, 2, 4))
+
+
+def kv_rank_head(P: int, H_kv: int, r: int) -> int:
+    """The kv head rank r's query heads read when H_kv < P (P a multiple of
+    H_kv): rank r holds query heads [r*H_q/P, (r+1)*H_q/P), all inside group
+    r*H_kv//P of the GQA grouping h -> h // (H_q/H_kv)."""
+    return (r * H_kv) // P
+
+
+def kv_seq_to_head(x_seq: np.ndarray, P: int) -> np.ndarray:
+    """K/V re-layout for the attention.  H_kv a multiple of P: seq_to_head.
+    H_kv < P with P a multiple of H_kv: rank r receives all n positions of
+    its one kv head (reading above): x_head[r][bb][t][0] =
+    x_seq[t // (n/P)][bb][t % (n/P)][kv_rank_head(P, H_kv, r)]."""
+    Ps, b, m, H, d = x_seq.shape
+    if Ps != P:
+        raise ValueError("bad shape for P")
+    if H % P == 0:
+        return seq_to_head(x_seq, P)
+    if P % H:
+        raise ValueError("H_kv must divide P or be divisible by it")
+    n = m * P
+    out = np.empty((P, b, n, 1, d), dtype=x_seq.dtype)
+    for r in range(P):
+        g = kv_rank_head(P, H, r)
+        for t in range(0, n, m):
+            out[r, :, t:t + m, 0] = x_seq[t // m, :, :, g]
+    return out
+
+
+def kv_head_to_seq_reduce(x_head: np.ndarray, P: int, H_kv: int) -> np.ndarray:
+    """Gradient of kv_seq_to_head.  H_kv a multiple of P: head_to_seq.
+    Otherwise x_seq[s][bb][u][g] = sum over ranks r with kv_rank_head(r) == g
+    of x_head[r][bb][s*(n/P) + u][0]."""
+    if H_kv % P == 0:
+        return head_to_seq(x_head, P)
+    Ps, b, n, one, d = x_head.shape
+    if Ps != P or one != 1 or P % H_kv or n % P:
+        raise ValueError("bad shape for P, H_kv")
+    m = n // P
+    out = np.zeros((P, b, m, H_kv, d), dtype=np.float64)
+    for r in range(P):
+        g = kv_rank_head(P, H_kv, r)
+        for s_ in range(P):
+            out[s_, :, :, g] += x_head[r, :, s_ * m:(s_ + 1) * m, 0]
+    return out
 
 
 def seq_to_head_window(x_seq: np.ndarray, P: int, r: int, t_lo: int, t_hi: int) -> np.ndarray:
@@ -491,18 +542,19 @@ def ulysses_attn_bwd(q_head, k_head, v_head, do_head, position_ids, P: int,
 
 def ulysses_layer_fwd(q_seq, k_seq, v_seq, position_ids, P: int, scale: Optional[float] = None):
     """seq-sharded q, k, v -> seq_to_head -> local attention -> head_to_seq."""
-    O_head, lse = ulysses_attn_fwd(seq_to_head(q_seq, P), seq_to_head(k_seq, P),
-                                   seq_to_head(v_seq, P), position_ids, P, scale)
+    O_head, lse = ulysses_attn_fwd(seq_to_head(q_seq, P), kv_seq_to_head(k_seq, P),
+                                   kv_seq_to_head(v_seq, P), position_ids, P, scale)
     return head_to_seq(O_head, P), lse
 
 
 def ulysses_layer_bwd(q_seq, k_seq, v_seq, do_seq, position_ids, P: int,
                       scale: Optional[float] = None):
     """Backward of the layer: re-layout dO, local attention backward, re-layout back."""
-    dQ, dK, dV = ulysses_attn_bwd(seq_to_head(q_seq, P), seq_to_head(k_seq, P),
-                                  seq_to_head(v_seq, P), seq_to_head(do_seq, P),
+    H_kv = k_seq.shape[3]
+    dQ, dK, dV = ulysses_attn_bwd(seq_to_head(q_seq, P), kv_seq_to_head(k_seq, P),
+                                  kv_seq_to_head(v_seq, P), seq_to_head(do_seq, P),
                                   position_ids, P, scale)
-    return head_to_seq(dQ, P), head_to_seq(dK, P), head_to_seq(dV, P)
+    return head_to_seq(dQ, P), kv_head_to_seq_reduce(dK, P, H_kv), kv_head_to_seq_reduce(dV, P, H_kv)
 
 
 # --------------------------------------------------------------------------
