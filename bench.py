@@ -252,15 +252,16 @@ def run_ours(args, w):
     seq = {k: host[k].to(dev) for k in host}
     pos = host_pos.to(dev)
     bf, f32 = torch.bfloat16, torch.float32
+    hkv_r = hkv // P if hkv >= P else 1   # kv heads per rank (one replicated head when H_kv < P)
     head = {"q": torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev),
-            "k": torch.empty((P, b, n, hkv // P, d), dtype=bf, device=dev),
-            "v": torch.empty((P, b, n, hkv // P, d), dtype=bf, device=dev),
+            "k": torch.empty((P, b, n, hkv_r, d), dtype=bf, device=dev),
+            "v": torch.empty((P, b, n, hkv_r, d), dtype=bf, device=dev),
             "do": torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev)}
     o_head = torch.empty((P, b, n, hq // P, d), dtype=f32, device=dev)
     lse = torch.empty((P, b, hq // P, n), dtype=f32, device=dev)
     o_seq = torch.empty((P, b, m, hq, d), dtype=f32, device=dev)
-    g_head = {"q": torch.empty_like(o_head), "k": torch.empty((P, b, n, hkv // P, d), dtype=f32, device=dev),
-              "v": torch.empty((P, b, n, hkv // P, d), dtype=f32, device=dev)}
+    g_head = {"q": torch.empty_like(o_head), "k": torch.empty((P, b, n, hkv_r, d), dtype=f32, device=dev),
+              "v": torch.empty((P, b, n, hkv_r, d), dtype=f32, device=dev)}
     g_seq = {"q": torch.empty((P, b, m, hq, d), dtype=f32, device=dev),
              "k": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev),
              "v": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev)}
@@ -272,14 +273,17 @@ def run_ours(args, w):
     # (the event records inside the timed backward are not kernels)
     launches_per_step = 3 + 2 + 1 + 1 + 4 + 3
 
-    relayout_bytes = 2 * sum(t.numel() * t.element_size() for t in (seq["q"], seq["k"], seq["v"], seq["do"]))
-    relayout_bytes += 2 * sum(t.numel() * t.element_size() for t in (o_seq, g_seq["q"], g_seq["k"], g_seq["v"]))
+    # every re-layout reads its source once and writes its destination once
+    nbytes = lambda t: t.numel() * t.element_size()   # noqa: E731
+    relayout_bytes = sum(nbytes(seq[k]) + nbytes(head[k]) for k in ("q", "k", "v", "do"))
+    relayout_bytes += nbytes(o_head) + nbytes(o_seq) + sum(nbytes(g_head[k]) + nbytes(g_seq[k]) for k in g_seq)
 
     def step(ev=None, kev=None):
         if ev is not None:
             ev[0].record(stream)
-        for k in ("q", "k", "v"):
-            uly.ulysses_seq_to_head(seq[k], head[k])
+        uly.ulysses_seq_to_head(seq["q"], head["q"])
+        for k in ("k", "v"):   # plain re-layout, or one copied kv head per rank when H_kv < P
+            uly.ulysses_kv_seq_to_head(seq[k], head[k])
         if ev is not None:
             ev[1].record(stream)
         uly.ulysses_attn_fwd(head["q"], head["k"], head["v"], pos, o_head, lse, ws_f)
@@ -297,8 +301,9 @@ def run_ours(args, w):
                                  g_head["q"], g_head["k"], g_head["v"], ws_b)
         if ev is not None:
             ev[4].record(stream)
-        for k in ("q", "k", "v"):
-            uly.ulysses_head_to_seq(g_head[k], g_seq[k])
+        uly.ulysses_head_to_seq(g_head["q"], g_seq["q"])
+        for k in ("k", "v"):   # the copies' gradients are summed when H_kv < P
+            uly.ulysses_kv_head_to_seq(g_head[k], g_seq[k])
         if ev is not None:
             ev[5].record(stream)
 
@@ -416,7 +421,8 @@ def run_ours(args, w):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "P": P, "b": b, "n": n, "h_q": hq, "h_kv": hkv, "d": d,
                    "samples": sum(len(r) for r in x["lengths"]), "pairs": pairs,
-                   "outputs": "fp32", "l2": "inputs larger than L2 (q 256 MiB, dO 256 MiB per step)",
+                   "outputs": "fp32",
+                   "l2": f"inputs larger than L2 (q {nbytes(seq['q']) >> 20} MiB, dO {nbytes(seq['do']) >> 20} MiB per step)",
                    "parallelism": f"{world} independent replica(s), one per GPU"},
         "detail": {
             "attn_fwd_tflops": fwd_tf, "attn_fwd_frac": fwd_tf / peak_t,

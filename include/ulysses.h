@@ -28,6 +28,11 @@
  *                    and wherever position_ids[t] == 0.
  *  - GQA: query head h reads kv head h / (h_q/h_kv); ranks split both head
  *    counts contiguously, so each rank's query heads read its own kv heads.
+ *    With fewer kv heads than ranks (h_kv < P, P a multiple of h_kv; the
+ *    pages are silent on this case) each rank holds one kv head, the copy
+ *    of head r*h_kv/P its query heads read: k_head / v_head are then
+ *    [P][b][n][1][d], made by ulysses_kv_seq_to_head, and the gradients
+ *    dK / dV go back through ulysses_kv_head_to_seq, which sums the copies.
  *  - Pointers are device pointers owned by the caller, 16-byte aligned.
  *    `stream` is a cudaStream_t (NULL = legacy default stream), passed as
  *    void* so this header needs no CUDA header.
@@ -96,6 +101,33 @@ uly_status ulysses_seq_to_head(const void* x_seq, void* x_head, int64_t b, int64
 uly_status ulysses_head_to_seq(const void* x_head, void* x_seq, int64_t b, int64_t n, int64_t H,
                                int64_t d, int32_t P, uly_dtype dt, void* stream);
 
+/*
+ * ulysses_kv_seq_to_head -- the first all-to-all for K and V, for any kv head
+ * count the attention accepts.  H_kv a multiple of P: exactly
+ * ulysses_seq_to_head.  H_kv < P with P a multiple of H_kv: every rank r
+ * receives all n tokens of kv head g(r) = r*H_kv/P, the one its query heads
+ * read (a reading: the pages are silent on this case):
+ *   x_head[r][bb][t][0][:] = x_seq[t/(n/P)][bb][t%(n/P)][g(r)][:]
+ * x_seq [P][b][n/P][H_kv][d], x_head [P][b][n][1][d]; dt ULY_BF16 or ULY_F32;
+ * d * element size a multiple of 16 bytes for the replicating case.
+ * Errors: as ulysses_seq_to_head; H_kv neither a multiple nor a divisor of
+ * P returns ULY_ERR_INVALID_ARG.  Bit-exact copy.
+ */
+uly_status ulysses_kv_seq_to_head(const void* x_seq, void* x_head, int64_t b, int64_t n, int64_t H_kv,
+                                  int64_t d, int32_t P, uly_dtype dt, void* stream);
+
+/*
+ * ulysses_kv_head_to_seq -- the backward of ulysses_kv_seq_to_head, for dK
+ * and dV.  H_kv a multiple of P: exactly ulysses_head_to_seq.  H_kv < P: the
+ * sum of the copies,
+ *   x_seq[s][bb][u][g][:] = sum over r with g(r) == g, ascending, of
+ *                           x_head[r][bb][s*(n/P) + u][0][:]
+ * accumulated in float32 and rounded once to dt (bitwise reproducible).
+ * Same layouts and errors as ulysses_kv_seq_to_head.
+ */
+uly_status ulysses_kv_head_to_seq(const void* x_head, void* x_seq, int64_t b, int64_t n, int64_t H_kv,
+                                  int64_t d, int32_t P, uly_dtype dt, void* stream);
+
 /* Workspace bytes ulysses_attn_fwd needs for `shape` (0 on invalid shape). */
 size_t ulysses_attn_fwd_workspace(const uly_shape* shape);
 
@@ -108,7 +140,8 @@ size_t ulysses_attn_fwd_workspace(const uly_shape* shape);
  * and row i:  O_i = sum_j softmax_j(scale * q_i . k_j) v_j over keys j <= i
  * in i's sample;  LSE_i = log sum_j exp(scale * q_i . k_j).
  *   q_head [P][b][n][h_q/P][d] bf16, k_head / v_head [P][b][n][h_kv/P][d]
- *   bf16, position_ids [b][n] int64 (device).
+ *   bf16 ([P][b][n][1][d] when h_kv < P), position_ids [b][n] int64
+ *   (device).
  *   rank: -1 computes every rank; 0 <= rank < P computes only that rank's
  *   slice (rows of other ranks in o_head / lse are left untouched).
  *   softmax_scale <= 0 selects 1/sqrt(d).

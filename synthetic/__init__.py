@@ -53,7 +53,7 @@ class Workload:
         return self.h_q // self.h_kv
 
 
-# The five workloads, named by what they are.
+# The workloads, named by what they are.
 WORKLOADS: Dict[str, Workload] = {
     w.name: w for w in (
         Workload(1, "tiny_p2_n256", P=2, b=1, n=256, h_q=4, h_kv=4, d=64, backward=False),
@@ -62,6 +62,8 @@ WORKLOADS: Dict[str, Workload] = {
         Workload(4, "long_p8_n512k", P=8, b=1, n=524288, h_q=32, h_kv=8, d=128,
                  backward=False, rank_by_rank=True),
         Workload(5, "roundtrip_p4_n128k", P=4, b=1, n=131072, h_q=32, h_kv=8, d=128),
+        # more ranks than kv heads: each rank holds a copy of one kv head
+        Workload(6, "llama8b_p16_n32k_kvrep", P=16, b=1, n=32768, h_q=32, h_kv=8, d=128),
     )
 }
 

@@ -67,7 +67,8 @@ def shape(b=1, n=1024, hq=32, hkv=8, d=128, P=4):
 @no_gpu
 @pytest.mark.parametrize("kw,rank,want", [
     (dict(n=1000, P=16), -1, INVALID),       # n % P
-    (dict(hkv=8, P=16), -1, INVALID),        # H_kv % P
+    (dict(hkv=6, P=4, hq=24), -1, INVALID),  # H_kv neither a multiple nor a divisor of P
+    (dict(hkv=3, P=4, hq=12), -1, INVALID),  # H_kv < P but does not divide P
     (dict(hq=12, hkv=8, P=4), -1, INVALID),  # H_q % H_kv
     (dict(P=0), -1, INVALID),
     ({}, 4, INVALID),                        # rank out of range
@@ -144,3 +145,23 @@ def test_loss_aggregate_rejects_pointers():
         args[i] = bad
         st = uly.lib.ulysses_sp_loss_aggregate(args[0], args[1], 1, 64, 4, -100, args[2], args[3], args[4], None)
         assert st == INVALID
+
+
+@no_gpu
+@pytest.mark.parametrize("H,P,want", [
+    (3, 4, INVALID),      # neither a multiple nor a divisor of P
+    (6, 4, INVALID),
+    (2, 0, INVALID),
+])
+def test_kv_relayout_rejects(H, P, want):
+    import ulysses_head_attention_b200 as uly
+    for fn in (uly.lib.ulysses_kv_seq_to_head, uly.lib.ulysses_kv_head_to_seq):
+        assert fn(F, F + (1 << 30), 1, 64, H, 128, P, 0, None) == want
+
+
+@no_gpu
+def test_kv_relayout_rejects_unsupported_row_and_overlap():
+    import ulysses_head_attention_b200 as uly
+    for fn in (uly.lib.ulysses_kv_seq_to_head, uly.lib.ulysses_kv_head_to_seq):
+        assert fn(F, F + (1 << 30), 1, 64, 2, 4, 4, 0, None) == UNSUPPORTED      # d * 2 bytes not a multiple of 16
+        assert fn(F, F + 1024, 1, 64, 2, 128, 4, 0, None) == INVALID            # overlapping buffers

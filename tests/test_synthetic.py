@@ -36,4 +36,6 @@ def test_packed_lengths_recipe():
 
 def test_workload_table_obeys_divisibility():
     for w in synthetic.WORKLOADS.values():
-        assert w.n % w.P == 0 and w.h_q % w.P == 0 and w.h_kv % w.P == 0 and w.h_q % w.h_kv == 0
+        assert w.n % w.P == 0 and w.h_q % w.P == 0 and w.h_q % w.h_kv == 0
+        # kv heads: divisible by P, or (kv-head replication) a divisor of P
+        assert w.h_kv % w.P == 0 or (w.h_kv < w.P and w.P % w.h_kv == 0)

@@ -28,7 +28,7 @@ ULY_BF16, ULY_F32 = 0, 1
 STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED", 3: "ULY_ERR_CUDA",
                 4: "ULY_ERR_WORKSPACE", 5: "ULY_ERR_TIMEOUT"}
 # Every symbol include/ulysses.h declares.
-EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
+EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head", "ulysses_kv_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_bwd_timed", "ulysses_attn_fwd_noalloc",
            "ulysses_sp_loss_aggregate", "ulysses_workspace_status", "ulysses_status_string")
 
@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "ulysses_seq_to_head": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
         "ulysses_head_to_seq": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
+        "ulysses_kv_seq_to_head": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
+        "ulysses_kv_head_to_seq": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
         "ulysses_attn_fwd_workspace": ([shp], sz),
         "ulysses_attn_fwd": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp, sz, vp], i32),
         "ulysses_attn_bwd_workspace": ([shp, i32], sz),
@@ -124,6 +126,28 @@ def ulysses_head_to_seq(x_head: torch.Tensor, x_seq: torch.Tensor, stream=None) 
         raise ValueError("x_seq shape/dtype does not match x_head")
     _check(lib.ulysses_head_to_seq(_dev(x_head, "x_head"), _dev(x_seq, "x_seq"), b, n, h * P, d, P,
                                    _dtype_code(x_head), _stream(stream)), "ulysses_head_to_seq")
+
+
+def ulysses_kv_seq_to_head(x_seq: torch.Tensor, x_head: torch.Tensor, stream=None) -> None:
+    """K/V x_seq (P, b, n/P, H_kv, d) -> x_head (P, b, n, max(H_kv/P, 1), d); one
+    replicated kv head per rank when H_kv < P."""
+    P, b, m, H, d = x_seq.shape
+    h = H // P if H >= P else 1
+    if tuple(x_head.shape) != (P, b, m * P, h, d) or x_head.dtype != x_seq.dtype:
+        raise ValueError("x_head shape/dtype does not match x_seq")
+    _check(lib.ulysses_kv_seq_to_head(_dev(x_seq, "x_seq"), _dev(x_head, "x_head"), b, m * P, H, d, P,
+                                      _dtype_code(x_seq), _stream(stream)), "ulysses_kv_seq_to_head")
+
+
+def ulysses_kv_head_to_seq(x_head: torch.Tensor, x_seq: torch.Tensor, stream=None) -> None:
+    """dK/dV x_head (P, b, n, max(H_kv/P, 1), d) -> x_seq (P, b, n/P, H_kv, d);
+    the replicas are summed when H_kv < P."""
+    P, b, m, H, d = x_seq.shape
+    h = H // P if H >= P else 1
+    if tuple(x_head.shape) != (P, b, m * P, h, d) or x_head.dtype != x_seq.dtype:
+        raise ValueError("x_seq shape/dtype does not match x_head")
+    _check(lib.ulysses_kv_head_to_seq(_dev(x_head, "x_head"), _dev(x_seq, "x_seq"), b, m * P, H, d, P,
+                                      _dtype_code(x_seq), _stream(stream)), "ulysses_kv_head_to_seq")
 
 
 def _attn_shape(q_head: torch.Tensor, k_head: torch.Tensor) -> UlyShape:

@@ -827,7 +827,7 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
       !aligned(dk_head, 16) || !aligned(dv_head, 16))
     return ULY_ERR_INVALID_ARG;
   const uly_shape& s = *shape;
-  const int64_t hq = s.h_q / s.P, hkv = s.h_kv / s.P, Pb = int64_t(s.P) * s.b;
+  const int64_t hq = s.h_q / s.P, hkv = kv_heads_per_rank(s), Pb = int64_t(s.P) * s.b;
   const size_t gsz = dtype_size(g_dtype);
   const size_t dqb = size_t(Pb * s.n * hq * s.d) * gsz, dkb = size_t(Pb * s.n * hkv * s.d) * gsz;
   const size_t qb = size_t(Pb * s.n * hq * s.d) * 2, kb = size_t(Pb * s.n * hkv * s.d) * 2;
@@ -900,7 +900,7 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.rank0 = int32_t(rank0);
     p.hq = int32_t(hq);
     p.hkv = int32_t(hkv);
-    p.G = int32_t(s.h_q / s.h_kv);
+    p.G = int32_t(group_per_rank(s));
     p.scale = scale;
     p.scale_log2 = scale * bwd::kLog2e;
     p.g_f32 = g_dtype == ULY_F32;
@@ -934,7 +934,7 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.P_sel = int32_t(P_sel);
     p.rank0 = int32_t(rank0);
     p.hq = int32_t(hq);
-    p.G = int32_t(s.h_q / s.h_kv);
+    p.G = int32_t(group_per_rank(s));
     p.ntiles = int32_t((s.n + bwd::dq::BM - 1) / bwd::dq::BM);
     p.scale = scale;
     p.scale_log2 = scale * bwd::kLog2e;

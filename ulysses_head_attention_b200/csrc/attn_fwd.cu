@@ -461,7 +461,7 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
   if (!o_head || !lse || !dtype_ok(o_dtype)) return ULY_ERR_INVALID_ARG;
   if (!aligned(o_head, 16) || !aligned(lse, 16)) return ULY_ERR_INVALID_ARG;
   const uly_shape& s = *shape;
-  const int64_t hq = s.h_q / s.P, hkv = s.h_kv / s.P, Pb = int64_t(s.P) * s.b;
+  const int64_t hq = s.h_q / s.P, hkv = kv_heads_per_rank(s), Pb = int64_t(s.P) * s.b;
   const int64_t ntiles = (s.n + fwd::BM - 1) / fwd::BM;
   const int64_t npairs = (ntiles + 1) / 2;
   const int64_t P_sel = rank < 0 ? s.P : 1;
@@ -498,7 +498,7 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
   p.P_sel = int32_t(P_sel);
   p.rank0 = rank < 0 ? 0 : rank;
   p.hq = int32_t(hq);
-  p.G = int32_t(s.h_q / s.h_kv);
+  p.G = int32_t(group_per_rank(s));
   p.ntiles = int32_t(ntiles);
   p.npairs = int32_t(npairs);
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf(float(s.d));

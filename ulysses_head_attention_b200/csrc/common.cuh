@@ -34,17 +34,25 @@ inline bool elems(int64_t b, int64_t n, int64_t H, int64_t d, int64_t* out) {
   return checked_mul(b, n, &t) && checked_mul(t, H, &t) && checked_mul(t, d, out);
 }
 
-// The divisibility rules of the pages: n and both head counts divisible by
-// P; H_q a multiple of H_kv.
+// The divisibility rules of the pages: n and the query head count divisible
+// by P; H_q a multiple of H_kv.  The kv head count is divisible by P, or
+// (fewer kv heads than ranks) divides P: then each rank holds one replicated
+// kv head (ulysses_kv_seq_to_head).
 inline uly_status check_shape(const uly_shape* s) {
   if (!s) return ULY_ERR_INVALID_ARG;
   if (s->P < 1 || s->b < 1 || s->n < 1 || s->h_q < 1 || s->h_kv < 1 || s->d < 1) return ULY_ERR_INVALID_ARG;
-  if (s->n % s->P || s->h_q % s->P || s->h_kv % s->P || s->h_q % s->h_kv) return ULY_ERR_INVALID_ARG;
+  if (s->n % s->P || s->h_q % s->P || s->h_q % s->h_kv) return ULY_ERR_INVALID_ARG;
+  if (s->h_kv % s->P && (s->h_kv > s->P || s->P % s->h_kv)) return ULY_ERR_INVALID_ARG;
   if (s->n > (int64_t(1) << 31) - 256) return ULY_ERR_UNSUPPORTED;   // TMA coordinates are int32
   int64_t e;
   if (!elems(s->b, s->n, s->h_q, s->d, &e)) return ULY_ERR_INVALID_ARG;
   return ULY_OK;
 }
+
+// kv heads one rank holds in the head layout: H_kv / P, or one replicated
+// head when H_kv < P.  Query heads per local kv head follow.
+inline int64_t kv_heads_per_rank(const uly_shape& s) { return s.h_kv >= s.P ? s.h_kv / s.P : 1; }
+inline int64_t group_per_rank(const uly_shape& s) { return (s.h_q / s.P) / kv_heads_per_rank(s); }
 
 inline uly_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA; }
 

@@ -138,8 +138,164 @@ uly_status relayout(const void* src, void* dst, int64_t b, int64_t n, int64_t H,
   return cuda_status(err);
 }
 
+// ---------------------------------------------------------------------------
+// K/V with fewer kv heads than ranks (H_kv < P, P a multiple of H_kv): every
+// rank r gets a copy of kv head g(r) = r*H_kv/P, the one its query heads
+// read (the pages are silent on this case; this is the plain reading).  The
+// gradient of the copies is the sum over the P/H_kv ranks holding a head.
+// Both are HBM-bound: 16-byte vectors, one CTA per (rank, batch row, tile of
+// tokens).
+// ---------------------------------------------------------------------------
+struct KvArgs {
+  int64_t b, m, n, H, P;   // batch rows, tokens per rank, tokens, kv heads, ranks
+  int64_t vrow;            // 16-byte vectors per head row (d * esize / 16)
+  int32_t tile_tokens;
+  int32_t tiles;           // tiles per (rank, batch row)
+};
+
+// x_head[r][bb][t][0][:] = x_seq[t / m][bb][t % m][g(r)][:]
+__global__ void __launch_bounds__(kThreads) kv_replicate_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                                KvArgs a) {
+  const int64_t tile = blockIdx.x % a.tiles;
+  const int64_t rb = blockIdx.x / a.tiles;            // r * b + bb
+  const int64_t r = rb / a.b, bb = rb % a.b;
+  const int64_t g = r * a.H / a.P;
+  const int64_t t0 = tile * a.tile_tokens;
+  const int64_t t1 = t0 + a.tile_tokens < a.n ? t0 + a.tile_tokens : a.n;
+  const int64_t total = (t1 - t0) * a.vrow;
+  uint4* out = dst + (rb * a.n + t0) * a.vrow;
+  for (int64_t k = threadIdx.x; k < total; k += kThreads) {
+    const int64_t t = t0 + k / a.vrow, c = k % a.vrow;
+    const int64_t s = t / a.m, u = t % a.m;
+    out[k] = src[(((s * a.b + bb) * a.m + u) * a.H + g) * a.vrow + c];
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void add8(float (&acc)[8], const uint4* p);
+template <>
+__device__ __forceinline__ void add8<uint16_t>(float (&acc)[8], const uint4* p) {
+  const uint4 v = *p;
+  acc[0] += __uint_as_float(v.x << 16); acc[1] += __uint_as_float(v.x & 0xFFFF0000u);
+  acc[2] += __uint_as_float(v.y << 16); acc[3] += __uint_as_float(v.y & 0xFFFF0000u);
+  acc[4] += __uint_as_float(v.z << 16); acc[5] += __uint_as_float(v.z & 0xFFFF0000u);
+  acc[6] += __uint_as_float(v.w << 16); acc[7] += __uint_as_float(v.w & 0xFFFF0000u);
+}
+template <>
+__device__ __forceinline__ void add8<float>(float (&acc)[8], const uint4* p) {
+  const uint4 v0 = p[0], v1 = p[1];
+  acc[0] += __uint_as_float(v0.x); acc[1] += __uint_as_float(v0.y);
+  acc[2] += __uint_as_float(v0.z); acc[3] += __uint_as_float(v0.w);
+  acc[4] += __uint_as_float(v1.x); acc[5] += __uint_as_float(v1.y);
+  acc[6] += __uint_as_float(v1.z); acc[7] += __uint_as_float(v1.w);
+}
+
+__device__ __forceinline__ uint32_t bf16_rne(float x) {
+  const uint32_t u = __float_as_uint(x);
+  if ((u & 0x7F800000u) == 0x7F800000u) return (u >> 16) | ((u & 0xFFFFu) ? 0x40u : 0u);   // inf / nan
+  return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+}
+
+// x_seq[s][bb][u][g][:] = sum over r in [g P/H, (g+1) P/H), ascending, of
+// x_head[r][bb][s m + u][0][:]; fp32 sums.  One thread per 8 elements.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) kv_reduce_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                             KvArgs a, int64_t d) {
+  constexpr int kVec = sizeof(T) == 2 ? 1 : 2;        // 16-byte vectors per 8 elements
+  const int64_t groups_per_row = d / 8;               // 8-element groups per head row
+  const int64_t tile = blockIdx.x % a.tiles;
+  const int64_t sb = blockIdx.x / a.tiles;            // s * b + bb (output rank, batch row)
+  const int64_t s = sb / a.b, bb = sb % a.b;
+  const int64_t u0 = tile * a.tile_tokens;
+  const int64_t u1 = u0 + a.tile_tokens < a.m ? u0 + a.tile_tokens : a.m;
+  const int64_t R = a.P / a.H;
+  const int64_t total = (u1 - u0) * a.H * groups_per_row;
+  for (int64_t k = threadIdx.x; k < total; k += kThreads) {
+    const int64_t c = k % groups_per_row;
+    const int64_t g = (k / groups_per_row) % a.H;
+    const int64_t u = u0 + k / (groups_per_row * a.H);
+    const int64_t t = s * a.m + u;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int64_t r = g * R; r < (g + 1) * R; ++r)
+      add8<T>(acc, src + ((r * a.b + bb) * a.n + t) * groups_per_row * kVec + c * kVec);
+    uint4* o = dst + ((sb * a.m + u) * a.H + g) * groups_per_row * kVec + c * kVec;
+    if (sizeof(T) == 2) {
+      o[0] = make_uint4(bf16_rne(acc[0]) | (bf16_rne(acc[1]) << 16), bf16_rne(acc[2]) | (bf16_rne(acc[3]) << 16),
+                        bf16_rne(acc[4]) | (bf16_rne(acc[5]) << 16), bf16_rne(acc[6]) | (bf16_rne(acc[7]) << 16));
+    } else {
+      o[0] = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                        __float_as_uint(acc[3]));
+      o[kVec - 1] = make_uint4(__float_as_uint(acc[4]), __float_as_uint(acc[5]), __float_as_uint(acc[6]),
+                               __float_as_uint(acc[7]));
+    }
+  }
+}
+
+// Validation shared by both directions; H < P, P % H == 0 here.  The seq
+// buffer holds b*n*H*d elements, the head buffer b*n*P*d (one head per rank).
+uly_status kv_check(const void* src, void* dst, int64_t b, int64_t n, int64_t H, int64_t d, int32_t P,
+                    uly_dtype dt, bool to_head, KvArgs* a) {
+  if (d % 8 || d * int64_t(dtype_size(dt)) % 16) return ULY_ERR_UNSUPPORTED;
+  int64_t e_seq, e_head;
+  if (!elems(b, n, H, d, &e_seq) || !elems(b, n, P, d, &e_head)) return ULY_ERR_INVALID_ARG;
+  const size_t es = dtype_size(dt);
+  const size_t src_bytes = size_t(to_head ? e_seq : e_head) * es, dst_bytes = size_t(to_head ? e_head : e_seq) * es;
+  if (overlaps(src, src_bytes, dst, dst_bytes)) return ULY_ERR_INVALID_ARG;
+  a->b = b;
+  a->n = n;
+  a->m = n / P;
+  a->H = H;
+  a->P = P;
+  a->vrow = d * int64_t(es) / 16;
+  return ULY_OK;
+}
+
+template <bool kToHead>
+uly_status kv_relayout(const void* src, void* dst, int64_t b, int64_t n, int64_t H, int64_t d, int32_t P,
+                       uly_dtype dt, void* stream) {
+  if (!src || !dst || !dtype_ok(dt)) return ULY_ERR_INVALID_ARG;
+  if (P < 1 || b < 1 || n < 1 || H < 1 || d < 1 || n % P) return ULY_ERR_INVALID_ARG;
+  if (H % P == 0) return relayout<kToHead>(src, dst, b, n, H, d, P, dt, stream);
+  if (P % H) return ULY_ERR_INVALID_ARG;
+  if (!aligned(src, 16) || !aligned(dst, 16)) return ULY_ERR_INVALID_ARG;
+  KvArgs a;
+  const uly_status st = kv_check(src, dst, b, n, H, d, P, dt, kToHead, &a);
+  if (st != ULY_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (kToHead) {
+    a.tile_tokens = int32_t(4096 / a.vrow > 0 ? 4096 / a.vrow : 1);
+    a.tiles = int32_t((n + a.tile_tokens - 1) / a.tile_tokens);
+    const int64_t grid = int64_t(P) * b * a.tiles;
+    if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
+    kv_replicate_kernel<<<unsigned(grid), kThreads, 0, cs>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), a);
+  } else {
+    const int64_t groups = H * (d / 8);                // 8-element groups per token of the output
+    a.tile_tokens = int32_t(2048 / groups > 0 ? 2048 / groups : 1);
+    a.tiles = int32_t((a.m + a.tile_tokens - 1) / a.tile_tokens);
+    const int64_t grid = int64_t(P) * b * a.tiles;
+    if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
+    if (dt == ULY_BF16)
+      kv_reduce_kernel<uint16_t><<<unsigned(grid), kThreads, 0, cs>>>(static_cast<const uint4*>(src),
+                                                                      static_cast<uint4*>(dst), a, d);
+    else
+      kv_reduce_kernel<float><<<unsigned(grid), kThreads, 0, cs>>>(static_cast<const uint4*>(src),
+                                                                   static_cast<uint4*>(dst), a, d);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 }  // namespace uly
+
+extern "C" uly_status ulysses_kv_seq_to_head(const void* x_seq, void* x_head, int64_t b, int64_t n, int64_t H_kv,
+                                             int64_t d, int32_t P, uly_dtype dt, void* stream) {
+  return uly::kv_relayout<true>(x_seq, x_head, b, n, H_kv, d, P, dt, stream);
+}
+
+extern "C" uly_status ulysses_kv_head_to_seq(const void* x_head, void* x_seq, int64_t b, int64_t n, int64_t H_kv,
+                                             int64_t d, int32_t P, uly_dtype dt, void* stream) {
+  return uly::kv_relayout<false>(x_head, x_seq, b, n, H_kv, d, P, dt, stream);
+}
 
 extern "C" uly_status ulysses_seq_to_head(const void* x_seq, void* x_head, int64_t b, int64_t n, int64_t H,
                                           int64_t d, int32_t P, uly_dtype dt, void* stream) {
