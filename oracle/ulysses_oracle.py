@@ -18,7 +18,15 @@ What is computed, step by step, and where the pages define it:
   5. Backward: the gradient of the attention with respect to q, k, v
      (training through the layer, [ACC-SP] custom training loop); the
      gradient of a re-layout is the inverse re-layout.
-  6. Weighted loss aggregation across the SP ranks -- [ACC-SP] custom
+  6. Attention over one block of keys, and the LSE merge of such blocks --
+     [ACC-SP] "How Ulysses SP differs from FSDP CP" and [BLOG] on ring
+     attention: the sequence is sharded, KV blocks travel between ranks, and
+     each rank combines the partial results of the blocks it saw.  A block's
+     partial result is (O_b, LSE_b) over the visible keys of the block; the
+     merge is LSE = log sum_b exp(LSE_b), O = sum_b exp(LSE_b - LSE) O_b.
+     The backward of a block, given the merged O and LSE, is that block's
+     share of dQ and the full dK, dV of its keys.
+  7. Weighted loss aggregation across the SP ranks -- [ACC-SP] custom
      training loop (each rank's loss weighted by its count of labels other
      than -100; ranks without such labels skipped; divided by
      max(total count, 1)) and [BLOG] "Loss aggregation".
@@ -67,6 +75,8 @@ __all__ = [
     "ulysses_layer_fwd", "ulysses_layer_bwd",
     "default_scale",
     "sp_good_tokens", "sp_loss_aggregate",
+    "attention_fwd_head_range", "attention_bwd_head_range", "lse_merge",
+    "ulysses_attn_fwd_range", "ulysses_attn_bwd_range",
 ]
 
 
@@ -555,6 +565,124 @@ def ulysses_layer_bwd(q_seq, k_seq, v_seq, do_seq, position_ids, P: int,
                                   kv_seq_to_head(v_seq, P), seq_to_head(do_seq, P),
                                   position_ids, P, scale)
     return head_to_seq(dQ, P), kv_head_to_seq_reduce(dK, P, H_kv), kv_head_to_seq_reduce(dV, P, H_kv)
+
+
+# --------------------------------------------------------------------------
+# Attention over one key block, and the merge of blocks (ring attention)
+# --------------------------------------------------------------------------
+
+def attention_fwd_head_range(q, k, v, seg_start, scale, k_lo: int, k_hi: int, block: int = 256):
+    """Attention of every query row over the keys j in [k_lo, k_hi) it may
+    see (same sample, j <= i).  Rows with no such key: O = 0, LSE = -inf."""
+    n = q.shape[0]
+    O = np.zeros((n, v.shape[1]))
+    lse = np.full(n, -np.inf)
+    for i0 in range(0, n, block):
+        i1 = min(n, i0 + block)
+        rows = np.arange(i0, i1)
+        lo = np.maximum(seg_start[i0:i1], k_lo)
+        hi = np.minimum(rows + 1, k_hi)
+        j0, j1 = int(lo.min()), int(hi.max())
+        if j1 <= j0:
+            continue
+        cols = np.arange(j0, j1)
+        vis = (cols[None, :] >= lo[:, None]) & (cols[None, :] < hi[:, None])
+        has = vis.any(axis=1)
+        S = np.where(vis, scale * (q[i0:i1] @ k[j0:j1].T), -np.inf)
+        m = np.where(has, S.max(axis=1), 0.0)
+        E = np.where(vis, np.exp(S - m[:, None]), 0.0)
+        l = E.sum(axis=1)
+        Ob, Lb = O[i0:i1], lse[i0:i1]
+        Ob[has] = (E[has] @ v[j0:j1]) / l[has, None]
+        Lb[has] = m[has] + np.log(l[has])
+    return O, lse
+
+
+def attention_bwd_head_range(q, k, v, dO, O, lse, seg_start, scale, k_lo: int, k_hi: int, block: int = 256):
+    """One key block's share of the attention gradients, given the merged
+    (full) O and LSE of every row: P_ij = exp(scale q_i.k_j - LSE_i) over the
+    block's visible keys, D_i = dO_i . O_i, dS = P (dO v^T - D).
+    Returns dQ (this block's share), dK and dV (complete for the block's
+    keys, zero for the others)."""
+    n = q.shape[0]
+    dQ, dK, dV = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    D = np.sum(dO * O, axis=1)
+    for i0 in range(0, n, block):
+        i1 = min(n, i0 + block)
+        rows = np.arange(i0, i1)
+        lo = np.maximum(seg_start[i0:i1], k_lo)
+        hi = np.minimum(rows + 1, k_hi)
+        j0, j1 = int(lo.min()), int(hi.max())
+        if j1 <= j0:
+            continue
+        cols = np.arange(j0, j1)
+        vis = (cols[None, :] >= lo[:, None]) & (cols[None, :] < hi[:, None])
+        S = scale * (q[i0:i1] @ k[j0:j1].T)
+        Pm = np.where(vis, np.exp(np.where(vis, S, 0.0) - lse[i0:i1, None]), 0.0)
+        dP = dO[i0:i1] @ v[j0:j1].T
+        dS = Pm * (dP - D[i0:i1, None])
+        dQ[i0:i1] += scale * (dS @ k[j0:j1])
+        dK[j0:j1] += scale * (dS.T @ q[i0:i1])
+        dV[j0:j1] += Pm.T @ dO[i0:i1]
+    return dQ, dK, dV
+
+
+def lse_merge(o_parts: np.ndarray, lse_parts: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Merge partial results of B key blocks (head layout):
+    o_parts [B][P][b][n][h][d], lse_parts [B][P][b][h][n] ->
+    LSE = log sum_b exp(LSE_b); O = sum_b exp(LSE_b - LSE) O_b.
+    Rows where every LSE_b is -inf: O = 0, LSE = -inf."""
+    B = o_parts.shape[0]
+    m = np.max(lse_parts, axis=0)                       # [P][b][h][n]
+    fin = np.isfinite(m)
+    msafe = np.where(fin, m, 0.0)
+    total = np.zeros_like(m)
+    for bk in range(B):
+        total += np.where(np.isfinite(lse_parts[bk]), np.exp(lse_parts[bk] - msafe), 0.0)
+    lse = np.where(fin, msafe + np.log(np.where(fin, total, 1.0)), -np.inf)
+    O = np.zeros(o_parts.shape[1:])
+    for bk in range(B):
+        w = np.where(fin & np.isfinite(lse_parts[bk]), np.exp(lse_parts[bk] - np.where(fin, lse, 0.0)), 0.0)
+        O += np.transpose(w, (0, 1, 3, 2))[..., None] * o_parts[bk]   # [P][b][n][h][1]
+    return O, lse
+
+
+def ulysses_attn_fwd_range(q_head, k_head, v_head, position_ids, P: int, k_lo: int, k_hi: int,
+                           scale: Optional[float] = None, rank: Optional[int] = None):
+    """ulysses_attn_fwd restricted to keys [k_lo, k_hi) (one ring block)."""
+    Ps, b, n, hq, d = q_head.shape
+    G = hq // k_head.shape[3]
+    scale = default_scale(d) if scale is None else scale
+    ss = segment_starts(position_ids)
+    O = np.zeros(q_head.shape[:4] + (v_head.shape[4],))
+    lse = np.full((P, b, hq, n), -np.inf)
+    for r in _ranks(P, rank):
+        for bb in range(b):
+            for j in range(hq):
+                O[r, bb, :, j], lse[r, bb, j] = attention_fwd_head_range(
+                    q_head[r, bb, :, j], k_head[r, bb, :, j // G], v_head[r, bb, :, j // G], ss[bb], scale, k_lo, k_hi)
+    return O, lse
+
+
+def ulysses_attn_bwd_range(q_head, k_head, v_head, do_head, o_head, lse, position_ids, P: int, k_lo: int,
+                           k_hi: int, scale: Optional[float] = None, rank: Optional[int] = None):
+    """One key block's share of the per-rank backward (head layout)."""
+    Ps, b, n, hq, d = q_head.shape
+    G = hq // k_head.shape[3]
+    scale = default_scale(d) if scale is None else scale
+    ss = segment_starts(position_ids)
+    dQ, dK, dV = np.zeros(q_head.shape), np.zeros(k_head.shape), np.zeros(v_head.shape)
+    for r in _ranks(P, rank):
+        for bb in range(b):
+            for j in range(hq):
+                g = j // G
+                a, bk, c = attention_bwd_head_range(q_head[r, bb, :, j], k_head[r, bb, :, g], v_head[r, bb, :, g],
+                                                    do_head[r, bb, :, j], o_head[r, bb, :, j], lse[r, bb, j],
+                                                    ss[bb], scale, k_lo, k_hi)
+                dQ[r, bb, :, j] = a
+                dK[r, bb, :, g] += bk
+                dV[r, bb, :, g] += c
+    return dQ, dK, dV
 
 
 # --------------------------------------------------------------------------
