@@ -180,6 +180,56 @@ uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* 
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Ring attention / the Ulysses + ring hybrid (Accelerate guide "Sequence
+ * parallelism", "How Ulysses SP differs from FSDP CP"; blog "Ulysses Sequence
+ * Parallelism: Training with Million-Token Contexts", ring attention): the
+ * sequence is cut into key/value blocks, every query meets one block at a
+ * time, and the partial results are merged by their log-sum-exp.
+ *
+ * ulysses_attn_fwd_kv_range -- ulysses_attn_fwd over the keys of one block:
+ * key j takes part for query i only if k_lo <= j < k_hi besides the usual
+ * rule (same sample, j <= i).  A row that sees no key of the block gets
+ * O = 0 and LSE = -inf.  Requires 0 <= k_lo < k_hi <= n (else
+ * ULY_ERR_INVALID_ARG); everything else as ulysses_attn_fwd.
+ */
+uly_status ulysses_attn_fwd_kv_range(const void* q_head, const void* k_head, const void* v_head,
+                                     const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                                     float softmax_scale, int64_t k_lo, int64_t k_hi, void* o_head,
+                                     uly_dtype o_dtype, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * ulysses_attn_bwd_kv_range -- one key block's share of the backward, given
+ * the merged (all blocks) o_head and lse: with P_ij = exp(scale q_i.k_j -
+ * LSE_i) over the block's visible keys, D_i = dO_i . O_i and
+ * dS = P (dO V^T - D), dq_head gets this block's share of dQ (the blocks'
+ * shares add up to dQ), dk_head / dv_head the complete dK, dV of the
+ * block's keys and zeros for every other key.  Same arguments as
+ * ulysses_attn_bwd plus k_lo, k_hi (0 <= k_lo < k_hi <= n).
+ */
+uly_status ulysses_attn_bwd_kv_range(const void* q_head, const void* k_head, const void* v_head,
+                                     const void* o_head, uly_dtype o_dtype, const float* lse,
+                                     const void* do_head, const int64_t* position_ids,
+                                     const uly_shape* shape, int32_t rank, float softmax_scale,
+                                     int64_t k_lo, int64_t k_hi, void* dq_head, void* dk_head,
+                                     void* dv_head, uly_dtype g_dtype, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/*
+ * ulysses_attn_lse_merge -- combines the partial results of nparts key
+ * blocks:  LSE = log sum_b exp(LSE_b),  O = sum_b exp(LSE_b - LSE) O_b.
+ * Rows where every LSE_b is -inf get O = 0, LSE = -inf.
+ *   o_parts    float [nparts][P][b][n][h_q/P][d] (head layout, fp32)
+ *   lse_parts  float [nparts][P][b][h_q/P][n]
+ *   o_head     [P][b][n][h_q/P][d] of o_dtype; lse [P][b][h_q/P][n] float.
+ * 1 <= nparts <= 32; d 64 or 128 (else ULY_ERR_UNSUPPORTED); outputs must
+ * not overlap inputs or each other; 16-byte aligned.  One launch; float32
+ * arithmetic.
+ */
+uly_status ulysses_attn_lse_merge(const float* o_parts, const float* lse_parts, int32_t nparts,
+                                  const uly_shape* shape, void* o_head, uly_dtype o_dtype, float* lse,
+                                  void* stream);
+
+/*
  * ulysses_attn_bwd_timed -- ulysses_attn_bwd that also records five
  * caller-owned CUDA events on `stream` around its kernels, for measuring
  * each kernel's device time (the pages have no counterpart; this is

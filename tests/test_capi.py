@@ -165,3 +165,23 @@ def test_kv_relayout_rejects_unsupported_row_and_overlap():
     for fn in (uly.lib.ulysses_kv_seq_to_head, uly.lib.ulysses_kv_head_to_seq):
         assert fn(F, F + (1 << 30), 1, 64, 2, 4, 4, 0, None) == UNSUPPORTED      # d * 2 bytes not a multiple of 16
         assert fn(F, F + 1024, 1, 64, 2, 128, 4, 0, None) == INVALID            # overlapping buffers
+
+
+@no_gpu
+def test_ring_entries_reject_bad_ranges_and_parts():
+    import ulysses_head_attention_b200 as uly
+    s = shape()
+    G = 1 << 30
+    for lo, hi in ((-1, 10), (10, 10), (0, 1025), (20, 5)):
+        st = uly.lib.ulysses_attn_fwd_kv_range(F, F + G, F + 2 * G, F + 3 * G, ctypes.byref(s), -1, 0.0, lo, hi,
+                                               F + 4 * G, 1, F + 5 * G, F + 6 * G, 1 << 24, None)
+        assert st == INVALID
+        st = uly.lib.ulysses_attn_bwd_kv_range(F, F + G, F + 2 * G, F + 3 * G, 1, F + 4 * G, F + 5 * G, F + 6 * G,
+                                               ctypes.byref(s), -1, 0.0, lo, hi, F + 7 * G, F + 8 * G, F + 9 * G, 1,
+                                               F + 10 * G, 1 << 26, None)
+        assert st == INVALID
+    for nparts in (0, 33):
+        assert uly.lib.ulysses_attn_lse_merge(F, F + G, nparts, ctypes.byref(s), F + 2 * G, 1, F + 3 * G,
+                                              None) == INVALID
+    assert uly.lib.ulysses_attn_lse_merge(F, F + G, 2, ctypes.byref(shape(d=96)), F + 2 * G, 1, F + 3 * G,
+                                          None) == UNSUPPORTED

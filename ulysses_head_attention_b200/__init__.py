@@ -30,6 +30,7 @@ STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED",
 # Every symbol include/ulysses.h declares.
 EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head", "ulysses_kv_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_bwd_timed", "ulysses_attn_fwd_noalloc",
+           "ulysses_attn_fwd_kv_range", "ulysses_attn_bwd_kv_range", "ulysses_attn_lse_merge",
            "ulysses_sp_loss_aggregate", "ulysses_workspace_status", "ulysses_status_string")
 
 
@@ -62,6 +63,10 @@ def _load() -> ctypes.CDLL:
         "ulysses_attn_bwd_timed": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i32, f32, vp, vp, vp, i32, vp, sz, vp,
                                     ctypes.POINTER(vp)], i32),
         "ulysses_attn_fwd_noalloc": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp], i32),
+        "ulysses_attn_fwd_kv_range": ([vp, vp, vp, vp, shp, i32, f32, i64, i64, vp, i32, vp, vp, sz, vp], i32),
+        "ulysses_attn_bwd_kv_range": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i32, f32, i64, i64, vp, vp, vp, i32,
+                                       vp, sz, vp], i32),
+        "ulysses_attn_lse_merge": ([vp, vp, i32, shp, vp, i32, vp, vp], i32),
         "ulysses_sp_loss_aggregate": ([vp, vp, i64, i64, i32, i64, vp, vp, vp, vp], i32),
         "ulysses_workspace_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "ulysses_status_string": ([i32], ctypes.c_char_p),
@@ -262,6 +267,47 @@ def ulysses_sp_loss_aggregate(losses, shift_labels, loss, good, dlosses, ignore_
                                          ignore_index, _dev(loss, "loss"), _dev(good, "good"),
                                          _dev(dlosses, "dlosses"), _stream(stream)),
            "ulysses_sp_loss_aggregate")
+
+
+def ulysses_attn_fwd_kv_range(q_head, k_head, v_head, position_ids, o_head, lse, ws, k_lo: int, k_hi: int,
+                              rank: int = -1, softmax_scale: float = 0.0, stream=None) -> None:
+    """Forward over the keys [k_lo, k_hi) only (one ring block)."""
+    shape = _attn_shape(q_head, k_head)
+    _check(lib.ulysses_attn_fwd_kv_range(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
+                                         _dev(position_ids, "position_ids"), ctypes.byref(shape), rank,
+                                         softmax_scale, k_lo, k_hi, _dev(o_head, "o_head"), _dtype_code(o_head),
+                                         _dev(lse, "lse"), _dev(ws, "ws"), ws.numel() * ws.element_size(),
+                                         _stream(stream)), "ulysses_attn_fwd_kv_range")
+
+
+def ulysses_attn_bwd_kv_range(q_head, k_head, v_head, o_head, lse, do_head, position_ids, dq_head, dk_head, dv_head,
+                              ws, k_lo: int, k_hi: int, rank: int = -1, softmax_scale: float = 0.0,
+                              stream=None) -> None:
+    """One key block's share of the backward, given the merged O and LSE."""
+    shape = _attn_shape(q_head, k_head)
+    if dk_head.dtype != dq_head.dtype or dv_head.dtype != dq_head.dtype:
+        raise TypeError("dq/dk/dv must share one dtype")
+    _check(lib.ulysses_attn_bwd_kv_range(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
+                                         _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
+                                         _dev(do_head, "do_head"), _dev(position_ids, "position_ids"),
+                                         ctypes.byref(shape), rank, softmax_scale, k_lo, k_hi,
+                                         _dev(dq_head, "dq_head"), _dev(dk_head, "dk_head"), _dev(dv_head, "dv_head"),
+                                         _dtype_code(dq_head), _dev(ws, "ws"), ws.numel() * ws.element_size(),
+                                         _stream(stream)), "ulysses_attn_bwd_kv_range")
+
+
+def ulysses_attn_lse_merge(o_parts, lse_parts, o_head, lse, h_kv: int, stream=None) -> None:
+    """Merge B partial results: o_parts float32 (B, P, b, n, h, d), lse_parts
+    float32 (B, P, b, h, n) -> o_head (P, b, n, h, d), lse (P, b, h, n)."""
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32 or lse.dtype != torch.float32:
+        raise TypeError("o_parts, lse_parts and lse must be float32")
+    B, P, b, n, h, d = o_parts.shape
+    if tuple(lse_parts.shape) != (B, P, b, h, n) or tuple(o_head.shape) != (P, b, n, h, d):
+        raise ValueError("shapes do not match")
+    shape = UlyShape(b, n, h * P, h_kv, d, P)
+    _check(lib.ulysses_attn_lse_merge(_dev(o_parts, "o_parts"), _dev(lse_parts, "lse_parts"), B,
+                                      ctypes.byref(shape), _dev(o_head, "o_head"), _dtype_code(o_head),
+                                      _dev(lse, "lse"), _stream(stream)), "ulysses_attn_lse_merge")
 
 
 def ulysses_workspace_status(ws: torch.Tensor, stream=None) -> int:

@@ -130,6 +130,7 @@ struct Params {
   void* dv;
   int* status;
   int64_t n, n_pad;
+  int64_t k_lo, k_hi;    // only keys in [k_lo, k_hi) take part (one ring block); 0, n otherwise
   int32_t b, P_sel, rank0, hq, hkv, G;
   float scale, scale_log2;
   int32_t g_f32;
@@ -207,7 +208,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   const int64_t q_end = se[last_key];      // query rows that see this key tile: [k0, q_end)
   const int qt_first = int(k0 / BQ);
   const int nqt = int((q_end + BQ - 1) / BQ) - qt_first;
-  const int niter = nqt * p.G;             // (query head, query tile) pairs, head-major
+  // (query head, query tile) pairs, head-major; none when the key tile lies
+  // outside [k_lo, k_hi) (its dK, dV are then zero)
+  const int niter = (k0 < p.k_hi && k0 + BKV > p.k_lo) ? nqt * p.G : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -250,7 +253,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       uint64_t* full = is_q ? bars->q_full : bars->do_full;
       uint64_t* empty = is_q ? bars->q_empty : bars->do_empty;
       tma_prefetch_desc(is_q ? &mq : &mdo);
-      if (is_q) {
+      if (is_q && niter > 0) {
         mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKV);
         for (int dc = 0; dc < D / 64; ++dc) {
           tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0), rb);
@@ -277,7 +280,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         issued = it + 1;
       }
       if (*abort_flag) {   // error path only: let every copy this thread started land
-        if (is_q) mbar_wait(&bars->kv_full, 0, nullptr, nullptr, p.limit_ns);
+        if (is_q && niter > 0) mbar_wait(&bars->kv_full, 0, nullptr, nullptr, p.limit_ns);
         for (int x = max(0, issued - ns); x < issued; ++x)
           mbar_wait(&full[x % ns], (x / ns) & 1, nullptr, nullptr, p.limit_ns);
       }
@@ -320,7 +323,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           umma_ts_warp(acc_tmem, a_tmem + a_col, bd + uint64_t(kk * 2048 / 16), id_g, (it > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait_warp(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns) && niter > 0 &&
+      bool ok = niter > 0 && mbar_wait_warp(&bars->kv_full, 0, abort_flag, p.status, p.limit_ns) &&
                 mbar_wait_warp(&bars->q_full[0], 0, abort_flag, p.status, p.limit_ns) &&
                 mbar_wait_warp(&bars->do_full[0], 0, abort_flag, p.status, p.limit_ns);
       if (ok) {
@@ -365,7 +368,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     const int row = ((warp - 4) & 3) * 32 + lane;    // key row within the tile
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t kj = k0 + row;
-    const int64_t kj_end = kj < p.n ? int64_t(se[kj]) : kj;   // query rows [kj, kj_end) see key kj
+    // query rows [kj, kj_end) see key kj (none for a key outside [k_lo, k_hi))
+    const int64_t kj_end = (kj < p.n && kj >= p.k_lo && kj < p.k_hi) ? int64_t(se[kj]) : kj;
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < niter; ++it) {
@@ -471,6 +475,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           uint32_t o[32];
           tmem_ld32(base + lane_off + c, o);
           tmem_ld_wait();
+          if (niter == 0) {   // no MMA ran: the accumulators were never written
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
           if (valid) {
             if (p.g_f32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + orow * D + c);
@@ -521,6 +529,7 @@ struct Params {
   void* dq;              // [P*b][n][hq][D]
   int* status;
   int64_t n, n_pad;
+  int64_t k_lo, k_hi;    // only keys in [k_lo, k_hi) take part (one ring block); 0, n otherwise
   int32_t b, P_sel, rank0, hq, G, ntiles;
   float scale, scale_log2;
   int32_t g_f32;
@@ -573,8 +582,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
   const int32_t* ss = p.segstart + int64_t(bb) * p.n;
   const int64_t seg_lo = ss[t0];
   const int64_t seg_hi = ss[last_row];
-  const int kv_first = int(seg_lo / BN);
-  const int nkv = int(last_row / BN) - kv_first + 1;
+  // key tiles: the tile's visible keys, clipped to [k_lo, k_hi); none -> dQ = 0
+  const int64_t key_lo = seg_lo > p.k_lo ? seg_lo : p.k_lo;
+  const int64_t key_hi = last_row < p.k_hi - 1 ? last_row : p.k_hi - 1;   // inclusive
+  const int kv_first = int(key_lo / BN);
+  const int nkv = key_hi >= key_lo ? int(key_hi / BN) - kv_first + 1 : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->qdo_full, 1);
@@ -688,7 +700,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         umma_commit_warp(&bars->v_empty[sv]);
         if (it >= 1 && !issue_dq(it - 1)) { ok = false; break; }
       }
-      if (ok) issue_dq(nkv - 1);
+      if (ok && nkv > 0) issue_dq(nkv - 1);
       umma_commit_warp(&bars->mma_final);
     }
   } else if (warp >= 4) {
@@ -698,6 +710,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     const int64_t i = t0 + row;
     const bool valid = i < p.n;
     const int64_t s_i = valid ? ss[i] : seg_hi;
+    // this row's keys: [row_lo, row_hi) = its sample's keys up to i, inside [k_lo, k_hi)
+    const int64_t row_lo = s_i > p.k_lo ? s_i : p.k_lo;
+    const int64_t row_hi = i + 1 < p.k_hi ? i + 1 : p.k_hi;
     float nl = 0.f, nd = 0.f;   // -LSE*log2e, -D of this row
     if (valid) {
       const int64_t si = stats_index(int64_t(rb) * p.hq + h, p.n_pad, i);
@@ -723,8 +738,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->dp_free);
-      // visible key columns c of this warpgroup: lo <= c < hi (keys s_i .. i)
-      const int64_t lo64 = s_i - k0, hi64 = valid ? i + 1 - k0 : lo64;
+      // visible key columns c of this warpgroup: lo <= c < hi (keys row_lo .. row_hi - 1)
+      const int64_t lo64 = row_lo - k0, hi64 = valid ? row_hi - k0 : lo64;
       const bool need_mask = lo64 > 0 || hi64 < 64;
       const int lo = int(lo64 < 0 ? 0 : (lo64 > 64 ? 64 : lo64));
       const int hi = int(hi64 < lo ? lo : (hi64 > 64 ? 64 : hi64));
@@ -761,6 +776,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
           uint32_t o[32];
           tmem_ld32(tDQ + lane_off + c + c2, o);
           tmem_ld_wait();
+          if (nkv == 0) {   // no MMA ran: the accumulator was never written
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
           if (valid) {
             if (p.g_f32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.dq) + orow * D + c + c2);
@@ -813,14 +832,16 @@ extern "C" size_t ulysses_attn_bwd_workspace(const uly_shape* s, uly_dtype g_dty
 
 // events: null, or five caller-owned cudaEvent_t recorded on the stream
 // before the segment-table, statistics, dK/dV and dQ kernels and after dQ.
+// k_lo, k_hi: the key range taking part ([0, n) for the plain backward).
 static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const void* v_head, const void* o_head,
                                 uly_dtype o_dtype, const float* lse, const void* do_head, const int64_t* position_ids,
-                                const uly_shape* shape, int32_t rank, float softmax_scale, void* dq_head,
-                                void* dk_head, void* dv_head, uly_dtype g_dtype, void* ws, size_t ws_bytes,
-                                void* stream, void* const* events) {
+                                const uly_shape* shape, int32_t rank, float softmax_scale, int64_t k_lo,
+                                int64_t k_hi, void* dq_head, void* dk_head, void* dv_head, uly_dtype g_dtype,
+                                void* ws, size_t ws_bytes, void* stream, void* const* events) {
   uly_status st = validate_attn(q_head, k_head, v_head, position_ids, shape, rank, ws, ws_bytes,
                                 shape ? ulysses_attn_bwd_workspace(shape, g_dtype) : 0);
   if (st != ULY_OK) return st;
+  if (k_lo < 0 || k_hi <= k_lo || k_hi > shape->n) return ULY_ERR_INVALID_ARG;
   if (!o_head || !lse || !do_head || !dq_head || !dk_head || !dv_head) return ULY_ERR_INVALID_ARG;
   if (!dtype_ok(o_dtype) || !dtype_ok(g_dtype)) return ULY_ERR_INVALID_ARG;
   if (!aligned(o_head, 16) || !aligned(lse, 16) || !aligned(do_head, 16) || !aligned(dq_head, 16) ||
@@ -895,6 +916,8 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.status = reinterpret_cast<int*>(wsb);
     p.n = s.n;
     p.n_pad = n_pad;
+    p.k_lo = k_lo;
+    p.k_hi = k_hi;
     p.b = int32_t(s.b);
     p.P_sel = int32_t(P_sel);
     p.rank0 = int32_t(rank0);
@@ -930,6 +953,8 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.status = reinterpret_cast<int*>(wsb);
     p.n = s.n;
     p.n_pad = n_pad;
+    p.k_lo = k_lo;
+    p.k_hi = k_hi;
     p.b = int32_t(s.b);
     p.P_sel = int32_t(P_sel);
     p.rank0 = int32_t(rank0);
@@ -964,8 +989,21 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
                                        const int64_t* position_ids, const uly_shape* shape, int32_t rank,
                                        float softmax_scale, void* dq_head, void* dk_head, void* dv_head,
                                        uly_dtype g_dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (check_shape(shape) != ULY_OK) return check_shape(shape);
   return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
-                       softmax_scale, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, nullptr);
+                       softmax_scale, 0, shape->n, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, nullptr);
+}
+
+extern "C" uly_status ulysses_attn_bwd_kv_range(const void* q_head, const void* k_head, const void* v_head,
+                                                const void* o_head, uly_dtype o_dtype, const float* lse,
+                                                const void* do_head, const int64_t* position_ids,
+                                                const uly_shape* shape, int32_t rank, float softmax_scale,
+                                                int64_t k_lo, int64_t k_hi, void* dq_head, void* dk_head,
+                                                void* dv_head, uly_dtype g_dtype, void* ws, size_t ws_bytes,
+                                                void* stream) {
+  if (check_shape(shape) != ULY_OK) return check_shape(shape);
+  return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
+                       softmax_scale, k_lo, k_hi, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, nullptr);
 }
 
 extern "C" uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_head, const void* v_head,
@@ -977,6 +1015,7 @@ extern "C" uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_h
   if (!events) return ULY_ERR_INVALID_ARG;
   for (int i = 0; i < 5; ++i)
     if (!events[i]) return ULY_ERR_INVALID_ARG;
+  if (check_shape(shape) != ULY_OK) return check_shape(shape);
   return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
-                       softmax_scale, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, events);
+                       softmax_scale, 0, shape->n, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, events);
 }

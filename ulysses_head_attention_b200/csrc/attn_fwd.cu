@@ -55,6 +55,7 @@ struct Params {
   void* o;                   // [P][b][n][hq][D]
   int* status;
   int64_t n;
+  int64_t k_lo, k_hi;        // keys outside [k_lo, k_hi) are not attended (one ring block); 0, n otherwise
   int32_t b, P_sel, rank0, hq, G, ntiles, npairs;
   float scale_log2;
   int32_t o_f32;
@@ -90,14 +91,19 @@ struct TileRange {
   bool valid;
 };
 
-__device__ __forceinline__ TileRange tile_range(const int32_t* ss, int64_t n, int tile, int ntiles) {
+// Key tiles are also clipped to [k_lo, k_hi); first > last means the query
+// tile sees no key there (0 <= k_lo < k_hi <= n).
+__device__ __forceinline__ TileRange tile_range(const int32_t* ss, int64_t n, int tile, int ntiles, int64_t k_lo,
+                                                int64_t k_hi) {
   TileRange tr;
   tr.valid = tile < ntiles;
   const int tl = tr.valid ? tile : ntiles - 1;
   tr.t0 = int64_t(tl) * BM;
   const int64_t last_row = (tr.t0 + BM - 1 < n - 1) ? (tr.t0 + BM - 1) : (n - 1);
-  tr.first = int(int64_t(ss[tr.t0]) / BN);
-  tr.last = int(last_row / BN);
+  const int64_t key_lo = int64_t(ss[tr.t0]) > k_lo ? int64_t(ss[tr.t0]) : k_lo;
+  const int64_t key_hi = last_row < k_hi - 1 ? last_row : k_hi - 1;   // last key, inclusive
+  tr.first = int(key_lo / BN);
+  tr.last = key_hi >= key_lo ? int(key_hi / BN) : tr.first - 1;
   tr.seg_hi = ss[last_row];
   return tr;
 }
@@ -124,10 +130,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   const int rb = r * p.b + bb;
   const int g = j / p.G;
   const int32_t* ss = p.segstart + int64_t(bb) * p.n;
-  const TileRange tr0 = tile_range(ss, p.n, 2 * pair, p.ntiles);
-  const TileRange tr1 = tile_range(ss, p.n, 2 * pair + 1, p.ntiles);
-  const int j_lo = tr0.first;                               // tile 1 starts no earlier
-  const int j_hi = tr1.valid ? tr1.last : tr0.last;
+  const TileRange tr0 = tile_range(ss, p.n, 2 * pair, p.ntiles, p.k_lo, p.k_hi);
+  const TileRange tr1 = tile_range(ss, p.n, 2 * pair + 1, p.ntiles, p.k_lo, p.k_hi);
+  const bool has0 = tr0.valid && tr0.last >= tr0.first, has1 = tr1.valid && tr1.last >= tr1.first;
+  // key tiles of the pair: tile 1 starts no earlier and ends no earlier than tile 0
+  const int j_lo = has0 ? tr0.first : (has1 ? tr1.first : 0);
+  const int j_hi = has1 ? tr1.last : (has0 ? tr0.last : -1);
   const int nkv = j_hi - j_lo + 1;
 
   if (threadIdx.x == 0) {
@@ -258,10 +266,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     const int64_t i = tr.t0 + row;
     const bool valid = tr.valid && i < p.n;
     const int64_t s_i = valid ? ss[i] : tr.seg_hi;
+    // this row's keys: [row_lo, row_hi) = its sample's keys up to i, inside [k_lo, k_hi)
+    const int64_t row_lo = s_i > p.k_lo ? s_i : p.k_lo;
+    const int64_t row_hi = i + 1 < p.k_hi ? i + 1 : p.k_hi;
+    const bool row_vis = valid && row_hi > row_lo;
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     float m_used = -INFINITY, l = 0.f;   // running max (log2 units, scaled) and row sum
     bool ok = true;
-    const int ntile = tr.valid ? tr.last - tr.first + 1 : 0;
+    const int ntile = tr.valid && tr.last >= tr.first ? tr.last - tr.first + 1 : 0;
     for (int c = 0; c < ntile; ++c) {
       const int64_t k0 = int64_t(tr.first + c) * BN;
       if (!mbar_wait(&bars->s_full[q], c & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
@@ -280,8 +292,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         x[64 + e] = __uint_as_float(a2[e]);
         x[96 + e] = __uint_as_float(a3[e]);
       }
-      // visible key columns: lo <= col < hi (keys s_i .. i)
-      const int64_t lo64 = s_i - k0, hi64 = valid ? i + 1 - k0 : lo64;
+      // visible key columns: lo <= col < hi (keys row_lo .. row_hi - 1)
+      const int64_t lo64 = row_lo - k0, hi64 = valid ? row_hi - k0 : lo64;
       if (lo64 > 0 || hi64 < BN) {
         const int lo = int(lo64 < 0 ? 0 : (lo64 > BN ? BN : lo64));
         const int hi = int(hi64 < lo ? lo : (hi64 > BN ? BN : hi64));
@@ -363,7 +375,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     // ---- epilogue: O / l and LSE
     if (ntile > 0 && mbar_wait(&bars->o_final[q], 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = row_vis ? 1.f / l : 0.f;   // a row that saw no key gets O = 0
       const int64_t orow = (int64_t(rb) * p.n + i) * p.hq + j;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
@@ -391,7 +403,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           }
         }
       }
-      if (valid) p.lse[(int64_t(rb) * p.hq + j) * p.n + i] = (m_used + log2f(l)) * 0.69314718055994531f;
+      if (valid)
+        p.lse[(int64_t(rb) * p.hq + j) * p.n + i] = row_vis ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    } else if (ntile == 0 && valid) {
+      // no key of [k_lo, k_hi) is visible to this query tile: O = 0, LSE = -inf
+      const int64_t orow = (int64_t(rb) * p.n + i) * p.hq + j;
+      if (p.o_f32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D);
+        for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D);
+        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      p.lse[(int64_t(rb) * p.hq + j) * p.n + i] = -INFINITY;
     }
   }
 
@@ -451,13 +475,15 @@ extern "C" size_t ulysses_attn_fwd_workspace(const uly_shape* s) {
   return seg_workspace_bytes(s->b, s->n);
 }
 
-extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, const void* v_head,
-                                       const int64_t* position_ids, const uly_shape* shape, int32_t rank,
-                                       float softmax_scale, void* o_head, uly_dtype o_dtype, float* lse, void* ws,
-                                       size_t ws_bytes, void* stream) {
+// k_lo, k_hi: the key range attended ([0, n) for the plain forward).
+static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const void* v_head,
+                                const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                                float softmax_scale, int64_t k_lo, int64_t k_hi, void* o_head, uly_dtype o_dtype,
+                                float* lse, void* ws, size_t ws_bytes, void* stream) {
   uly_status st = validate_attn(q_head, k_head, v_head, position_ids, shape, rank, ws, ws_bytes,
                                 shape ? ulysses_attn_fwd_workspace(shape) : 0);
   if (st != ULY_OK) return st;
+  if (k_lo < 0 || k_hi <= k_lo || k_hi > shape->n) return ULY_ERR_INVALID_ARG;
   if (!o_head || !lse || !dtype_ok(o_dtype)) return ULY_ERR_INVALID_ARG;
   if (!aligned(o_head, 16) || !aligned(lse, 16)) return ULY_ERR_INVALID_ARG;
   const uly_shape& s = *shape;
@@ -494,6 +520,8 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
   p.o = o_head;
   p.status = reinterpret_cast<int*>(wsb);
   p.n = s.n;
+  p.k_lo = k_lo;
+  p.k_hi = k_hi;
   p.b = int32_t(s.b);
   p.P_sel = int32_t(P_sel);
   p.rank0 = rank < 0 ? 0 : rank;
@@ -507,6 +535,25 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
   p.limit_ns = 2000000000ull;
   e = s.d == 128 ? fwd::launch<128>(mq, mk, mv, p, grid, cs) : fwd::launch<64>(mq, mk, mv, p, grid, cs);
   return cuda_status(e);
+}
+
+extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, const void* v_head,
+                                       const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                                       float softmax_scale, void* o_head, uly_dtype o_dtype, float* lse, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  if (check_shape(shape) != ULY_OK) return check_shape(shape);
+  return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, 0, shape->n, o_head,
+                       o_dtype, lse, ws, ws_bytes, stream);
+}
+
+extern "C" uly_status ulysses_attn_fwd_kv_range(const void* q_head, const void* k_head, const void* v_head,
+                                                const int64_t* position_ids, const uly_shape* shape, int32_t rank,
+                                                float softmax_scale, int64_t k_lo, int64_t k_hi, void* o_head,
+                                                uly_dtype o_dtype, float* lse, void* ws, size_t ws_bytes,
+                                                void* stream) {
+  if (check_shape(shape) != ULY_OK) return check_shape(shape);
+  return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, k_lo, k_hi, o_head,
+                       o_dtype, lse, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
