@@ -391,6 +391,50 @@ def run_ours(args, w):
     e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, dev) / args.steps
     e2e_value = whole_job_tflops(world, fwd_flops + bwd_flops, e2e_ms)
 
+    # ---- ring attention over R key blocks (forward + LSE merge, then the
+    # blocks' backward from the merged O / LSE), timed on its own
+    R = 4
+    cuts = [n * i // R for i in range(R + 1)]
+    o_parts = torch.empty((R,) + tuple(o_head.shape), dtype=f32, device=dev)
+    l_parts = torch.empty((R,) + tuple(lse.shape), dtype=f32, device=dev)
+    o_ring, l_ring = torch.empty_like(o_head), torch.empty_like(lse)
+    g_ring = {k: torch.empty_like(g_head[k]) for k in g_head}
+
+    def ring_fwd():
+        for i in range(R):
+            uly.ulysses_attn_fwd_kv_range(head["q"], head["k"], head["v"], pos, o_parts[i], l_parts[i], ws_f,
+                                          cuts[i], cuts[i + 1])
+        uly.ulysses_attn_lse_merge(o_parts, l_parts, o_ring, l_ring, hkv)
+
+    def ring_bwd():
+        for i in range(R):
+            uly.ulysses_attn_bwd_kv_range(head["q"], head["k"], head["v"], o_ring, l_ring, head["do"], pos,
+                                          g_ring["q"], g_ring["k"], g_ring["v"], ws_b, cuts[i], cuts[i + 1])
+
+    ring_fwd()
+    ring_bwd()
+    torch.cuda.synchronize()
+    rf = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    reps = 3
+    rf[0].record(stream)
+    for _ in range(reps):
+        ring_fwd()
+    rf[1].record(stream)
+    for _ in range(reps):
+        ring_bwd()
+    rf[2].record(stream)
+    torch.cuda.synchronize()
+    for ws in (ws_f, ws_b):
+        if uly.ulysses_workspace_status(ws) != 0:
+            raise RuntimeError("a kernel reported a pipeline timeout in the ring measurement")
+    ring_fwd_ms = rf[0].elapsed_time(rf[1]) / reps
+    ring_bwd_ms = rf[1].elapsed_time(rf[2]) / reps
+    ring_stat = {"blocks": R, "fwd_ms": ring_fwd_ms, "fwd_tflops": fwd_flops / (ring_fwd_ms * 1e-3) / 1e12,
+                 "bwd_ms_per_block_pass": ring_bwd_ms, "bwd_tflops": bwd_flops / (ring_bwd_ms * 1e-3) / 1e12,
+                 "launches": {"fwd": R * 2 + 1, "bwd": R * 4},
+                 "note": "keys cut into R equal blocks; forward = R key-range forwards + one LSE merge; "
+                         "backward = R key-range backwards from the merged O and LSE (one block's dQ share each)"}
+
     # ---- weighted SP loss aggregation (the custom training loop's per-rank loss
     # weighting), timed on its own: it needs a model's per-rank losses, which
     # this path does not produce, so it is not part of the step
@@ -435,6 +479,7 @@ def run_ours(args, w):
             "bwd_flops_with_recompute_convention": 10 * d * hq * pairs,
             "peaks": peaks,
             "sp_loss_aggregate": loss_stat,
+            "ring_attention": ring_stat,
         },
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": dom_tf / peak_t, "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
