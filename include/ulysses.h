@@ -128,6 +128,22 @@ uly_status ulysses_kv_seq_to_head(const void* x_seq, void* x_head, int64_t b, in
 uly_status ulysses_kv_head_to_seq(const void* x_head, void* x_seq, int64_t b, int64_t n, int64_t H_kv,
                                   int64_t d, int32_t P, uly_dtype dt, void* stream);
 
+/*
+ * ulysses_transpose_runs -- dst[j][i][:] = src[i][j][:] for i < A, j < B and
+ * runs of run_bytes bytes: the local permutations around a real all-to-all
+ * between processes ("How Ulysses works", steps 3 and 5, with each rank a
+ * separate GPU).  Before the exchange, rank r's seq shard [b*n/P][P][h*d]
+ * becomes P contiguous send chunks [P][b*n/P][h*d] (A = b*n/P, B = P,
+ * run = h*d*element size); after it, the received chunks [P][b][n/P*h*d]
+ * become the head layout [b][n][h][d] (A = P, B = b, run = n/P*h*d*element
+ * size); the way back uses the same call with the roles swapped.  Any
+ * alignment (the widest vector both pointers allow); out of place (buffers
+ * must not overlap).  Errors: null pointer, A, B or run_bytes < 1, size
+ * overflow, overlap: ULY_ERR_INVALID_ARG.  Bit-exact copy.
+ */
+uly_status ulysses_transpose_runs(const void* src, void* dst, int64_t A, int64_t B, int64_t run_bytes,
+                                  void* stream);
+
 /* Workspace bytes ulysses_attn_fwd needs for `shape` (0 on invalid shape). */
 size_t ulysses_attn_fwd_workspace(const uly_shape* shape);
 

@@ -185,3 +185,13 @@ def test_ring_entries_reject_bad_ranges_and_parts():
                                               None) == INVALID
     assert uly.lib.ulysses_attn_lse_merge(F, F + G, 2, ctypes.byref(shape(d=96)), F + 2 * G, 1, F + 3 * G,
                                           None) == UNSUPPORTED
+
+
+@no_gpu
+def test_transpose_rejects():
+    import ulysses_head_attention_b200 as uly
+    G = 1 << 30
+    assert uly.lib.ulysses_transpose_runs(0, F, 2, 2, 16, None) == INVALID
+    assert uly.lib.ulysses_transpose_runs(F, F + G, 0, 2, 16, None) == INVALID
+    assert uly.lib.ulysses_transpose_runs(F, F + G, 2, 2, 0, None) == INVALID
+    assert uly.lib.ulysses_transpose_runs(F, F + 32, 2, 2, 16, None) == INVALID   # overlap

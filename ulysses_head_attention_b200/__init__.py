@@ -28,7 +28,8 @@ ULY_BF16, ULY_F32 = 0, 1
 STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED", 3: "ULY_ERR_CUDA",
                 4: "ULY_ERR_WORKSPACE", 5: "ULY_ERR_TIMEOUT"}
 # Every symbol include/ulysses.h declares.
-EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head", "ulysses_kv_head_to_seq", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
+EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head", "ulysses_kv_head_to_seq",
+           "ulysses_transpose_runs", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_bwd_timed", "ulysses_attn_fwd_noalloc",
            "ulysses_attn_fwd_kv_range", "ulysses_attn_bwd_kv_range", "ulysses_attn_lse_merge",
            "ulysses_sp_loss_aggregate", "ulysses_workspace_status", "ulysses_status_string")
@@ -56,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "ulysses_head_to_seq": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
         "ulysses_kv_seq_to_head": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
         "ulysses_kv_head_to_seq": ([vp, vp, i64, i64, i64, i64, i32, i32, vp], i32),
+        "ulysses_transpose_runs": ([vp, vp, i64, i64, i64, vp], i32),
         "ulysses_attn_fwd_workspace": ([shp], sz),
         "ulysses_attn_fwd": ([vp, vp, vp, vp, shp, i32, f32, vp, i32, vp, vp, sz, vp], i32),
         "ulysses_attn_bwd_workspace": ([shp, i32], sz),
@@ -153,6 +155,15 @@ def ulysses_kv_head_to_seq(x_head: torch.Tensor, x_seq: torch.Tensor, stream=Non
         raise ValueError("x_seq shape/dtype does not match x_head")
     _check(lib.ulysses_kv_head_to_seq(_dev(x_head, "x_head"), _dev(x_seq, "x_seq"), b, m * P, H, d, P,
                                       _dtype_code(x_seq), _stream(stream)), "ulysses_kv_head_to_seq")
+
+
+def ulysses_transpose_runs(src: torch.Tensor, dst: torch.Tensor, A: int, B: int, run_bytes: int,
+                           stream=None) -> None:
+    """dst[j][i][:] = src[i][j][:] over runs of run_bytes bytes (i < A, j < B)."""
+    if src.numel() * src.element_size() != A * B * run_bytes or dst.numel() * dst.element_size() != A * B * run_bytes:
+        raise ValueError("buffer sizes do not match A * B * run_bytes")
+    _check(lib.ulysses_transpose_runs(_dev(src, "src"), _dev(dst, "dst"), A, B, run_bytes, _stream(stream)),
+           "ulysses_transpose_runs")
 
 
 def _attn_shape(q_head: torch.Tensor, k_head: torch.Tensor) -> UlyShape:

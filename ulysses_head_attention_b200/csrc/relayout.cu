@@ -284,6 +284,37 @@ uly_status kv_relayout(const void* src, void* dst, int64_t b, int64_t n, int64_t
   return cuda_status(cudaGetLastError());
 }
 
+// ---------------------------------------------------------------------------
+// dst[j][i][:] = src[i][j][:] for runs of run_bytes: the local permutations
+// around a real (multi-process) all-to-all.  One CTA per (j, tile of i): it
+// writes one contiguous block of dst and reads T runs of src at pitch B runs.
+// ---------------------------------------------------------------------------
+template <typename V>
+__global__ void __launch_bounds__(kThreads) transpose_runs_kernel(const V* __restrict__ src, V* __restrict__ dst,
+                                                                  int64_t A, int64_t B, int64_t vrun, int64_t tile,
+                                                                  int64_t tiles) {
+  const int64_t j = blockIdx.x / tiles, i0 = (blockIdx.x % tiles) * tile;
+  const int64_t i1 = i0 + tile < A ? i0 + tile : A;
+  const int64_t total = (i1 - i0) * vrun;
+  V* out = dst + (j * A + i0) * vrun;
+  for (int64_t k = threadIdx.x; k < total; k += kThreads) {
+    const int64_t i = i0 + k / vrun, c = k % vrun;
+    out[k] = src[(i * B + j) * vrun + c];
+  }
+}
+
+template <typename V>
+cudaError_t launch_transpose(const void* src, void* dst, int64_t A, int64_t B, int64_t run_bytes, cudaStream_t cs) {
+  const int64_t vrun = run_bytes / int64_t(sizeof(V));
+  const int64_t tile = (65536 / run_bytes) > 0 ? (65536 / run_bytes) : 1;   // ~64 KB per CTA
+  const int64_t tiles = (A + tile - 1) / tile;
+  const int64_t grid = B * tiles;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  transpose_runs_kernel<V><<<unsigned(grid), kThreads, 0, cs>>>(static_cast<const V*>(src), static_cast<V*>(dst), A, B,
+                                                               vrun, tile, tiles);
+  return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace uly
 
@@ -305,4 +336,23 @@ extern "C" uly_status ulysses_seq_to_head(const void* x_seq, void* x_head, int64
 extern "C" uly_status ulysses_head_to_seq(const void* x_head, void* x_seq, int64_t b, int64_t n, int64_t H,
                                           int64_t d, int32_t P, uly_dtype dt, void* stream) {
   return uly::relayout<false>(x_head, x_seq, b, n, H, d, P, dt, stream);
+}
+
+extern "C" uly_status ulysses_transpose_runs(const void* src, void* dst, int64_t A, int64_t B, int64_t run_bytes,
+                                             void* stream) {
+  using namespace uly;
+  if (!src || !dst || A < 1 || B < 1 || run_bytes < 1) return ULY_ERR_INVALID_ARG;
+  int64_t bytes;
+  if (!checked_mul(A, B, &bytes) || !checked_mul(bytes, run_bytes, &bytes)) return ULY_ERR_INVALID_ARG;
+  if (overlaps(src, size_t(bytes), dst, size_t(bytes))) return ULY_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  const bool a16 = aligned(src, 16) && aligned(dst, 16), a8 = aligned(src, 8) && aligned(dst, 8),
+             a4 = aligned(src, 4) && aligned(dst, 4), a2 = aligned(src, 2) && aligned(dst, 2);
+  if (run_bytes % 16 == 0 && a16) e = launch_transpose<uint4>(src, dst, A, B, run_bytes, cs);
+  else if (run_bytes % 8 == 0 && a8) e = launch_transpose<uint2>(src, dst, A, B, run_bytes, cs);
+  else if (run_bytes % 4 == 0 && a4) e = launch_transpose<uint32_t>(src, dst, A, B, run_bytes, cs);
+  else if (run_bytes % 2 == 0 && a2) e = launch_transpose<uint16_t>(src, dst, A, B, run_bytes, cs);
+  else e = launch_transpose<uint8_t>(src, dst, A, B, run_bytes, cs);
+  return cuda_status(e);
 }
