@@ -89,3 +89,47 @@ def test_all_to_all_round_trip_over_gloo(world):
     assert [r[0] for r in res] == list(range(world))
     assert all(r[1] and r[2] and r[3] is True for r in res), res
     assert all(p.exitcode == 0 for p in procs)
+
+
+def _rank_dies(rank, world, port, root, out):
+    sys.path.insert(0, root)
+    import time
+    import torch
+    import torch.distributed as dist
+    from ulysses_head_attention_b200 import distributed as udist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out.put((rank, "left before the exchange"))
+        out.close()
+        out.join_thread()               # the message is out before the process goes
+        os._exit(0)                     # a rank that never joins the all-to-all
+    t0 = time.time()
+    try:
+        udist.seq_to_head(torch.zeros((1, 4, 2 * world, 2)), transpose=numpy_transpose, exchange=gloo_exchange)
+        out.put((rank, "completed"))
+    except Exception as e:               # the survivor must get an error, not hang
+        out.put((rank, f"error after {time.time() - t0:.1f}s: {type(e).__name__}"))
+    out.close()
+    out.join_thread()
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_exchange_with_an_error():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies, args=(r, 2, port, ROOT, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        res = dict(out.get(timeout=120) for _ in range(2))
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert res[1] == "left before the exchange"
+    assert res[0].startswith("error after"), res[0]
