@@ -19,7 +19,7 @@
 //               block's 64 values of -LSE*log2e followed by its 64 values of
 //               -D (negated so they feed packed fused multiply-adds).
 //  * bwd_dkdv:  one CTA per (rank, batch row, kv head, 128-key tile),
-//               heaviest first.  Loops over the G query heads of the kv head
+//               group by group, heaviest key tile first in each.  Loops over the G query heads of the kv head
 //               and the 128-row query tiles that can see the key tile:
 //                 warp 0      TMA producer (K, V once; Q, dO, row stats ring)
 //                 warp 1      TMEM owner, single-thread MMA issuer
@@ -194,9 +194,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int per_tile = p.P_sel * p.b * p.hkv;
-  const int kt = int(blockIdx.x / per_tile);
-  int rem = int(blockIdx.x % per_tile);
+  // (rank, batch row, kv head) groups run one after another, so the CTAs
+  // resident at any time share their query heads' Q / dO tiles in L2; inside
+  // a group the key tiles go heaviest (first) to lightest (last)
+  const int nkt = int((p.n + BKV - 1) / BKV);
+  const int kt = int(blockIdx.x % nkt);
+  int rem = int(blockIdx.x / nkt);
   const int g = rem % p.hkv;
   rem /= p.hkv;
   const int bb = rem % p.b;
