@@ -48,11 +48,11 @@ KERNEL_SOURCES = {
                              ("ulysses_head_attention_b200/csrc/sm100.cuh", None, None),
                              ("ulysses_head_attention_b200/csrc/common.cuh", None, None)),
 }
-# llama8b_p4_n32k, one launch (ncu, dram__bytes_read.sum 4.28 GB + dram__bytes_write.sum 246.83 MB,
-# as ncu printed them); see profiles/attn_bwd_dkdv_kernel.md
+# llama8b_p4_n32k, one launch: ncu dram__bytes_read.sum 692503552 + dram__bytes_write.sum 244745216
+# bytes (--print-units base); see profiles/attn_bwd_dkdv_kernel.md
 TRAFFIC = {
-    "attn_bwd_dkdv_kernel": {"workload": "llama8b_p4_n32k", "bytes_per_launch": 4.28e9 + 246.83e6,
-                             "sources_sha256": "f8604d95571327241bbb0f8de753d89c5727e5512e23054c983a3c7c5fbe4b43"},
+    "attn_bwd_dkdv_kernel": {"workload": "llama8b_p4_n32k", "bytes_per_launch": 692503552 + 244745216,
+                             "sources_sha256": "512677325366df9ff6cfb9268a1e45f8125519207cc557136848e3c3049a48c8"},
 }
 
 
@@ -393,71 +393,81 @@ def run_ours(args, w):
 
     # ---- ring attention over R key blocks (forward + LSE merge, then the
     # blocks' backward from the merged O / LSE), timed on its own
-    R = 4
-    cuts = [n * i // R for i in range(R + 1)]
-    o_parts = torch.empty((R,) + tuple(o_head.shape), dtype=f32, device=dev)
-    l_parts = torch.empty((R,) + tuple(lse.shape), dtype=f32, device=dev)
-    o_ring, l_ring = torch.empty_like(o_head), torch.empty_like(lse)
-    g_ring = {k: torch.empty_like(g_head[k]) for k in g_head}
+    extras = {}
 
-    def ring_fwd():
-        for i in range(R):
-            uly.ulysses_attn_fwd_kv_range(head["q"], head["k"], head["v"], pos, o_parts[i], l_parts[i], ws_f,
-                                          cuts[i], cuts[i + 1])
-        uly.ulysses_attn_lse_merge(o_parts, l_parts, o_ring, l_ring, hkv)
+    def measure_ring():
+        R = 4
+        cuts = [n * i // R for i in range(R + 1)]
+        o_parts = torch.empty((R,) + tuple(o_head.shape), dtype=f32, device=dev)
+        l_parts = torch.empty((R,) + tuple(lse.shape), dtype=f32, device=dev)
+        o_ring, l_ring = torch.empty_like(o_head), torch.empty_like(lse)
+        g_ring = {k: torch.empty_like(g_head[k]) for k in g_head}
 
-    def ring_bwd():
-        for i in range(R):
-            uly.ulysses_attn_bwd_kv_range(head["q"], head["k"], head["v"], o_ring, l_ring, head["do"], pos,
-                                          g_ring["q"], g_ring["k"], g_ring["v"], ws_b, cuts[i], cuts[i + 1])
+        def ring_fwd():
+            for i in range(R):
+                uly.ulysses_attn_fwd_kv_range(head["q"], head["k"], head["v"], pos, o_parts[i], l_parts[i], ws_f,
+                                              cuts[i], cuts[i + 1])
+            uly.ulysses_attn_lse_merge(o_parts, l_parts, o_ring, l_ring, hkv)
 
-    ring_fwd()
-    ring_bwd()
-    torch.cuda.synchronize()
-    rf = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    reps = 3
-    rf[0].record(stream)
-    for _ in range(reps):
+        def ring_bwd():
+            for i in range(R):
+                uly.ulysses_attn_bwd_kv_range(head["q"], head["k"], head["v"], o_ring, l_ring, head["do"], pos,
+                                              g_ring["q"], g_ring["k"], g_ring["v"], ws_b, cuts[i], cuts[i + 1])
+
         ring_fwd()
-    rf[1].record(stream)
-    for _ in range(reps):
         ring_bwd()
-    rf[2].record(stream)
-    torch.cuda.synchronize()
-    for ws in (ws_f, ws_b):
-        if uly.ulysses_workspace_status(ws) != 0:
-            raise RuntimeError("a kernel reported a pipeline timeout in the ring measurement")
-    ring_fwd_ms = rf[0].elapsed_time(rf[1]) / reps
-    ring_bwd_ms = rf[1].elapsed_time(rf[2]) / reps
-    ring_stat = {"blocks": R, "fwd_ms": ring_fwd_ms, "fwd_tflops": fwd_flops / (ring_fwd_ms * 1e-3) / 1e12,
-                 "bwd_ms_per_block_pass": ring_bwd_ms, "bwd_tflops": bwd_flops / (ring_bwd_ms * 1e-3) / 1e12,
-                 "launches": {"fwd": R * 2 + 1, "bwd": R * 4},
-                 "note": "keys cut into R equal blocks; forward = R key-range forwards + one LSE merge; "
-                         "backward = R key-range backwards from the merged O and LSE (one block's dQ share each)"}
+        torch.cuda.synchronize()
+        rf = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        reps = 3
+        rf[0].record(stream)
+        for _ in range(reps):
+            ring_fwd()
+        rf[1].record(stream)
+        for _ in range(reps):
+            ring_bwd()
+        rf[2].record(stream)
+        torch.cuda.synchronize()
+        for ws in (ws_f, ws_b):
+            if uly.ulysses_workspace_status(ws) != 0:
+                raise RuntimeError("a kernel reported a pipeline timeout in the ring measurement")
+        ring_fwd_ms = rf[0].elapsed_time(rf[1]) / reps
+        ring_bwd_ms = rf[1].elapsed_time(rf[2]) / reps
+        ring_stat = {"blocks": R, "fwd_ms": ring_fwd_ms, "fwd_tflops": fwd_flops / (ring_fwd_ms * 1e-3) / 1e12,
+                     "bwd_ms_per_block_pass": ring_bwd_ms, "bwd_tflops": bwd_flops / (ring_bwd_ms * 1e-3) / 1e12,
+                     "launches": {"fwd": R * 2 + 1, "bwd": R * 4},
+                     "note": "keys cut into R equal blocks; forward = R key-range forwards + one LSE merge; "
+                             "backward = R key-range backwards from the merged O and LSE (one block's dQ share each)"}
+        extras["ring_attention"] = ring_stat
 
     # ---- weighted SP loss aggregation (the custom training loop's per-rank loss
     # weighting), timed on its own: it needs a model's per-rank losses, which
     # this path does not produce, so it is not part of the step
-    lab = synthetic.sft_shift_labels(w.wid, x["lengths"])
-    lab_sh = torch.from_numpy(np.ascontiguousarray(lab.reshape(b, P, m).transpose(1, 0, 2))).to(dev)
-    l_in = torch.from_numpy(synthetic.rank_losses(w.wid, P)).to(dev)
-    l_out, l_good, l_dl = (torch.empty(1, device=dev), torch.empty(P, dtype=torch.int64, device=dev),
-                           torch.empty(P, device=dev))
-    for _ in range(5):
-        uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
-    torch.cuda.synchronize()
-    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 50
-    s3.record(stream)
-    for _ in range(reps):
-        uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
-    e3.record(stream)
-    torch.cuda.synchronize()
-    loss_us = s3.elapsed_time(e3) * 1e3 / reps
-    loss_bytes = lab_sh.numel() * 8 + 3 * P * 8 + 4
-    loss_stat = {"us_per_call": loss_us, "bytes_per_call": loss_bytes,
-                 "gbs": loss_bytes / (loss_us * 1e-6) / 1e9, "launches_per_call": 2,
-                 "labels": "packed SFT: per sample a U[0.1, 0.6) prompt fraction and the last position are -100"}
+    def measure_loss():
+        lab = synthetic.sft_shift_labels(w.wid, x["lengths"])
+        lab_sh = torch.from_numpy(np.ascontiguousarray(lab.reshape(b, P, m).transpose(1, 0, 2))).to(dev)
+        l_in = torch.from_numpy(synthetic.rank_losses(w.wid, P)).to(dev)
+        l_out, l_good, l_dl = (torch.empty(1, device=dev), torch.empty(P, dtype=torch.int64, device=dev),
+                               torch.empty(P, device=dev))
+        for _ in range(5):
+            uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
+        torch.cuda.synchronize()
+        s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 50
+        s3.record(stream)
+        for _ in range(reps):
+            uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
+        e3.record(stream)
+        torch.cuda.synchronize()
+        loss_us = s3.elapsed_time(e3) * 1e3 / reps
+        loss_bytes = lab_sh.numel() * 8 + 3 * P * 8 + 4
+        loss_stat = {"us_per_call": loss_us, "bytes_per_call": loss_bytes,
+                     "gbs": loss_bytes / (loss_us * 1e-6) / 1e9, "launches_per_call": 2,
+                     "labels": "packed SFT: per sample a U[0.1, 0.6) prompt fraction and the last position are -100"}
+        extras["sp_loss_aggregate"] = loss_stat
+
+    if not args.no_extras:
+        measure_ring()
+        measure_loss()
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -478,8 +488,7 @@ def run_ours(args, w):
             "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
             "bwd_flops_with_recompute_convention": 10 * d * hq * pairs,
             "peaks": peaks,
-            "sp_loss_aggregate": loss_stat,
-            "ring_attention": ring_stat,
+            **extras,
         },
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": dom_tf / peak_t, "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
@@ -550,6 +559,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the separately timed ring-attention and loss-aggregation measurements")
     ap.add_argument("--profile-case", action="store_true",
                     help="run one small forward + backward for an ncu capture, then exit (no timing, no JSON)")
     args = ap.parse_args()
