@@ -118,21 +118,27 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples (every 50 ms) of SM clock and clock-event reasons; only
+    samples read inside the marked window (the timed region) are kept."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.sw_power_cap,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.active")
+    # NVML clock-event reason bits, for the names of whatever else is active
+    BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.lines = []
+        self.window = (0.0, float("inf"))
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
@@ -140,22 +146,29 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)   # let the last in-window line arrive
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=5)
-        sm, smax, reasons = [], None, set()
+        sm, smax, reasons, masks = [], None, set(), set()
         names = ("sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
-        for ln in self.lines:
+        t0, t1 = self.window
+        for t, ln in self.lines:
+            if not (t0 <= t <= t1 + 0.06):
+                continue
             parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 7:
+            if len(parts) < 8:
                 continue
             try:
                 sm.append(float(parts[0]))
@@ -165,8 +178,17 @@ class ClockSampler:
             for nm, val in zip(names, parts[3:7]):
                 if val.lower() == "active":
                     reasons.add(nm)
+            try:
+                mask = int(parts[7], 16)
+            except ValueError:
+                continue
+            masks.add(mask)
+            for bit, nm in self.BITS.items():
+                if mask & bit:
+                    reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_mhz_min": min(sm) if sm else None, "sm_mhz_max": max(sm) if sm else None,
+                "reasons": sorted(reasons), "active_masks": sorted(hex(m) for m in masks), "samples": len(sm)}
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
@@ -326,12 +348,14 @@ def run_ours(args, w):
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
+    t_region0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for i in range(args.steps):
         step(evs[i], kevs[i])
     end.record(stream)
     torch.cuda.synchronize()
+    clocks.mark(t_region0, time.time())
     barrier()
     clk = clocks.stop()
     ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
@@ -554,7 +578,7 @@ def run_profile_case():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
