@@ -19,17 +19,20 @@
 //               block's 64 values of -LSE*log2e followed by its 64 values of
 //               -D (negated so they feed packed fused multiply-adds).
 //  * bwd_dkdv:  one CTA per (rank, batch row, kv head, 128-key tile),
-//               group by group, heaviest key tile first in each.  Loops over the G query heads of the kv head
-//               and the 128-row query tiles that can see the key tile:
-//                 warp 0      TMA producer (K, V once; Q, dO, row stats ring)
-//                 warp 1      TMEM owner, single-thread MMA issuer
+//               group by group, heaviest key tile first in each.  Loops over
+//               the G query heads of the kv head and the 128-row query tiles
+//               that can see the key tile:
+//                 warp 0      TMA producer: K, V once; the Q ring (3 stages)
+//                 warp 2      TMA producer: the dO + row-statistics ring (2)
+//                 warp 1      TMEM owner; issues the MMAs as a converged warp
 //                 warps 4..11 thread = key row, two warpgroups each taking
-//                             64 of the 128 query columns: P^T, dS^T from S^T, dP^T
+//                             64 of the 128 query columns
 //               S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128: the
-//               shape runs the tensor core at full rate, N = 64 does not) go
-//               to TMEM; P^T and dS^T go back over them as bf16 and feed
+//               shape runs the tensor core at full rate, N = 64 does not)
+//               go to TMEM; the softmax frees S^T as soon as it has read it,
+//               then writes P^T and dS^T as bf16 over dP^T, and they feed
 //               dV += P^T dO, dK += dS^T Q as A-from-TMEM MMAs accumulating
-//               in TMEM across the whole group.
+//               in TMEM across the whole group (details at the kernel).
 //               TMEM: dK [0,128) dV [128,256) S^T [256,384) dP^T [384,512).
 //  * bwd_dq:    one CTA per (rank, batch row, query head, 128-row tile),
 //               heaviest first; the forward's structure (K and V rings fed
@@ -40,6 +43,8 @@
 //               warpgroups (64 columns each) turn them into dS (bf16, over S)
 //               and dQ += dS K accumulates in TMEM.
 //               TMEM: S_0 [0,128) S_1 [128,256) dP [256,384) dQ [384,512).
+// Every kernel also takes a key range [k_lo, k_hi) (the whole sequence for
+// ulysses_attn_bwd): one ring block's share of the gradients.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>

@@ -13,13 +13,14 @@
 // traffic per flop (every CTA streams its head's whole visible K/V prefix).
 //   warp 0       TMA producer: Q tiles once, then K tiles into a 2-stage ring
 //   warp 2       TMA producer: V tiles into a 2-stage ring
-//   warp 1       TMEM owner and single-thread tcgen05 MMA issuer
+//   warp 1       TMEM owner; issues the tcgen05 MMAs as a converged warp
+//                (elect.sync picks the issuing lane)
 //   warps 4..7   softmax of query tile 0, thread = query row
 //   warps 8..11  softmax of query tile 1
 // Per key tile j the MMAs are issued as PV_0(j-1), S_0(j), PV_1(j-1), S_1(j)
 // (S_q = Q_q K^T, PV_q: O_q += P_q V), each pair as one burst after all of
-// its waits (a wait by the issuing thread stalls MMA issue for a few hundred
-// cycles, so waits are batched).  While one warpgroup turns S into P the
+// its waits (a wait in the issuing warp leaves the tensor pipe short of
+// work, so waits are batched).  While one warpgroup turns S into P the
 // tensor core works on the other tile, and S_q(j) completing implies
 // PV_q(j-1) completed, so the lazy O rescale needs no extra wait.  The
 // softmax writes P (bf16) back over S; PV reads it as the A operand from TMEM.
@@ -29,7 +30,9 @@
 // Keys a tile cannot see are never loaded: a tile's key range starts at the
 // key tile holding the sample start of its first row and ends at its
 // diagonal; per-element masks run only on tiles that straddle the diagonal
-// or a sample start.
+// or a sample start.  A key range [k_lo, k_hi) (the whole sequence for
+// ulysses_attn_fwd; one ring block for ulysses_attn_fwd_kv_range) clips both;
+// rows that see no key of it get O = 0 and LSE = -inf.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
