@@ -576,15 +576,20 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int per_tile = p.P_sel * p.b * p.hq;
-  const int tile = p.ntiles - 1 - int(blockIdx.x / per_tile);
-  int rem = int(blockIdx.x % per_tile);
-  const int h = rem % p.hq;
-  rem /= p.hq;
+  // (rank, batch row, kv head) groups one after another (resident CTAs share
+  // one kv head's K / V in L2); inside a group: heaviest tile first, the G
+  // query heads of a tile next to each other
+  const int per_group = p.ntiles * p.G;
+  const int w = int(blockIdx.x % per_group);
+  int rem = int(blockIdx.x / per_group);
+  const int tile = p.ntiles - 1 - w / p.G;
+  const int hkv = p.hq / p.G;
+  const int g = rem % hkv;
+  const int h = g * p.G + w % p.G;
+  rem /= hkv;
   const int bb = rem % p.b;
   const int r = p.rank0 + rem / p.b;
   const int rb = r * p.b + bb;
-  const int g = h / p.G;
   const int64_t t0 = int64_t(tile) * BM;
   const int64_t last_row = (t0 + BM - 1 < p.n - 1) ? (t0 + BM - 1) : (p.n - 1);
   const int32_t* ss = p.segstart + int64_t(bb) * p.n;

@@ -123,15 +123,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work item: heaviest (last) pairs of query tiles first
-  const int per_pair = p.P_sel * p.b * p.hq;
-  const int pair = p.npairs - 1 - int(blockIdx.x / per_pair);
-  int rem = int(blockIdx.x % per_pair);
-  const int j = rem % p.hq;
-  rem /= p.hq;
+  // (rank, batch row, kv head) groups run one after another, so resident CTAs
+  // share one kv head's K / V in L2; inside a group: heaviest pair first,
+  // the G query heads of a pair next to each other
+  const int per_group = p.npairs * p.G;
+  const int w = int(blockIdx.x % per_group);
+  int rem = int(blockIdx.x / per_group);
+  const int pair = p.npairs - 1 - w / p.G;
+  const int hkv = p.hq / p.G;
+  const int g = rem % hkv;
+  const int j = g * p.G + w % p.G;
+  rem /= hkv;
   const int bb = rem % p.b;
   const int r = p.rank0 + rem / p.b;
   const int rb = r * p.b + bb;
-  const int g = j / p.G;
   const int32_t* ss = p.segstart + int64_t(bb) * p.n;
   const TileRange tr0 = tile_range(ss, p.n, 2 * pair, p.ntiles, p.k_lo, p.k_hi);
   const TileRange tr1 = tile_range(ss, p.n, 2 * pair + 1, p.ntiles, p.k_lo, p.k_hi);
