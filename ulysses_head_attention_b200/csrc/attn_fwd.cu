@@ -50,7 +50,10 @@ constexpr int BN = 128;        // keys per tile
 constexpr int NS = 2;          // K/V stages
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
-constexpr int kMufuPairs = 40;              // of the 64 column pairs per row, the rest use exp2_poly
+#ifndef FWD_MUFU_PAIRS
+#define FWD_MUFU_PAIRS 48
+#endif
+constexpr int kMufuPairs = FWD_MUFU_PAIRS;  // of the 64 column pairs per row, the rest use exp2_poly
 
 struct Params {
   const int32_t* segstart;   // [b][n]
