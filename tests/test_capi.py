@@ -195,3 +195,85 @@ def test_transpose_rejects():
     assert uly.lib.ulysses_transpose_runs(F, F + G, 0, 2, 16, None) == INVALID
     assert uly.lib.ulysses_transpose_runs(F, F + G, 2, 2, 0, None) == INVALID
     assert uly.lib.ulysses_transpose_runs(F, F + 32, 2, 2, 16, None) == INVALID   # overlap
+
+
+def _attn_tensors(P=2, b=1, n=8, hq=2, hkv=1, d=4, o=torch.float32, g=torch.float32):
+    """Host tensors with the layouts of one attention call (never launched)."""
+    bf = torch.bfloat16
+    return dict(q_head=torch.zeros(P, b, n, hq, d, dtype=bf), k_head=torch.zeros(P, b, n, hkv, d, dtype=bf),
+                v_head=torch.zeros(P, b, n, hkv, d, dtype=bf), position_ids=torch.zeros(b, n, dtype=torch.int64),
+                o_head=torch.zeros(P, b, n, hq, d, dtype=o), lse=torch.zeros(P, b, hq, n),
+                do_head=torch.zeros(P, b, n, hq, d, dtype=bf), dq_head=torch.zeros(P, b, n, hq, d, dtype=g),
+                dk_head=torch.zeros(P, b, n, hkv, d, dtype=g), dv_head=torch.zeros(P, b, n, hkv, d, dtype=g),
+                ws=torch.zeros(256, dtype=torch.uint8))
+
+
+FWD_ARGS = ("q_head", "k_head", "v_head", "position_ids", "o_head", "lse", "ws")
+BWD_ARGS = ("q_head", "k_head", "v_head", "o_head", "lse", "do_head", "position_ids", "dq_head", "dk_head",
+            "dv_head", "ws")
+
+
+@pytest.mark.parametrize("name,bad,exc", [
+    ("v_head", torch.zeros(2, 1, 8, 2, 4, dtype=torch.bfloat16), ValueError),   # v heads differ from k
+    ("position_ids", torch.zeros(8, dtype=torch.int64), ValueError),            # not [b][n]
+    ("position_ids", torch.zeros(1, 8, dtype=torch.int32), TypeError),
+    ("o_head", torch.zeros(2, 1, 4, 2, 4), ValueError),                         # too few rows
+    ("o_head", torch.zeros(2, 1, 8, 2, 4, dtype=torch.float16), TypeError),
+    ("lse", torch.zeros(2, 1, 8, 2), ValueError),                               # [P][b][n][h], transposed
+    ("q_head", torch.zeros(2, 1, 8, 2, 4), TypeError),                          # fp32 q
+])
+def test_binding_checks_forward_layouts_before_launch(name, bad, exc):
+    """A mis-sized or mistyped tensor is refused by the binding, before any
+    pointer reaches the library (these are host tensors: nothing launches)."""
+    import ulysses_head_attention_b200 as uly
+    t = _attn_tensors()
+    t[name] = bad
+    args = [t[a] for a in FWD_ARGS]
+    for fn in (uly.ulysses_attn_fwd, lambda *a: uly.ulysses_attn_fwd_kv_range(*a, k_lo=0, k_hi=8)):
+        with pytest.raises(exc, match=name):
+            fn(*args)
+    with pytest.raises(exc, match=name):
+        uly.ulysses_attn_fwd_noalloc(*args[:-1])
+
+
+@pytest.mark.parametrize("name,bad,exc", [
+    ("do_head", torch.zeros(2, 1, 8, 2, 4), TypeError),                          # dO must be bf16
+    ("dq_head", torch.zeros(2, 1, 8, 1, 4), ValueError),
+    ("dk_head", torch.zeros(2, 1, 8, 1, 4, dtype=torch.bfloat16), TypeError),    # dtype differs from dq
+    ("dv_head", torch.zeros(2, 1, 8, 2, 4), ValueError),
+])
+def test_binding_checks_backward_layouts_before_launch(name, bad, exc):
+    import ulysses_head_attention_b200 as uly
+    t = _attn_tensors()
+    t[name] = bad
+    args = [t[a] for a in BWD_ARGS]
+    with pytest.raises(exc, match=name):
+        uly.ulysses_attn_bwd(*args)
+    with pytest.raises(exc, match=name):
+        uly.ulysses_attn_bwd_kv_range(*args, k_lo=0, k_hi=8)
+    with pytest.raises(exc, match=name):
+        uly.ulysses_attn_bwd_timed(*args, events=[None] * 5)
+
+
+def test_binding_refuses_host_tensors():
+    """Well-formed layouts on the host still never reach the library."""
+    import ulysses_head_attention_b200 as uly
+    t = _attn_tensors()
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        uly.ulysses_attn_fwd(*[t[a] for a in FWD_ARGS])
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        uly.ulysses_attn_bwd(*[t[a] for a in BWD_ARGS])
+
+
+def test_binding_checks_merge_layouts():
+    import ulysses_head_attention_b200 as uly
+    o_parts, lse_parts = torch.zeros(3, 2, 1, 8, 2, 4), torch.zeros(3, 2, 1, 2, 8)
+    o_head, lse = torch.zeros(2, 1, 8, 2, 4), torch.zeros(2, 1, 2, 8)
+    with pytest.raises(ValueError, match="lse_parts"):
+        uly.ulysses_attn_lse_merge(o_parts, lse_parts[:2], o_head, lse, h_kv=2)
+    with pytest.raises(ValueError, match="lse"):
+        uly.ulysses_attn_lse_merge(o_parts, lse_parts, o_head, lse[:, :, :1], h_kv=2)
+    with pytest.raises(ValueError, match="o_head"):
+        uly.ulysses_attn_lse_merge(o_parts, lse_parts, o_head[:1], lse, h_kv=2)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        uly.ulysses_attn_lse_merge(o_parts, lse_parts, o_head, lse, h_kv=2)

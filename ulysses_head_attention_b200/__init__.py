@@ -113,6 +113,58 @@ def _stream(stream: Optional[torch.cuda.Stream]) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+_BF16, _F32, _I64, _OUT = (torch.bfloat16,), (torch.float32,), (torch.int64,), (torch.bfloat16, torch.float32)
+
+
+def _expect(t, shape, dtypes, name: str) -> None:
+    """Shape and dtype of one argument: the kernels index every buffer by the
+    call's shape, so a smaller tensor would be read or written out of bounds."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} is {t.dtype}, expected {' or '.join(str(x) for x in dtypes)}")
+
+
+def _one_device(stream, **tensors) -> None:
+    """Every tensor on the CUDA device the kernels launch on (the stream's)."""
+    for name, t in tensors.items():
+        _dev(t, name)
+    dev = (stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device()))
+    for name, t in tensors.items():
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the launch is on {dev}")
+
+
+def _check_attn(q_head, k_head, v_head, position_ids, o_head, lse, stream, do_head=None, dq_head=None,
+                dk_head=None, dv_head=None, ws=None) -> None:
+    """Layouts of the attention calls (head layout, per virtual rank)."""
+    if not isinstance(q_head, torch.Tensor) or q_head.dim() != 5:
+        raise ValueError("q_head must be [P][b][n][h_q/P][d]")
+    P, b, n, hq, d = q_head.shape
+    if not isinstance(k_head, torch.Tensor) or k_head.dim() != 5:
+        raise ValueError("k_head must be [P][b][n][h_kv/P][d]")
+    hkv = k_head.shape[3]
+    _expect(q_head, (P, b, n, hq, d), _BF16, "q_head")
+    _expect(k_head, (P, b, n, hkv, d), _BF16, "k_head")
+    _expect(v_head, (P, b, n, hkv, d), _BF16, "v_head")
+    _expect(position_ids, (b, n), _I64, "position_ids")
+    _expect(o_head, (P, b, n, hq, d), _OUT, "o_head")
+    _expect(lse, (P, b, hq, n), _F32, "lse")
+    grads = {}
+    if do_head is not None:
+        _expect(do_head, (P, b, n, hq, d), _BF16, "do_head")
+        _expect(dq_head, (P, b, n, hq, d), _OUT, "dq_head")
+        _expect(dk_head, (P, b, n, hkv, d), (dq_head.dtype,), "dk_head")
+        _expect(dv_head, (P, b, n, hkv, d), (dq_head.dtype,), "dv_head")
+        grads = dict(do_head=do_head, dq_head=dq_head, dk_head=dk_head, dv_head=dv_head)
+    if ws is not None:
+        grads["ws"] = ws
+    _one_device(stream, q_head=q_head, k_head=k_head, v_head=v_head, position_ids=position_ids, o_head=o_head,
+                lse=lse, **grads)
+
+
 def make_shape(b: int, n: int, h_q: int, h_kv: int, d: int, P: int) -> UlyShape:
     return UlyShape(b, n, h_q, h_kv, d, P)
 
@@ -122,6 +174,7 @@ def ulysses_seq_to_head(x_seq: torch.Tensor, x_head: torch.Tensor, stream=None) 
     P, b, m, H, d = x_seq.shape
     if tuple(x_head.shape) != (P, b, m * P, H // P, d) or x_head.dtype != x_seq.dtype:
         raise ValueError("x_head shape/dtype does not match x_seq")
+    _one_device(stream, x_seq=x_seq, x_head=x_head)
     _check(lib.ulysses_seq_to_head(_dev(x_seq, "x_seq"), _dev(x_head, "x_head"), b, m * P, H, d, P,
                                    _dtype_code(x_seq), _stream(stream)), "ulysses_seq_to_head")
 
@@ -131,6 +184,7 @@ def ulysses_head_to_seq(x_head: torch.Tensor, x_seq: torch.Tensor, stream=None) 
     P, b, n, h, d = x_head.shape
     if tuple(x_seq.shape) != (P, b, n // P, h * P, d) or x_seq.dtype != x_head.dtype:
         raise ValueError("x_seq shape/dtype does not match x_head")
+    _one_device(stream, x_head=x_head, x_seq=x_seq)
     _check(lib.ulysses_head_to_seq(_dev(x_head, "x_head"), _dev(x_seq, "x_seq"), b, n, h * P, d, P,
                                    _dtype_code(x_head), _stream(stream)), "ulysses_head_to_seq")
 
@@ -142,6 +196,7 @@ def ulysses_kv_seq_to_head(x_seq: torch.Tensor, x_head: torch.Tensor, stream=Non
     h = H // P if H >= P else 1
     if tuple(x_head.shape) != (P, b, m * P, h, d) or x_head.dtype != x_seq.dtype:
         raise ValueError("x_head shape/dtype does not match x_seq")
+    _one_device(stream, x_seq=x_seq, x_head=x_head)
     _check(lib.ulysses_kv_seq_to_head(_dev(x_seq, "x_seq"), _dev(x_head, "x_head"), b, m * P, H, d, P,
                                       _dtype_code(x_seq), _stream(stream)), "ulysses_kv_seq_to_head")
 
@@ -153,6 +208,7 @@ def ulysses_kv_head_to_seq(x_head: torch.Tensor, x_seq: torch.Tensor, stream=Non
     h = H // P if H >= P else 1
     if tuple(x_head.shape) != (P, b, m * P, h, d) or x_head.dtype != x_seq.dtype:
         raise ValueError("x_seq shape/dtype does not match x_head")
+    _one_device(stream, x_head=x_head, x_seq=x_seq)
     _check(lib.ulysses_kv_head_to_seq(_dev(x_head, "x_head"), _dev(x_seq, "x_seq"), b, m * P, H, d, P,
                                       _dtype_code(x_seq), _stream(stream)), "ulysses_kv_head_to_seq")
 
@@ -162,6 +218,7 @@ def ulysses_transpose_runs(src: torch.Tensor, dst: torch.Tensor, A: int, B: int,
     """dst[j][i][:] = src[i][j][:] over runs of run_bytes bytes (i < A, j < B)."""
     if src.numel() * src.element_size() != A * B * run_bytes or dst.numel() * dst.element_size() != A * B * run_bytes:
         raise ValueError("buffer sizes do not match A * B * run_bytes")
+    _one_device(stream, src=src, dst=dst)
     _check(lib.ulysses_transpose_runs(_dev(src, "src"), _dev(dst, "dst"), A, B, run_bytes, _stream(stream)),
            "ulysses_transpose_runs")
 
@@ -190,12 +247,8 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 def ulysses_attn_fwd(q_head, k_head, v_head, position_ids, o_head, lse, ws, rank: int = -1,
                      softmax_scale: float = 0.0, stream=None) -> None:
     """Local causal attention of every rank (or `rank`) on its head slice."""
+    _check_attn(q_head, k_head, v_head, position_ids, o_head, lse, stream, ws=ws)
     shape = _attn_shape(q_head, k_head)
-    for t, nm in ((k_head, "k_head"), (v_head, "v_head"), (q_head, "q_head")):
-        if t.dtype != torch.bfloat16:
-            raise TypeError(f"{nm} must be bfloat16")
-    if position_ids.dtype != torch.int64:
-        raise TypeError("position_ids must be int64")
     _check(lib.ulysses_attn_fwd(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
                                 _dev(position_ids, "position_ids"), ctypes.byref(shape), rank, softmax_scale,
                                 _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
@@ -208,12 +261,8 @@ def ulysses_attn_fwd_noalloc(q_head, k_head, v_head, position_ids, o_head, lse, 
     """ulysses_attn_fwd without a workspace, for callers that cannot allocate
     device memory: the library's fixed per-GPU scratch (b*n <= 524288 tokens)
     is used instead.  Calls that overlap on the GPU race on that scratch."""
+    _check_attn(q_head, k_head, v_head, position_ids, o_head, lse, stream)
     shape = _attn_shape(q_head, k_head)
-    for t, nm in ((k_head, "k_head"), (v_head, "v_head"), (q_head, "q_head")):
-        if t.dtype != torch.bfloat16:
-            raise TypeError(f"{nm} must be bfloat16")
-    if position_ids.dtype != torch.int64:
-        raise TypeError("position_ids must be int64")
     _check(lib.ulysses_attn_fwd_noalloc(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
                                         _dev(position_ids, "position_ids"), ctypes.byref(shape), rank,
                                         softmax_scale, _dev(o_head, "o_head"), _dtype_code(o_head),
@@ -224,9 +273,9 @@ def ulysses_attn_fwd_noalloc(q_head, k_head, v_head, position_ids, o_head, lse, 
 def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse, do_head, position_ids, dq_head, dk_head, dv_head, ws,
                      rank: int = -1, softmax_scale: float = 0.0, stream=None) -> None:
     """Gradients dQ, dK, dV of the local attention (head layout)."""
+    _check_attn(q_head, k_head, v_head, position_ids, o_head, lse, stream, do_head, dq_head, dk_head, dv_head,
+                ws)
     shape = _attn_shape(q_head, k_head)
-    if dk_head.dtype != dq_head.dtype or dv_head.dtype != dq_head.dtype:
-        raise TypeError("dq/dk/dv must share one dtype")
     _check(lib.ulysses_attn_bwd(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
                                 _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
                                 _dev(do_head, "do_head"), _dev(position_ids, "position_ids"), ctypes.byref(shape),
@@ -242,9 +291,9 @@ def ulysses_attn_bwd_timed(q_head, k_head, v_head, o_head, lse, do_head, positio
     kernels (before sample tables, statistics, dK/dV, dQ; after dQ)."""
     if len(events) != 5:
         raise ValueError("five events are needed")
+    _check_attn(q_head, k_head, v_head, position_ids, o_head, lse, stream, do_head, dq_head, dk_head, dv_head,
+                ws)
     shape = _attn_shape(q_head, k_head)
-    if dk_head.dtype != dq_head.dtype or dv_head.dtype != dq_head.dtype:
-        raise TypeError("dq/dk/dv must share one dtype")
     handles = []
     for ev in events:
         if ev.cuda_event == 0:   # torch creates the handle lazily, at the first record
@@ -274,6 +323,7 @@ def ulysses_sp_loss_aggregate(losses, shift_labels, loss, good, dlosses, ignore_
     P, b, m = shift_labels.shape
     if losses.numel() != P or good.numel() != P or dlosses.numel() != P or loss.numel() != 1:
         raise ValueError("losses, good and dlosses need P elements, loss one")
+    _one_device(stream, losses=losses, shift_labels=shift_labels, loss=loss, good=good, dlosses=dlosses)
     _check(lib.ulysses_sp_loss_aggregate(_dev(losses, "losses"), _dev(shift_labels, "shift_labels"), b, m * P, P,
                                          ignore_index, _dev(loss, "loss"), _dev(good, "good"),
                                          _dev(dlosses, "dlosses"), _stream(stream)),
@@ -283,6 +333,7 @@ def ulysses_sp_loss_aggregate(losses, shift_labels, loss, good, dlosses, ignore_
 def ulysses_attn_fwd_kv_range(q_head, k_head, v_head, position_ids, o_head, lse, ws, k_lo: int, k_hi: int,
                               rank: int = -1, softmax_scale: float = 0.0, stream=None) -> None:
     """Forward over the keys [k_lo, k_hi) only (one ring block)."""
+    _check_attn(q_head, k_head, v_head, position_ids, o_head, lse, stream, ws=ws)
     shape = _attn_shape(q_head, k_head)
     _check(lib.ulysses_attn_fwd_kv_range(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
                                          _dev(position_ids, "position_ids"), ctypes.byref(shape), rank,
@@ -295,9 +346,9 @@ def ulysses_attn_bwd_kv_range(q_head, k_head, v_head, o_head, lse, do_head, posi
                               ws, k_lo: int, k_hi: int, rank: int = -1, softmax_scale: float = 0.0,
                               stream=None) -> None:
     """One key block's share of the backward, given the merged O and LSE."""
+    _check_attn(q_head, k_head, v_head, position_ids, o_head, lse, stream, do_head, dq_head, dk_head, dv_head,
+                ws)
     shape = _attn_shape(q_head, k_head)
-    if dk_head.dtype != dq_head.dtype or dv_head.dtype != dq_head.dtype:
-        raise TypeError("dq/dk/dv must share one dtype")
     _check(lib.ulysses_attn_bwd_kv_range(_dev(q_head, "q_head"), _dev(k_head, "k_head"), _dev(v_head, "v_head"),
                                          _dev(o_head, "o_head"), _dtype_code(o_head), _dev(lse, "lse"),
                                          _dev(do_head, "do_head"), _dev(position_ids, "position_ids"),
@@ -312,9 +363,13 @@ def ulysses_attn_lse_merge(o_parts, lse_parts, o_head, lse, h_kv: int, stream=No
     float32 (B, P, b, h, n) -> o_head (P, b, n, h, d), lse (P, b, h, n)."""
     if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32 or lse.dtype != torch.float32:
         raise TypeError("o_parts, lse_parts and lse must be float32")
+    if o_parts.dim() != 6:
+        raise ValueError("o_parts must be [B][P][b][n][h_q/P][d]")
     B, P, b, n, h, d = o_parts.shape
-    if tuple(lse_parts.shape) != (B, P, b, h, n) or tuple(o_head.shape) != (P, b, n, h, d):
-        raise ValueError("shapes do not match")
+    _expect(lse_parts, (B, P, b, h, n), _F32, "lse_parts")
+    _expect(o_head, (P, b, n, h, d), _OUT, "o_head")
+    _expect(lse, (P, b, h, n), _F32, "lse")
+    _one_device(stream, o_parts=o_parts, lse_parts=lse_parts, o_head=o_head, lse=lse)
     shape = UlyShape(b, n, h * P, h_kv, d, P)
     _check(lib.ulysses_attn_lse_merge(_dev(o_parts, "o_parts"), _dev(lse_parts, "lse_parts"), B,
                                       ctypes.byref(shape), _dev(o_head, "o_head"), _dtype_code(o_head),
