@@ -277,3 +277,19 @@ def test_binding_checks_merge_layouts():
         uly.ulysses_attn_lse_merge(o_parts, lse_parts, o_head[:1], lse, h_kv=2)
     with pytest.raises(ValueError, match="CUDA tensor"):
         uly.ulysses_attn_lse_merge(o_parts, lse_parts, o_head, lse, h_kv=2)
+
+
+@no_gpu
+def test_noalloc_forward_refuses_before_touching_the_device():
+    """Bad shapes and shapes beyond the fixed scratch (b * n > 524288 tokens)
+    are refused on the host, before the scratch lookup or any launch."""
+    import ulysses_head_attention_b200 as uly
+    G = 1 << 30
+
+    def call(s, rank=-1):
+        return uly.lib.ulysses_attn_fwd_noalloc(F, F + G, F + 2 * G, F + 3 * G, ctypes.byref(s), rank, 0.0,
+                                                F + 4 * G, 1, F + 5 * G, None)
+    assert call(shape(n=1000, P=16)) == INVALID
+    assert call(shape(b=1, n=1 << 20)) == WORKSPACE
+    assert call(shape(b=2, n=1 << 19)) == WORKSPACE
+    assert uly.ulysses_attn_fwd_workspace(shape(b=1, n=1 << 19)) <= 256 + 2 * 4 * (1 << 19)
