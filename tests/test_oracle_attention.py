@@ -60,6 +60,9 @@ def test_segment_tables(pos):
     seg = oracle.segment_ids(pos)
     for t in range(len(pos)):
         assert (seg == seg[t]).sum() == e[t] - s[t]
+    # sample indices count from 0 at token 0, one up at every later start
+    assert seg[0] == 0
+    assert np.array_equal(np.diff(seg), (pos[1:] == 0).astype(seg.dtype))
 
 
 def test_packed_visibility_golden():

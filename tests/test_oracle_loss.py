@@ -81,3 +81,12 @@ def test_single_rank_is_its_own_loss():
     labels = np.array([[[3, -100, 4]]])
     loss, good, grad = oracle.sp_loss_aggregate(np.array([2.5]), labels)
     assert (loss, int(good[0]), grad[0]) == (2.5, 2, 1.0)
+
+
+def test_ignore_index_is_the_only_excluded_label():
+    """Only labels equal to the ignore index are left out: with ignore_index
+    = -1, the -100 labels count and the -1 labels do not."""
+    labels = np.array([[[-1, -100, 7]], [[-1, -1, -1]]])
+    loss, good, grad = oracle.sp_loss_aggregate(np.array([3.0, float("nan")]), labels, ignore_index=-1)
+    assert good.tolist() == [2, 0]
+    assert (loss, grad.tolist()) == (3.0, [1.0, 0.0])

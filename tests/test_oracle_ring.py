@@ -92,3 +92,28 @@ def test_block_backward_shares_add_up(cuts):
         assert np.allclose(gk[a:b], dk_ref[a:b], atol=1e-11) and not gk[:a].any() and not gk[b:].any()
         assert np.allclose(gv[a:b], dv_ref[a:b], atol=1e-11) and not gv[:a].any() and not gv[b:].any()
     assert np.allclose(dq, dq_ref, atol=1e-11)
+
+
+@pytest.mark.parametrize("base", [0.0, 1000.0, -1000.0, 700.0])
+def test_merge_closed_form_at_extreme_lse(base):
+    """Two blocks with LSE base and base + ln 3 weigh their outputs 1/4 and
+    3/4, and the merged LSE is base + ln 4, however large |base| is (the
+    merge must not form exp(LSE) itself)."""
+    o = np.zeros((2, 1, 1, 1, 1, 2))
+    o[0, ..., 0] = 1.0
+    o[1, ..., 1] = 1.0
+    l = np.array([base, base + math.log(3.0)]).reshape(2, 1, 1, 1, 1)
+    O, L = oracle.lse_merge(o, l)
+    # base + ln 3 is stored to the ulp of |base| (1.1e-13 at 1000), which the
+    # weights inherit
+    assert np.allclose(O[0, 0, 0, 0], [0.25, 0.75], rtol=0, atol=1e-12)
+    assert L[0, 0, 0, 0] == pytest.approx(base + math.log(4.0), abs=1e-12)
+
+
+def test_merge_of_blocks_far_apart_keeps_the_dominant_one():
+    """LSEs 800 and -800: the second block's weight exp(-1600) is 0 in any
+    float format, so the merge returns the first block unchanged."""
+    o = np.stack([np.full((1, 1, 1, 1, 3), 2.0), np.full((1, 1, 1, 1, 3), -5.0)])
+    l = np.array([800.0, -800.0]).reshape(2, 1, 1, 1, 1)
+    O, L = oracle.lse_merge(o, l)
+    assert np.array_equal(O[0, 0, 0, 0], [2.0, 2.0, 2.0]) and L[0, 0, 0, 0] == 800.0
