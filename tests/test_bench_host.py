@@ -1,7 +1,7 @@
 """Host-side pieces of bench.py that decide what the JSON line says, on CPU:
 the clock record of the timed region, the recorded DRAM traffic and when it
-stops applying, the measured-peak file and its fallback, and the causal pair
-count behind the FLOP figures."""
+stops applying, the measured-peak file and its fallback, the causal pair
+count behind the FLOP figures, and the reference (CPU oracle) arm's line."""
 import json
 import sys
 
@@ -104,3 +104,24 @@ def test_pair_count_is_the_causal_segmented_mask(lengths):
         seg = [i for i, L in enumerate(row) for _ in range(L)]
         brute += sum(1 for i in range(len(seg)) for j in range(i + 1) if seg[i] == seg[j])
     assert bench.pairs_of(lengths) == brute
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` (the CPU oracle arm) prints one JSON line
+    with the keys the driver reads, on a small workload."""
+    import os
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_p2_n256", "--steps", "2", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=300, env=dict(os.environ, RANK="0"))
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["unit"] == "TFLOP/s" and out["value"] > 0
+    assert out["metric"] == bench.METRIC and out["higher_is_better"] is True
+    assert (out["steps"], out["warmup"], out["n_gpus"]) == (2, 1, 1)
+    assert out["config"]["workload"] == "tiny_p2_n256"
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
+    assert out["e2e"] == {"value": out["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
