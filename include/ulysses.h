@@ -37,7 +37,8 @@
  *    `stream` is a cudaStream_t (NULL = legacy default stream), passed as
  *    void* so this header needs no CUDA header.
  *  - Calls only enqueue work on `stream` and return; results are valid once
- *    the stream has run.  Outputs are fully overwritten.  The library
+ *    the stream has run.  Outputs are fully overwritten (the attention
+ *    calls' rank >= 0 mode: that rank's part of them).  The library
  *    allocates no device memory; scratch space is the caller's workspace,
  *    sized by the *_workspace queries.  The only mutable global state is
  *    ulysses_attn_fwd_noalloc's fixed per-GPU scratch array (see there),
