@@ -117,3 +117,37 @@ def test_kv_all_to_alls_on_gpu_equal_the_one_gpu_relayouts(cuda_device, P, H_kv,
     back = torch.empty((P, b, m, H_kv, d), dtype=torch.float32, device=cuda_device)
     uly.ulysses_kv_head_to_seq(gs, back)
     assert torch.equal(grads, back)
+
+
+def _fake_kv_seq_to_head(x_seq, x_head, stream=None):
+    """The binding's contract and shape rule for ulysses_kv_seq_to_head, on host tensors."""
+    P, b, m, H, d = x_seq.shape
+    assert tuple(x_head.shape) == (P, b, m * P, H // P if H >= P else 1, d) and x_head.dtype == x_seq.dtype
+    assert x_seq.is_contiguous() and x_head.is_contiguous() and x_seq.dtype == torch.bfloat16
+    x_head.view(torch.int16).numpy()[:] = oracle.kv_seq_to_head(x_seq.view(torch.int16).numpy(), P)
+
+
+def _fake_kv_head_to_seq(x_head, x_seq, stream=None):
+    P, b, m, H, d = x_seq.shape
+    assert tuple(x_head.shape) == (P, b, m * P, H // P if H >= P else 1, d) and x_head.dtype == x_seq.dtype
+    assert x_seq.is_contiguous() and x_head.is_contiguous()
+    out = oracle.kv_head_to_seq_reduce(x_head.double().numpy(), P, H)
+    x_seq.copy_(torch.from_numpy(out).to(x_seq.dtype))
+
+
+def _fake_transpose_runs(src, dst, A, B, run_bytes, stream=None):
+    assert src.numel() * src.element_size() == A * B * run_bytes == dst.numel() * dst.element_size()
+    _numpy_transpose(src, dst, A, B, run_bytes)
+
+
+@pytest.mark.parametrize("P,H_kv,b,m", [(4, 2, 1, 8), (8, 2, 2, 4), (16, 8, 1, 4), (4, 1, 1, 8)])
+def test_kernel_wrappers_hand_the_binding_valid_shapes(P, H_kv, b, m, monkeypatch):
+    """The module's default kernel wrappers, with the binding replaced by host
+    stand-ins that enforce its shape rules: the views the wrappers build for
+    the kv copy and sum kernels are the ones those calls accept, and the
+    results equal the oracle's."""
+    from ulysses_head_attention_b200 import distributed as udist
+    monkeypatch.setattr(udist, "ulysses_kv_seq_to_head", _fake_kv_seq_to_head)
+    monkeypatch.setattr(udist, "ulysses_kv_head_to_seq", _fake_kv_head_to_seq)
+    monkeypatch.setattr(udist, "ulysses_transpose_runs", _fake_transpose_runs)
+    _run(P, H_kv, b, m, 8, torch.device("cpu"), monkeypatch, {"fwd": {}, "bwd": {}})
