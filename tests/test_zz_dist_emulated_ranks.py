@@ -1,15 +1,18 @@
-"""The K/V all-to-alls of ulysses_head_attention_b200.distributed for fewer
-kv heads than ranks, with P ranks emulated by P host threads in one process.
+"""The all-to-alls of ulysses_head_attention_b200.distributed (seq_to_head /
+head_to_seq, and kv_seq_to_head / kv_head_to_seq for fewer kv heads than
+ranks), with P ranks emulated by P host threads in one process.
 
-Each thread runs the module's kv_seq_to_head / kv_head_to_seq for its rank;
+Each thread runs the module's call for its rank;
 the exchange stand-in publishes the rank's send buffer, waits for every rank
 on a host barrier (bounded), copies chunk r of every rank s into slot s of
 its receive buffer, and waits again.  No kernel waits on another: all
 waiting is on the host.  On the GPU the pack, copy, sum and unpack steps are
-the library's kernels, and the result must equal the one-GPU kv re-layouts
-(ulysses_kv_seq_to_head / ulysses_kv_head_to_seq) bit for bit, and the
-oracle.  The same harness runs on the CPU with numpy stand-ins for the
-kernels, which checks the harness itself where no GPU is present.
+the library's kernels, and the result must equal the one-GPU re-layouts
+(ulysses_seq_to_head, ulysses_kv_seq_to_head / ulysses_kv_head_to_seq) bit
+for bit, and the oracle.  The same harness runs on the CPU with numpy
+stand-ins for the kernels, or with the module's own kernel wrappers over a
+shape-checking stand-in of the binding, which checks the harness and the
+wrappers' views where no GPU is present.
 """
 import threading
 
@@ -151,3 +154,36 @@ def test_kernel_wrappers_hand_the_binding_valid_shapes(P, H_kv, b, m, monkeypatc
     monkeypatch.setattr(udist, "ulysses_kv_head_to_seq", _fake_kv_head_to_seq)
     monkeypatch.setattr(udist, "ulysses_transpose_runs", _fake_transpose_runs)
     _run(P, H_kv, b, m, 8, torch.device("cpu"), monkeypatch, {"fwd": {}, "bwd": {}})
+
+
+def _run_plain(P, H, b, m, d, device, monkeypatch, kernels):
+    """seq_to_head / head_to_seq of the module (H divisible by P), emulated ranks."""
+    from ulysses_head_attention_b200 import distributed as udist
+    monkeypatch.setattr(udist, "_group_size", lambda group: P)
+    rng = np.random.default_rng(P * 100 + H)
+    x = rng.integers(-2 ** 15, 2 ** 15, (P, b, m, H, d)).astype(np.int16)
+    xs = torch.from_numpy(x).view(torch.bfloat16).to(device)
+    heads = torch.stack(emulate_ranks(P, lambda r, ex: udist.seq_to_head(xs[r].contiguous(), exchange=ex,
+                                                                          **kernels)))
+    assert np.array_equal(heads.view(torch.int16).cpu().numpy(), oracle.seq_to_head(x, P))
+    back = torch.stack(emulate_ranks(P, lambda r, ex: udist.head_to_seq(heads[r].contiguous(), exchange=ex,
+                                                                         **kernels)))
+    assert torch.equal(back.view(torch.int16), xs.view(torch.int16))
+    return xs, heads
+
+
+@pytest.mark.parametrize("P,H,b,m", [(2, 4, 2, 4), (4, 8, 1, 8)])
+def test_plain_wrappers_hand_the_binding_valid_shapes(P, H, b, m, monkeypatch):
+    from ulysses_head_attention_b200 import distributed as udist
+    monkeypatch.setattr(udist, "ulysses_transpose_runs", _fake_transpose_runs)
+    _run_plain(P, H, b, m, 8, torch.device("cpu"), monkeypatch, {})
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("P,H,b,m", [(4, 32, 1, 256), (8, 8, 2, 64)])
+def test_plain_all_to_alls_on_gpu_equal_the_one_gpu_relayout(cuda_device, P, H, b, m, monkeypatch):
+    import ulysses_head_attention_b200 as uly
+    xs, heads = _run_plain(P, H, b, m, 128, cuda_device, monkeypatch, {})
+    one = torch.empty((P, b, m * P, H // P, 128), dtype=torch.bfloat16, device=cuda_device)
+    uly.ulysses_seq_to_head(xs, one)
+    assert torch.equal(heads.view(torch.int16), one.view(torch.int16))
