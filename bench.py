@@ -252,10 +252,10 @@ def run_ours(args, w):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)   # before the process group, so NCCL binds this rank's GPU
+    dev = torch.device("cuda", local)
     if world > 1:
         dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
     peaks = load_peaks()
 
     P, b, n, hq, hkv, d = w.P, w.b, w.n, w.h_q, w.h_kv, w.d
@@ -338,7 +338,7 @@ def run_ours(args, w):
 
     def barrier():
         if world > 1:
-            dist.barrier()
+            dist.barrier(device_ids=[local])
 
     # ---- device-timed region: K steps, inputs resident in HBM
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
