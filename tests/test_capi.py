@@ -51,12 +51,23 @@ INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 4
     ((0, F + 1 << 30, 1, 64, 32, 128, 4), INVALID),         # null input
     ((F + 8, F + 1 << 30, 1, 64, 32, 128, 4), INVALID),     # misaligned
     ((F, F + 1024, 1, 64, 32, 128, 4), INVALID),            # overlapping buffers
+    ((F, F + (1 << 30), 1, 0, 32, 128, 4), INVALID),        # empty sequence
+    ((F, F + (1 << 30), 0, 64, 32, 128, 4), INVALID),       # no batch rows
+    ((F, F + (1 << 30), 1, 64, 32, 0, 4), INVALID),         # empty head dimension
 ])
 def test_relayout_rejects(args, want):
     import ulysses_head_attention_b200 as uly
     src, dst, b, n, H, d, P = args
     for fn in (uly.lib.ulysses_seq_to_head, uly.lib.ulysses_head_to_seq):
         assert fn(src, dst, b, n, H, d, P, 0, None) == want
+
+
+@no_gpu
+def test_relayout_rejects_unknown_dtype():
+    import ulysses_head_attention_b200 as uly
+    for fn in (uly.lib.ulysses_seq_to_head, uly.lib.ulysses_head_to_seq, uly.lib.ulysses_kv_seq_to_head,
+               uly.lib.ulysses_kv_head_to_seq):
+        assert fn(F, F + (1 << 30), 1, 64, 32, 128, 4, 7, None) == INVALID
 
 
 def shape(b=1, n=1024, hq=32, hkv=8, d=128, P=4):
@@ -74,6 +85,10 @@ def shape(b=1, n=1024, hq=32, hkv=8, d=128, P=4):
     ({}, 4, INVALID),                        # rank out of range
     ({}, -2, INVALID),
     (dict(d=96), -1, UNSUPPORTED),           # head dim not implemented
+    (dict(n=0), -1, INVALID),                # empty sequence
+    (dict(b=0), -1, INVALID),                # no batch rows
+    (dict(hq=0), -1, INVALID),
+    (dict(n=1 << 31, P=4), -1, UNSUPPORTED),  # beyond the int32 TMA coordinates
 ])
 def test_attention_rejects_shapes(kw, rank, want):
     import ulysses_head_attention_b200 as uly
