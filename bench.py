@@ -35,25 +35,27 @@ sys.path.insert(0, ROOT)
 import synthetic  # noqa: E402
 
 METRIC = "causal attn TFLOP/s fwd & fwd+bwd (% bf16 peak); re-layout GB/s (% HBM)"
-DEFAULT_WORKLOAD = "llama8b_p4_n32k"
+DEFAULT_WORKLOAD = "roundtrip_p4_n128k"
 
 
-# DRAM traffic per launch of the dominant kernel, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum; the capture's command and
-# figures are in the profile named).  It applies only while the kernel's
-# sources hash to the value recorded with it; otherwise traffic is null.
+# DRAM traffic per launch of a kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum, --print-units base) of the
+# named workload.  It applies only while the kernel's sources hash to the
+# value recorded with it; otherwise traffic is null.
 KERNEL_SOURCES = {
     # kernel -> (file, first line of its source region or None for the whole file, ...)
     "attn_bwd_dkdv_kernel": (("ulysses_head_attention_b200/csrc/attn_bwd.cu", "namespace dkdv {", "}  // namespace dkdv"),
                              ("ulysses_head_attention_b200/csrc/sm100.cuh", None, None),
                              ("ulysses_head_attention_b200/csrc/common.cuh", None, None)),
+    "attn_bwd_dq_kernel": (("ulysses_head_attention_b200/csrc/attn_bwd.cu", "namespace dq {", "}  // namespace dq"),
+                           ("ulysses_head_attention_b200/csrc/sm100.cuh", None, None),
+                           ("ulysses_head_attention_b200/csrc/common.cuh", None, None)),
+    "attn_fwd_kernel": (("ulysses_head_attention_b200/csrc/attn_fwd.cu", "namespace fwd {", "}  // namespace fwd"),
+                        ("ulysses_head_attention_b200/csrc/sm100.cuh", None, None),
+                        ("ulysses_head_attention_b200/csrc/common.cuh", None, None)),
 }
-# llama8b_p4_n32k, one launch: ncu dram__bytes_read.sum 692503552 + dram__bytes_write.sum 244745216
-# bytes (--print-units base); see profiles/attn_bwd_dkdv_kernel.md
-TRAFFIC = {
-    "attn_bwd_dkdv_kernel": {"workload": "llama8b_p4_n32k", "bytes_per_launch": 692503552 + 244745216,
-                             "sources_sha256": "512677325366df9ff6cfb9268a1e45f8125519207cc557136848e3c3049a48c8"},
-}
+# kernel -> {"workload", "bytes_per_launch", "sources_sha256"}
+TRAFFIC = {}
 
 
 def sources_sha256(kernel: str) -> str:
@@ -118,8 +120,9 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples (every 50 ms) of SM clock and clock-event reasons; only
-    samples read inside the marked window (the timed region) are kept."""
+    """nvidia-smi samples (every 50 ms) of SM clock and clock-event reasons,
+    kept with their host time stamps; summary(t0, t1) reports the samples
+    read inside one timed window."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.sw_power_cap,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.active")
@@ -132,7 +135,6 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.lines = []
-        self.window = (0.0, float("inf"))
 
     def start(self):
         try:
@@ -148,12 +150,9 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append((time.time(), line.strip()))
 
-    def mark(self, t0: float, t1: float):
-        self.window = (t0, t1)
-
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return
         time.sleep(0.1)   # let the last in-window line arrive
         self.proc.terminate()
         try:
@@ -161,10 +160,13 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm, smax, reasons, masks = [], None, set(), set()
         names = ("sw_power_cap", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
-        t0, t1 = self.window
-        for t, ln in self.lines:
+        for t, ln in list(self.lines):
             if not (t0 <= t <= t1 + 0.06):
                 continue
             parts = [x.strip() for x in ln.split(",")]
@@ -244,6 +246,176 @@ def run_reference(args, w):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+# Kernel launches of one step: s2h q, k, v (3); forward: segments + attention
+# (2); h2s O (1); s2h dO (1); backward: segments, largest magnitudes, fp16
+# copies, row statistics, dK/dV, dQ (6); h2s dQ, dK, dV (3).
+LAUNCHES_FWD_BWD = 3 + 2 + 1 + 1 + 6 + 3
+# tcgen05 dense bf16 rate per SM and clock (M = 128, N = 256, K = 16 in 128 cycles)
+TENSOR_FLOP_PER_CLK_SM = 8192
+NUM_SMS = 148
+
+
+class Layer:
+    """Device buffers and the step of one workload: seq-sharded inputs in
+    HBM, the re-layouts, the attention calls, fp32 outputs."""
+
+    def __init__(self, w, x, dev, uly, pin=True):
+        import torch
+        self.w, self.uly, self.dev = w, uly, dev
+        P, b, n, hq, hkv, d = w.P, w.b, w.n, w.h_q, w.h_kv, w.d
+        m = n // P
+        self.pairs = pairs_of(x["lengths"])
+        self.fwd_flops = 4 * d * hq * self.pairs
+        self.bwd_flops = 8 * d * hq * self.pairs if w.backward else 0
+        bf, f32 = torch.bfloat16, torch.float32
+
+        def host(bits):   # pinned when the end-to-end measurement copies from it every step
+            t = torch.from_numpy(bits.reshape(P, b, m, bits.shape[2], d).view(np.int16)).view(bf)
+            return t.pin_memory() if pin else t
+
+        keys = ("q", "k", "v", "do") if w.backward else ("q", "k", "v")
+        self.host = {k: host(x[k]) for k in keys}
+        self.host_pos = torch.from_numpy(x["position_ids"])
+        if pin:
+            self.host_pos = self.host_pos.pin_memory()
+        self.seq = {k: self.host[k].to(dev) for k in keys}
+        self.pos = self.host_pos.to(dev)
+        hkv_r = hkv // P if hkv >= P else 1   # kv heads per rank (one replicated head when H_kv < P)
+        self.head = {"q": torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev),
+                     "k": torch.empty((P, b, n, hkv_r, d), dtype=bf, device=dev),
+                     "v": torch.empty((P, b, n, hkv_r, d), dtype=bf, device=dev)}
+        if w.backward:
+            self.head["do"] = torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev)
+        self.o_head = torch.empty((P, b, n, hq // P, d), dtype=f32, device=dev)
+        self.lse = torch.empty((P, b, hq // P, n), dtype=f32, device=dev)
+        self.o_seq = torch.empty((P, b, m, hq, d), dtype=f32, device=dev)
+        self.shape = uly.make_shape(b, n, hq, hkv, d, P)
+        self.ws_f = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(self.shape), dev)
+        nbytes = lambda t: t.numel() * t.element_size()   # noqa: E731
+        # every re-layout reads its source once and writes its destination once
+        self.relayout_bytes = sum(nbytes(self.seq[k]) + nbytes(self.head[k]) for k in keys)
+        self.relayout_bytes += nbytes(self.o_head) + nbytes(self.o_seq)
+        self.l2_note = f"inputs larger than L2 (q {nbytes(self.seq['q']) >> 20} MiB per step)"
+        if w.backward:
+            self.g_head = {"q": torch.empty_like(self.o_head),
+                           "k": torch.empty((P, b, n, hkv_r, d), dtype=f32, device=dev),
+                           "v": torch.empty((P, b, n, hkv_r, d), dtype=f32, device=dev)}
+            self.g_seq = {"q": torch.empty((P, b, m, hq, d), dtype=f32, device=dev),
+                          "k": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev),
+                          "v": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev)}
+            self.ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(self.shape, uly.ULY_F32), dev)
+            self.relayout_bytes += sum(nbytes(self.g_head[k]) + nbytes(self.g_seq[k]) for k in self.g_seq)
+        # forward-only workloads run s2h(q, k, v), the forward (rank by rank when
+        # asked) and h2s(O)
+        self.launches = LAUNCHES_FWD_BWD if w.backward else 3 + 2 * (P if w.rank_by_rank else 1) + 1
+
+    def step(self, ev=None, kev=None):
+        """One pass of the path.  ev: 6 events around its stages; kev: 5 events
+        around the backward's kernels."""
+        uly, h, s = self.uly, self.head, self.seq
+        mark = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        mark(0)
+        uly.ulysses_seq_to_head(s["q"], h["q"])
+        for k in ("k", "v"):   # plain re-layout, or one copied kv head per rank when H_kv < P
+            uly.ulysses_kv_seq_to_head(s[k], h[k])
+        mark(1)
+        if self.w.rank_by_rank:   # each virtual rank's head slice in turn
+            for r in range(self.w.P):
+                uly.ulysses_attn_fwd(h["q"], h["k"], h["v"], self.pos, self.o_head, self.lse, self.ws_f, rank=r)
+        else:
+            uly.ulysses_attn_fwd(h["q"], h["k"], h["v"], self.pos, self.o_head, self.lse, self.ws_f)
+        mark(2)
+        uly.ulysses_head_to_seq(self.o_head, self.o_seq)
+        if not self.w.backward:
+            mark(3), mark(4), mark(5)
+            return
+        uly.ulysses_seq_to_head(s["do"], h["do"])
+        mark(3)
+        g = self.g_head
+        if kev is not None:   # the same call, with events around its kernels
+            uly.ulysses_attn_bwd_timed(h["q"], h["k"], h["v"], self.o_head, self.lse, h["do"], self.pos,
+                                       g["q"], g["k"], g["v"], self.ws_b, kev)
+        else:
+            uly.ulysses_attn_bwd(h["q"], h["k"], h["v"], self.o_head, self.lse, h["do"], self.pos,
+                                 g["q"], g["k"], g["v"], self.ws_b)
+        mark(4)
+        uly.ulysses_head_to_seq(g["q"], self.g_seq["q"])
+        for k in ("k", "v"):   # the copies' gradients are summed when H_kv < P
+            uly.ulysses_kv_head_to_seq(g[k], self.g_seq[k])
+        mark(5)
+
+    def check_status(self, where: str):
+        for ws in ((self.ws_f, self.ws_b) if self.w.backward else (self.ws_f,)):
+            if self.uly.ulysses_workspace_status(ws) != 0:
+                raise RuntimeError(f"a kernel reported a pipeline timeout {where}")
+
+
+def time_layer(layer, steps: int, warmup: int, clocks, barrier=lambda: None):
+    """Warm-up, then `steps` steps bracketed by a barrier and a synchronize.
+    Returns the device time of the region, per-stage and per-kernel means and
+    the clock record of the window."""
+    import torch
+    for _ in range(warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    layer.check_status("during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
+    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        layer.step(evs[i], kevs[i] if layer.w.backward else None)
+    end.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    layer.check_status("in the timed region")
+    names = ("s2h_qkv", "attn_fwd", "h2s_o_s2h_do", "attn_bwd", "h2s_grads")
+    st = {k: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, k in enumerate(names)}
+    km = {}
+    if layer.w.backward:
+        km = {"bwd_prep (segments, magnitudes, fp16 copies, statistics)":
+              statistics.mean(e[0].elapsed_time(e[2]) for e in kevs),
+              "attn_bwd_dkdv_kernel": statistics.mean(e[2].elapsed_time(e[3]) for e in kevs),
+              "attn_bwd_dq_kernel": statistics.mean(e[3].elapsed_time(e[4]) for e in kevs)}
+    return {"ms_total": start.elapsed_time(end), "stage_ms": st, "kernel_ms": km,
+            "clocks": clocks.summary(t0, t1), "seconds": t1 - t0}
+
+
+def clock_peak_tflops(sm_mhz):
+    """The tensor pipe's dense bf16 rate at the sampled SM clock."""
+    return None if not sm_mhz else TENSOR_FLOP_PER_CLK_SM * NUM_SMS * sm_mhz * 1e6 / 1e12
+
+
+def layer_figures(layer, t, peaks):
+    """Absolute figures and fractions of one timed workload."""
+    st = t["stage_ms"]
+    fwd_tf = layer.fwd_flops / (st["attn_fwd"] * 1e-3) / 1e12
+    # the burst peak for short timed regions, the sustained one for long ones
+    basis = "bf16_tflops_sustained" if t["seconds"] >= 2.0 else "bf16_tflops"
+    peak = peaks[basis]
+    cpk = clock_peak_tflops(t["clocks"].get("sm_mhz"))
+    relayout_ms = st["s2h_qkv"] + st["h2s_o_s2h_do"] + st["h2s_grads"]
+    out = {"pairs": layer.pairs, "ms_per_step": t["ms_total"] / max(1, t["steps"]), "steps": t["steps"],
+           "stage_ms": st, "peak_basis": f"{basis} ({peaks['source']})",
+           "attn_fwd_tflops": fwd_tf, "attn_fwd_frac": fwd_tf / peak,
+           "attn_fwd_frac_of_clock_peak": fwd_tf / cpk if cpk else None,
+           "relayout_gbs": layer.relayout_bytes / (relayout_ms * 1e-3) / 1e9,
+           "relayout_bytes": layer.relayout_bytes, "clocks": t["clocks"]}
+    out["relayout_frac"] = out["relayout_gbs"] / peaks["hbm_gbs"]
+    if layer.w.backward:
+        bwd_tf = layer.bwd_flops / (st["attn_bwd"] * 1e-3) / 1e12
+        fb_tf = (layer.fwd_flops + layer.bwd_flops) / ((st["attn_fwd"] + st["attn_bwd"]) * 1e-3) / 1e12
+        out.update({"attn_bwd_tflops": bwd_tf, "attn_bwd_frac": bwd_tf / peak,
+                    "attn_fwd_bwd_tflops": fb_tf, "attn_fwd_bwd_frac": fb_tf / peak,
+                    "attn_fwd_bwd_frac_of_clock_peak": fb_tf / cpk if cpk else None,
+                    "bwd_kernel_ms": t["kernel_ms"]})
+    return out
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -258,269 +430,73 @@ def run_ours(args, w):
         dist.init_process_group("nccl", init_method="env://", timeout=__import__("datetime").timedelta(seconds=120))
     peaks = load_peaks()
 
-    P, b, n, hq, hkv, d = w.P, w.b, w.n, w.h_q, w.h_kv, w.d
-    m = n // P
-    x = synthetic.make_inputs(w)
-    pairs = pairs_of(x["lengths"])
-    fwd_flops = 4 * d * hq * pairs
-    bwd_flops = 8 * d * hq * pairs
-
-    def pinned(bits):
-        t = torch.from_numpy(bits.reshape(P, b, m, bits.shape[2], d).view(np.int16)).view(torch.bfloat16)
-        return t.pin_memory()
-
-    host = {k: pinned(x[k]) for k in ("q", "k", "v", "do")}
-    host_pos = torch.from_numpy(x["position_ids"]).pin_memory()
-    seq = {k: host[k].to(dev) for k in host}
-    pos = host_pos.to(dev)
-    bf, f32 = torch.bfloat16, torch.float32
-    hkv_r = hkv // P if hkv >= P else 1   # kv heads per rank (one replicated head when H_kv < P)
-    head = {"q": torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev),
-            "k": torch.empty((P, b, n, hkv_r, d), dtype=bf, device=dev),
-            "v": torch.empty((P, b, n, hkv_r, d), dtype=bf, device=dev),
-            "do": torch.empty((P, b, n, hq // P, d), dtype=bf, device=dev)}
-    o_head = torch.empty((P, b, n, hq // P, d), dtype=f32, device=dev)
-    lse = torch.empty((P, b, hq // P, n), dtype=f32, device=dev)
-    o_seq = torch.empty((P, b, m, hq, d), dtype=f32, device=dev)
-    g_head = {"q": torch.empty_like(o_head), "k": torch.empty((P, b, n, hkv_r, d), dtype=f32, device=dev),
-              "v": torch.empty((P, b, n, hkv_r, d), dtype=f32, device=dev)}
-    g_seq = {"q": torch.empty((P, b, m, hq, d), dtype=f32, device=dev),
-             "k": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev),
-             "v": torch.empty((P, b, m, hkv, d), dtype=f32, device=dev)}
-    shape = uly.make_shape(b, n, hq, hkv, d, P)
-    ws_f = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(shape), dev)
-    ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, uly.ULY_F32), dev)
-    stream = torch.cuda.current_stream()
-    # s2h x3; fwd: segments + attn_fwd; h2s O; s2h dO; bwd: segments + bwd_pre + bwd_dkdv + bwd_dq; h2s x3
-    # (the event records inside the timed backward are not kernels)
-    launches_per_step = 3 + 2 + 1 + 1 + 4 + 3
-
-    # every re-layout reads its source once and writes its destination once
-    nbytes = lambda t: t.numel() * t.element_size()   # noqa: E731
-    relayout_bytes = sum(nbytes(seq[k]) + nbytes(head[k]) for k in ("q", "k", "v", "do"))
-    relayout_bytes += nbytes(o_head) + nbytes(o_seq) + sum(nbytes(g_head[k]) + nbytes(g_seq[k]) for k in g_seq)
-
-    def step(ev=None, kev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        uly.ulysses_seq_to_head(seq["q"], head["q"])
-        for k in ("k", "v"):   # plain re-layout, or one copied kv head per rank when H_kv < P
-            uly.ulysses_kv_seq_to_head(seq[k], head[k])
-        if ev is not None:
-            ev[1].record(stream)
-        uly.ulysses_attn_fwd(head["q"], head["k"], head["v"], pos, o_head, lse, ws_f)
-        if ev is not None:
-            ev[2].record(stream)
-        uly.ulysses_head_to_seq(o_head, o_seq)
-        uly.ulysses_seq_to_head(seq["do"], head["do"])
-        if ev is not None:
-            ev[3].record(stream)
-        if kev is not None:   # the same call, with events around its four kernels
-            uly.ulysses_attn_bwd_timed(head["q"], head["k"], head["v"], o_head, lse, head["do"], pos,
-                                       g_head["q"], g_head["k"], g_head["v"], ws_b, kev)
-        else:
-            uly.ulysses_attn_bwd(head["q"], head["k"], head["v"], o_head, lse, head["do"], pos,
-                                 g_head["q"], g_head["k"], g_head["v"], ws_b)
-        if ev is not None:
-            ev[4].record(stream)
-        uly.ulysses_head_to_seq(g_head["q"], g_seq["q"])
-        for k in ("k", "v"):   # the copies' gradients are summed when H_kv < P
-            uly.ulysses_kv_head_to_seq(g_head[k], g_seq[k])
-        if ev is not None:
-            ev[5].record(stream)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    for ws in (ws_f, ws_b):
-        if uly.ulysses_workspace_status(ws) != 0:
-            raise RuntimeError("a kernel reported a pipeline timeout during warm-up")
-
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    # ---- device-timed region: K steps, inputs resident in HBM
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    t_region0 = time.time()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(args.steps):
-        step(evs[i], kevs[i])
-    end.record(stream)
-    torch.cuda.synchronize()
-    clocks.mark(t_region0, time.time())
-    barrier()
-    clk = clocks.stop()
-    ms_total = max_over_ranks(start.elapsed_time(end), world, dev)
-    ms_step = ms_total / args.steps
-    stage = {"s2h_qkv": [], "attn_fwd": [], "h2s_o_s2h_do": [], "attn_bwd": [], "h2s_grads": []}
-    for e in evs:
-        for k, (a, bnd) in zip(stage, ((0, 1), (1, 2), (2, 3), (3, 4), (4, 5))):
-            stage[k].append(e[a].elapsed_time(e[bnd]))
-    st_ms = {k: statistics.mean(v) for k, v in stage.items()}
-    # per-kernel device time inside the backward call (events on the launching stream)
-    k_ms = {"attn_bwd_dkdv_kernel": statistics.mean(e[2].elapsed_time(e[3]) for e in kevs),
-            "attn_bwd_dq_kernel": statistics.mean(e[3].elapsed_time(e[4]) for e in kevs),
-            "bwd_pre_kernel": statistics.mean(e[1].elapsed_time(e[2]) for e in kevs)}
-    # algorithmic flops per launch: dK/dV runs S, dP, dV, dK (4 products of 2*d flops
-    # per visible pair); dQ runs S, dP, dQ (3)
-    k_flops = {"attn_bwd_dkdv_kernel": 8 * d * hq * pairs, "attn_bwd_dq_kernel": 6 * d * hq * pairs}
-    dom = max(k_flops, key=lambda kname: k_ms[kname])
-    dom_tf = k_flops[dom] / (k_ms[dom] * 1e-3) / 1e12
-    for ws in (ws_f, ws_b):
-        if uly.ulysses_workspace_status(ws) != 0:
-            raise RuntimeError("a kernel reported a pipeline timeout in the timed region")
 
-    value = whole_job_tflops(world, fwd_flops + bwd_flops, ms_step)
-    fwd_tf = fwd_flops / (st_ms["attn_fwd"] * 1e-3) / 1e12
-    bwd_tf = bwd_flops / (st_ms["attn_bwd"] * 1e-3) / 1e12
-    relayout_ms = st_ms["s2h_qkv"] + st_ms["h2s_o_s2h_do"] + st_ms["h2s_grads"]
-    relayout_gbs = relayout_bytes / (relayout_ms * 1e-3) / 1e9
-    peak_t = peaks["bf16_tflops_sustained"]
+    x = synthetic.make_inputs(w)
+    layer = Layer(w, x, dev, uly)
+    warm = max(args.warmup, 3)
+    t = time_layer(layer, args.steps, warm, clocks, barrier)
+    t["steps"] = args.steps
+    ms_step = max_over_ranks(t["ms_total"], world, dev) / args.steps
+    fig = layer_figures(layer, t, peaks)
+    value = whole_job_tflops(world, layer.fwd_flops + layer.bwd_flops, ms_step)
+    clk = t["clocks"]
 
-    # ---- end to end: pinned host inputs in, all outputs back to pinned host
-    h_out = {"o": torch.empty(o_seq.shape, dtype=f32, pin_memory=True)}
-    for k in g_seq:
-        h_out[k] = torch.empty(g_seq[k].shape, dtype=f32, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_pos.numel() * 8
-    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    # ---- the dominant kernel's roofline: its algorithmic flops per launch (the
+    # method's products it completes; recomputed S and dP are not counted) over
+    # its event-timed duration
+    if w.backward:
+        d, hq, pairs = w.d, w.h_q, layer.pairs
+        k_ms = {"attn_fwd_kernel": t["stage_ms"]["attn_fwd"],
+                "attn_bwd_dkdv_kernel": t["kernel_ms"]["attn_bwd_dkdv_kernel"],
+                "attn_bwd_dq_kernel": t["kernel_ms"]["attn_bwd_dq_kernel"]}
+        # forward: S and PV; dK/dV kernel: dP, dV, dK; dQ kernel: dQ
+        k_flops = {"attn_fwd_kernel": 4 * d * hq * pairs, "attn_bwd_dkdv_kernel": 6 * d * hq * pairs,
+                   "attn_bwd_dq_kernel": 2 * d * hq * pairs}
+        dom = max(k_ms, key=lambda kname: k_ms[kname])
+        dom_tf = k_flops[dom] / (k_ms[dom] * 1e-3) / 1e12
+        basis = "bf16_tflops_sustained" if t["seconds"] >= 2.0 else "bf16_tflops"
+        cpk = clock_peak_tflops(clk.get("sm_mhz"))
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peaks[basis], "unit": "TFLOP/s",
+                    "frac": dom_tf / peaks[basis], "peak_kind": f"{basis} ({peaks['source']})",
+                    "frac_of_clock_peak": dom_tf / cpk if cpk else None,
+                    "flops_per_launch": k_flops[dom], "ms_per_launch": k_ms[dom],
+                    "kernel_tflops": {kn: k_flops[kn] / (k_ms[kn] * 1e-3) / 1e12 for kn in k_ms},
+                    "traffic": recorded_traffic(dom, w.name)}
+    else:
+        roofline = None
 
-    def e2e_step():
-        for k in host:
-            seq[k].copy_(host[k], non_blocking=True)
-        pos.copy_(host_pos, non_blocking=True)
-        step()
-        h_out["o"].copy_(o_seq, non_blocking=True)
-        for k in g_seq:
-            h_out[k].copy_(g_seq[k], non_blocking=True)
+    # ---- end to end: pinned host inputs in, all outputs back to pinned host,
+    # copies on their own streams so they overlap the attention kernels
+    e2e = measure_e2e(layer, args.steps, barrier, world, dev) if w.backward else None
 
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e2.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, dev) / args.steps
-    e2e_value = whole_job_tflops(world, fwd_flops + bwd_flops, e2e_ms)
-
-    # ---- ring attention over R key blocks (forward + LSE merge, then the
-    # blocks' backward from the merged O / LSE), timed on its own
+    # ---- the other workloads, each timed the same way in this run
     extras = {}
-
-    def measure_ring():
-        R = 4
-        cuts = [n * i // R for i in range(R + 1)]
-        o_parts = torch.empty((R,) + tuple(o_head.shape), dtype=f32, device=dev)
-        l_parts = torch.empty((R,) + tuple(lse.shape), dtype=f32, device=dev)
-        o_ring, l_ring = torch.empty_like(o_head), torch.empty_like(lse)
-        g_ring = {k: torch.empty_like(g_head[k]) for k in g_head}
-
-        def ring_fwd():
-            for i in range(R):
-                uly.ulysses_attn_fwd_kv_range(head["q"], head["k"], head["v"], pos, o_parts[i], l_parts[i], ws_f,
-                                              cuts[i], cuts[i + 1])
-            uly.ulysses_attn_lse_merge(o_parts, l_parts, o_ring, l_ring, hkv)
-
-        def ring_bwd():
-            for i in range(R):
-                uly.ulysses_attn_bwd_kv_range(head["q"], head["k"], head["v"], o_ring, l_ring, head["do"], pos,
-                                              g_ring["q"], g_ring["k"], g_ring["v"], ws_b, cuts[i], cuts[i + 1])
-
-        ring_fwd()
-        ring_bwd()
-        torch.cuda.synchronize()
-        rf = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        reps = 3
-        rf[0].record(stream)
-        for _ in range(reps):
-            ring_fwd()
-        rf[1].record(stream)
-        for _ in range(reps):
-            ring_bwd()
-        rf[2].record(stream)
-        torch.cuda.synchronize()
-        for ws in (ws_f, ws_b):
-            if uly.ulysses_workspace_status(ws) != 0:
-                raise RuntimeError("a kernel reported a pipeline timeout in the ring measurement")
-        ring_fwd_ms = rf[0].elapsed_time(rf[1]) / reps
-        ring_bwd_ms = rf[1].elapsed_time(rf[2]) / reps
-        ring_stat = {"blocks": R, "fwd_ms": ring_fwd_ms, "fwd_tflops": fwd_flops / (ring_fwd_ms * 1e-3) / 1e12,
-                     "bwd_ms_per_block_pass": ring_bwd_ms, "bwd_tflops": bwd_flops / (ring_bwd_ms * 1e-3) / 1e12,
-                     "launches": {"fwd": R * 2 + 1, "bwd": R * 4},
-                     "note": "keys cut into R equal blocks; forward = R key-range forwards + one LSE merge; "
-                             "backward = R key-range backwards from the merged O and LSE (one block's dQ share each)"}
-        extras["ring_attention"] = ring_stat
-
-    # ---- weighted SP loss aggregation (the custom training loop's per-rank loss
-    # weighting), timed on its own: it needs a model's per-rank losses, which
-    # this path does not produce, so it is not part of the step
-    def measure_loss():
-        lab = synthetic.sft_shift_labels(w.wid, x["lengths"])
-        lab_sh = torch.from_numpy(np.ascontiguousarray(lab.reshape(b, P, m).transpose(1, 0, 2))).to(dev)
-        l_in = torch.from_numpy(synthetic.rank_losses(w.wid, P)).to(dev)
-        l_out, l_good, l_dl = (torch.empty(1, device=dev), torch.empty(P, dtype=torch.int64, device=dev),
-                               torch.empty(P, device=dev))
-        for _ in range(5):
-            uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
-        torch.cuda.synchronize()
-        s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 50
-        s3.record(stream)
-        for _ in range(reps):
-            uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
-        e3.record(stream)
-        torch.cuda.synchronize()
-        loss_us = s3.elapsed_time(e3) * 1e3 / reps
-        loss_bytes = lab_sh.numel() * 8 + 3 * P * 8 + 4
-        loss_stat = {"us_per_call": loss_us, "bytes_per_call": loss_bytes,
-                     "gbs": loss_bytes / (loss_us * 1e-6) / 1e9, "launches_per_call": 2,
-                     "labels": "packed SFT: per sample a U[0.1, 0.6) prompt fraction and the last position are -100"}
-        extras["sp_loss_aggregate"] = loss_stat
-
     if not args.no_extras:
-        measure_ring()
-        measure_loss()
+        extras["configs"] = measure_configs(args, w, dev, uly, peaks, clocks)
+        extras.update(measure_ring(layer, dev))
+        extras["sp_loss_aggregate"] = measure_loss(layer, x, dev)
+    clocks.stop()
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "P": P, "b": b, "n": n, "h_q": hq, "h_kv": hkv, "d": d,
-                   "samples": sum(len(r) for r in x["lengths"]), "pairs": pairs,
-                   "outputs": "fp32",
-                   "l2": f"inputs larger than L2 (q {nbytes(seq['q']) >> 20} MiB, dO {nbytes(seq['do']) >> 20} MiB per step)",
-                   "parallelism": f"{world} independent replica(s), one per GPU"},
-        "detail": {
-            "attn_fwd_tflops": fwd_tf, "attn_fwd_frac": fwd_tf / peak_t,
-            "attn_bwd_tflops": bwd_tf, "attn_bwd_frac": bwd_tf / peak_t,
-            "attn_fwd_bwd_tflops": (fwd_flops + bwd_flops) / ((st_ms["attn_fwd"] + st_ms["attn_bwd"]) * 1e-3) / 1e12,
-            "relayout_gbs": relayout_gbs, "relayout_frac": relayout_gbs / peaks["hbm_gbs"],
-            "stage_ms": st_ms, "bwd_kernel_ms": k_ms,
-            "bwd_kernel_tflops": {kname: k_flops[kname] / (k_ms[kname] * 1e-3) / 1e12 for kname in k_flops},
-            "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
-            "bwd_flops_with_recompute_convention": 10 * d * hq * pairs,
-            "peaks": peaks,
-            **extras,
-        },
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": dom_tf / peak_t, "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
-                     "flops_per_launch": k_flops[dom], "ms_per_launch": k_ms[dom],
-                     "traffic": recorded_traffic(dom, w.name)},
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms},
-        "gpu_launches": launches_per_step * args.steps,
+        "config": {"workload": w.name, "P": w.P, "b": w.b, "n": w.n, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
+                   "samples": sum(len(r) for r in x["lengths"]), "pairs": layer.pairs, "outputs": "fp32",
+                   "l2": layer.l2_note, "parallelism": f"{world} independent replica(s), one per GPU"},
+        "detail": {**fig, "fwd_flops": layer.fwd_flops, "bwd_flops": layer.bwd_flops,
+                   "bwd_flops_with_recompute_convention": 10 * w.d * w.h_q * layer.pairs,
+                   "peaks": peaks, **extras},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": layer.launches * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -540,18 +516,209 @@ def run_ours(args, w):
     return 0
 
 
+def measure_e2e(layer, steps, barrier, world, dev):
+    """The same metric with every step's inputs copied in from pinned host
+    memory and its outputs (O, dQ, dK, dV) copied back, inside the timed
+    region.  Host-to-device copies run on one side stream and device-to-host
+    copies on another, each ordered against the compute stream by events, so
+    that step i+1's inputs arrive and step i's outputs leave while attention
+    runs."""
+    import torch
+    f32 = torch.float32
+    main = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    h_out = {"o": torch.empty(layer.o_seq.shape, dtype=f32, pin_memory=True)}
+    for k in layer.g_seq:
+        h_out[k] = torch.empty(layer.g_seq[k].shape, dtype=f32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in layer.host.values()) + layer.host_pos.numel() * 8
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    uly, h, s, g = layer.uly, layer.head, layer.seq, layer.g_head
+    # position_ids are read by the backward too, which still runs when the
+    # next step's inputs arrive: two buffers, used by alternate steps
+    pos = [layer.pos, torch.empty_like(layer.pos)]
+    ev = lambda: torch.cuda.Event()   # noqa: E731
+
+    def run(n_steps):
+        # state carried between steps: the events the next copies wait on
+        inputs_free, o_free, g_free = ev(), ev(), ev()
+        inputs_free.record(main), o_free.record(main), g_free.record(main)
+        for i in range(n_steps):
+            p_i = pos[i % 2]   # last read by step i - 2, whose backward finished before inputs_free
+            up.wait_event(inputs_free)
+            with torch.cuda.stream(up):
+                for k in ("q", "k", "v"):
+                    s[k].copy_(layer.host[k], non_blocking=True)
+                p_i.copy_(layer.host_pos, non_blocking=True)
+                qkv_in = ev(); qkv_in.record(up)
+                s["do"].copy_(layer.host["do"], non_blocking=True)
+                do_in = ev(); do_in.record(up)
+            main.wait_event(qkv_in)
+            uly.ulysses_seq_to_head(s["q"], h["q"])
+            for k in ("k", "v"):
+                uly.ulysses_kv_seq_to_head(s[k], h[k])
+            uly.ulysses_attn_fwd(h["q"], h["k"], h["v"], p_i, layer.o_head, layer.lse, layer.ws_f)
+            main.wait_event(o_free)
+            uly.ulysses_head_to_seq(layer.o_head, layer.o_seq)
+            o_ready = ev(); o_ready.record(main)
+            main.wait_event(do_in)
+            uly.ulysses_seq_to_head(s["do"], h["do"])
+            inputs_free = ev(); inputs_free.record(main)   # q, k, v, dO consumed: next inputs may land
+            down.wait_event(o_ready)
+            with torch.cuda.stream(down):
+                h_out["o"].copy_(layer.o_seq, non_blocking=True)
+                o_free = ev(); o_free.record(down)
+            uly.ulysses_attn_bwd(h["q"], h["k"], h["v"], layer.o_head, layer.lse, h["do"], p_i,
+                                 g["q"], g["k"], g["v"], layer.ws_b)
+            main.wait_event(g_free)
+            uly.ulysses_head_to_seq(g["q"], layer.g_seq["q"])
+            for k in ("k", "v"):
+                uly.ulysses_kv_head_to_seq(g[k], layer.g_seq[k])
+            g_ready = ev(); g_ready.record(main)
+            down.wait_event(g_ready)
+            with torch.cuda.stream(down):
+                for k in layer.g_seq:
+                    h_out[k].copy_(layer.g_seq[k], non_blocking=True)
+                g_free = ev(); g_free.record(down)
+        main.wait_event(o_free)
+        main.wait_event(g_free)
+
+    run(1)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(main)
+    run(steps)
+    e2.record(main)
+    torch.cuda.synchronize()
+    barrier()
+    layer.check_status("in the end-to-end region")
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, dev) / steps
+    return {"value": whole_job_tflops(world, layer.fwd_flops + layer.bwd_flops, e2e_ms), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "copies": "pinned host; H2D and D2H on two side streams ordered by events, overlapping attention"}
+
+
+# the other workloads timed in the same run: (name, steps, warm-up)
+OTHER_CONFIGS = (("tiny_p2_n256", 20, 3), ("llama8b_p4_n32k", 5, 3), ("packed_sft_p8_n64k", 5, 3),
+                 ("long_p8_n512k", 2, 1))
+
+
+def measure_configs(args, w_main, dev, uly, peaks, clocks):
+    import torch
+    res = {}
+    for name, steps, warm in OTHER_CONFIGS:
+        if name == w_main.name:
+            continue
+        wk = synthetic.WORKLOADS[name]
+        lay = Layer(wk, synthetic.make_inputs(wk), dev, uly, pin=False)
+        t = time_layer(lay, steps, warm, clocks)
+        t["steps"] = steps
+        res[name] = layer_figures(lay, t, peaks)
+        del lay
+        torch.cuda.empty_cache()
+    return res
+
+
+def measure_ring(layer, dev):
+    """Ring attention over R key blocks (forward + LSE merge, then the blocks'
+    backward from the merged O / LSE), timed on its own."""
+    import torch
+    if not layer.w.backward:
+        return {}
+    uly, h, w = layer.uly, layer.head, layer.w
+    R, n, f32 = 4, w.n, torch.float32
+    cuts = [n * i // R for i in range(R + 1)]
+    o_parts = torch.empty((R,) + tuple(layer.o_head.shape), dtype=f32, device=dev)
+    l_parts = torch.empty((R,) + tuple(layer.lse.shape), dtype=f32, device=dev)
+    o_ring, l_ring = torch.empty_like(layer.o_head), torch.empty_like(layer.lse)
+    g_ring = {k: torch.empty_like(layer.g_head[k]) for k in layer.g_head}
+
+    def ring_fwd():
+        for i in range(R):
+            uly.ulysses_attn_fwd_kv_range(h["q"], h["k"], h["v"], layer.pos, o_parts[i], l_parts[i], layer.ws_f,
+                                          cuts[i], cuts[i + 1])
+        uly.ulysses_attn_lse_merge(o_parts, l_parts, o_ring, l_ring, w.h_kv)
+
+    def ring_bwd():
+        for i in range(R):
+            uly.ulysses_attn_bwd_kv_range(h["q"], h["k"], h["v"], o_ring, l_ring, h["do"], layer.pos,
+                                          g_ring["q"], g_ring["k"], g_ring["v"], layer.ws_b, cuts[i], cuts[i + 1])
+
+    ring_fwd()
+    ring_bwd()
+    torch.cuda.synchronize()
+    rf = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    reps = 2
+    rf[0].record()
+    for _ in range(reps):
+        ring_fwd()
+    rf[1].record()
+    for _ in range(reps):
+        ring_bwd()
+    rf[2].record()
+    torch.cuda.synchronize()
+    layer.check_status("in the ring measurement")
+    fwd_ms = rf[0].elapsed_time(rf[1]) / reps
+    bwd_ms = rf[1].elapsed_time(rf[2]) / reps
+    del o_parts, l_parts, o_ring, l_ring, g_ring
+    torch.cuda.empty_cache()
+    return {"ring_attention": {
+        "blocks": R, "fwd_ms": fwd_ms, "fwd_tflops": layer.fwd_flops / (fwd_ms * 1e-3) / 1e12,
+        "bwd_ms_per_block_pass": bwd_ms, "bwd_tflops": layer.bwd_flops / (bwd_ms * 1e-3) / 1e12,
+        "launches": {"fwd": R * 2 + 1, "bwd": R * 6},
+        "note": "keys cut into R equal blocks; forward = R key-range forwards + one LSE merge; "
+                "backward = R key-range backwards from the merged O and LSE (one block's dQ share each)"}}
+
+
+def measure_loss(layer, x, dev):
+    """Weighted SP loss aggregation (the custom training loop's per-rank loss
+    weighting), timed on its own: it needs a model's per-rank losses, which
+    this path does not produce, so it is not part of the step."""
+    import torch
+    w, uly = layer.w, layer.uly
+    P, b, m = w.P, w.b, w.n // w.P
+    lab = synthetic.sft_shift_labels(w.wid, x["lengths"])
+    lab_sh = torch.from_numpy(np.ascontiguousarray(lab.reshape(b, P, m).transpose(1, 0, 2))).to(dev)
+    l_in = torch.from_numpy(synthetic.rank_losses(w.wid, P)).to(dev)
+    l_out, l_good, l_dl = (torch.empty(1, device=dev), torch.empty(P, dtype=torch.int64, device=dev),
+                           torch.empty(P, device=dev))
+    for _ in range(5):
+        uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
+    torch.cuda.synchronize()
+    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 50
+    s3.record()
+    for _ in range(reps):
+        uly.ulysses_sp_loss_aggregate(l_in, lab_sh, l_out, l_good, l_dl)
+    e3.record()
+    torch.cuda.synchronize()
+    loss_us = s3.elapsed_time(e3) * 1e3 / reps
+    loss_bytes = lab_sh.numel() * 8 + 3 * P * 8 + 4
+    return {"us_per_call": loss_us, "bytes_per_call": loss_bytes,
+            "gbs": loss_bytes / (loss_us * 1e-6) / 1e9, "launches_per_call": 2,
+            "labels": "packed SFT: per sample a U[0.1, 0.6) prompt fraction and the last position are -100"}
+
+
 # ----------------------------------------------------------------------------- profiling case
 def run_profile_case():
-    """One forward + one backward on a small case for ncu captures: P = 4,
-    b = 1, n = 16384, H_q = 32, H_kv = 8, d = 128, one causal sample,
-    virtual rank 0 only (its 8 query heads), standard-normal bf16 inputs
-    drawn on the device (seed 0).  Each tensor is above L2's size, the
-    device holds well under 1 GB.  Times nothing."""
+    """Small launches of the step's kernels for ncu captures: one seq_to_head
+    re-layout of a Llama-8B-shaped q (P = 4, n = 32768, 32 heads, d = 128:
+    256 MiB in, 256 MiB out, each above L2's size), then one forward and one
+    backward of virtual rank 0 at P = 4, b = 1, n = 16384, H_q = 32,
+    H_kv = 8, d = 128 (its 8 query heads), one causal sample,
+    standard-normal bf16 inputs drawn on the device (seed 0).  The device
+    holds about 2 GB.  Times nothing."""
     import torch
     import ulysses_head_attention_b200 as uly
     dev = torch.device("cuda:0")
-    P, b, n, hq, hkv, d = 4, 1, 16384, 32, 8, 128
     g = torch.Generator(device=dev).manual_seed(0)
+    P, b, hq, hkv, d = 4, 1, 32, 8, 128
+    x_seq = torch.randn((P, b, 32768 // P, hq, d), device=dev, generator=g).to(torch.bfloat16)
+    x_head = torch.empty((P, b, 32768, hq // P, d), dtype=torch.bfloat16, device=dev)
+    uly.ulysses_seq_to_head(x_seq, x_head)
+    del x_seq, x_head
+    n = 16384
 
     def mk(h):
         return torch.randn((P, b, n, h // P, d), device=dev, generator=g).to(torch.bfloat16)

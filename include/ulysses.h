@@ -247,11 +247,54 @@ uly_status ulysses_attn_lse_merge(const float* o_parts, const float* lse_parts, 
                                   void* stream);
 
 /*
+ * Block calls: one block of query rows against one block of key rows, each
+ * stored compactly (ring attention, where a rank holds only its own
+ * sequence block and receives the others' key blocks one at a time).
+ *   q_blk, o_blk, do_blk, dq_blk  [P][b][q_rows][h_q/P][d]: global rows
+ *                                 [q_base, q_base + q_rows)
+ *   k_blk, v_blk, dk_blk, dv_blk  [P][b][k_rows][kv heads per rank][d]:
+ *                                 global keys [k_base, k_base + k_rows)
+ *   lse_blk                       [P][b][h_q/P][q_rows]
+ *   position_ids                  [b][n], the whole sequence's (sample
+ *                                 starts are global)
+ * q_base and k_base are multiples of 128, both blocks lie inside [0, n)
+ * (ULY_ERR_INVALID_ARG otherwise).  All P ranks' head slices are computed.
+ * Query i sees key j iff j <= i, both in one sample, and j in the key block.
+ * ulysses_attn_fwd_block gives each query row's partial O and LSE over the
+ * key block (O = 0, LSE = -inf for a row that sees none of it), to be
+ * combined with ulysses_attn_lse_merge.  ulysses_attn_bwd_block takes the
+ * merged O and LSE of the query block and gives the key block's share of
+ * dQ and the query block's contributions to dK and dV (all overwritten).
+ * Workspaces as for the whole-sequence calls with the same shape.  Only
+ * the tiles of the two blocks are launched.
+ */
+uly_status ulysses_attn_fwd_block(const void* q_blk, const void* k_blk, const void* v_blk,
+                                  const int64_t* position_ids, const uly_shape* shape, int64_t q_base,
+                                  int64_t q_rows, int64_t k_base, int64_t k_rows, float softmax_scale,
+                                  void* o_blk, uly_dtype o_dtype, float* lse_blk, void* ws, size_t ws_bytes,
+                                  void* stream);
+uly_status ulysses_attn_bwd_block(const void* q_blk, const void* k_blk, const void* v_blk, const void* o_blk,
+                                  uly_dtype o_dtype, const float* lse_blk, const void* do_blk,
+                                  const int64_t* position_ids, const uly_shape* shape, int64_t q_base,
+                                  int64_t q_rows, int64_t k_base, int64_t k_rows, float softmax_scale,
+                                  void* dq_blk, void* dk_blk, void* dv_blk, uly_dtype g_dtype, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/*
+ * ulysses_accumulate -- dst[i] += src[i] for i < count, float32 (count a
+ * multiple of 4, both 16-byte aligned; dst == src is allowed, other
+ * overlaps are not).  The ring passes' sums of dQ shares and of the dK / dV
+ * that travel with a key block.
+ */
+uly_status ulysses_accumulate(float* dst, const float* src, int64_t count, void* stream);
+
+/*
  * ulysses_attn_bwd_timed -- ulysses_attn_bwd that also records five
  * caller-owned CUDA events on `stream` around its kernels, for measuring
  * each kernel's device time (the pages have no counterpart; this is
  * instrumentation).  events[0] before the sample-table kernel, events[1]
- * before the row-statistics kernel, events[2] before the dK/dV kernel,
+ * before the preparation kernels (largest magnitudes, fp16 operand copies,
+ * row statistics), events[2] before the dK/dV kernel,
  * events[3] before the dQ kernel, events[4] after it.  `events` points to
  * five cudaEvent_t handles (as void*), created by the caller on the current
  * device; a null array or a null handle returns ULY_ERR_INVALID_ARG and
@@ -332,6 +375,92 @@ uly_status ulysses_sp_loss_aggregate(const float* losses, const int64_t* shift_l
  * error cases the outputs are invalid).
  */
 uly_status ulysses_workspace_status(void* ws, void* stream, int32_t* code);
+
+/*
+ * Between GPUs: the two all-to-alls fused with the re-layout
+ * ----------------------------------------------------------
+ * Blog "How Ulysses works", steps 3 and 5, with one GPU per rank: each rank
+ * stores its chunks straight into its peers' buffers over NVLink (plain
+ * stores through peer-mapped pointers; no collective library, no TMA), then
+ * releases one flag per destination.  A consumer runs ulysses_wait_flags on
+ * its own flag array before reading what it received.
+ *
+ * ulysses_seq_to_head_push -- rank `rank` of P sends its seq shard
+ *   x_seq [b][n/P][H][d] (its own device memory) to every rank s:
+ *     dst_heads[s][bb][rank*n/P + t][j] = x_seq[bb][t][s*H/P + j]
+ *   dst_heads[s] is rank s's head-layout buffer [b][n][H/P][d] (for
+ *   s != rank a peer-mapped pointer, e.g. from ulysses_ipc_open).  Once all
+ *   of rank s's rows are stored and fenced at system scope, `epoch` is
+ *   stored with release semantics into dst_flags[s][rank] (dst_flags[s]:
+ *   rank s's uint32 flag array of P slots).
+ * ulysses_head_to_seq_push -- the inverse, for O and the gradients: rank
+ *   `rank` holds x_head [b][n][H/P][d] (heads [rank*H/P, (rank+1)*H/P) of
+ *   all tokens) and sends tokens [s*n/P, (s+1)*n/P) to rank s:
+ *     dst_seqs[s][bb][t][rank*H/P + j] = x_head[bb][s*n/P + t][j]
+ *   then releases dst_flags[s][rank] = epoch.
+ *   Both: arrays dst_* hold P pointers (host memory); P <= 64; dtype bf16
+ *   or fp32; H/P*d*element size a multiple of 16 bytes (else
+ *   ULY_ERR_UNSUPPORTED); epoch != 0 (a flag's 0 means "nothing yet"; use a
+ *   new epoch per exchange); ws: device workspace of >= 4*P bytes, 256-byte
+ *   aligned, for the per-destination completion counters (cleared by the
+ *   call).  The caller guarantees that no destination is still reading the
+ *   buffer from an earlier exchange (e.g. a barrier or double buffering).
+ *
+ * ulysses_wait_flags -- one warp polls flags[0..count) with acquire loads
+ *   at system scope until every slot holds `epoch` or a later epoch
+ *   (compared modulo 2^32: slot - epoch as a signed 32-bit number is >= 0;
+ *   epochs grow by one per exchange, so a slot never lags or leads by 2^31 or
+ *   more).  Kernels enqueued after
+ *   it on `stream` then see the data the flags released.  Gives up after
+ *   limit_ns (in [1 us, 60 s]) and records ULY_ERR_TIMEOUT in the status
+ *   word at the start of ws (256-byte aligned device memory; read it with
+ *   ulysses_workspace_status).
+ *
+ * ulysses_release_flags -- stores `epoch` (!= 0) into each of `count` (1..64)
+ *   uint32 slots (device addresses, this GPU's or peer-mapped), each after a
+ *   system-scope fence and with release semantics: everything enqueued on
+ *   `stream` before it is visible to whoever acquires a slot.  The "buffer
+ *   free" signal of a receiver to its senders; the push calls do the same
+ *   for their data.
+ *
+ * ulysses_ipc_handle / ulysses_ipc_open / ulysses_ipc_close -- the CUDA IPC
+ *   handle (64 bytes) of a device allocation, opened in another process as
+ *   a peer-mapped pointer (peer access enabled lazily), and closed again.
+ *   Host-side plumbing for the push calls; ULY_ERR_CUDA when CUDA refuses.
+ */
+uly_status ulysses_seq_to_head_push(const void* x_seq, void* const* dst_heads, uint32_t* const* dst_flags,
+                                    int32_t rank, int64_t b, int64_t n, int64_t H, int64_t d, int32_t P,
+                                    uly_dtype dtype, uint32_t epoch, void* ws, size_t ws_bytes, void* stream);
+uly_status ulysses_head_to_seq_push(const void* x_head, void* const* dst_seqs, uint32_t* const* dst_flags,
+                                    int32_t rank, int64_t b, int64_t n, int64_t H, int64_t d, int32_t P,
+                                    uly_dtype dtype, uint32_t epoch, void* ws, size_t ws_bytes, void* stream);
+uly_status ulysses_wait_flags(const uint32_t* flags, int32_t count, uint32_t epoch, uint64_t limit_ns, void* ws,
+                              void* stream);
+uly_status ulysses_release_flags(uint32_t* const* slots, int32_t count, uint32_t epoch, void* stream);
+uly_status ulysses_ipc_handle(const void* dev_ptr, void* handle_out);
+uly_status ulysses_ipc_open(const void* handle, void** dev_ptr_out);
+uly_status ulysses_ipc_close(void* dev_ptr);
+
+/*
+ * ulysses_selftest_wait_timeout -- runs the failure path of the attention
+ * kernels' bounded waits on purpose, so that it can be checked on a GPU.
+ * (Not a step of the method: the pages have no counterpart; it tests the
+ * library's own failure detection.)  One CTA of the attention kernels'
+ * shape allocates TMEM, starts one bulk copy of workspace bytes
+ * [256, 1280) into shared memory, and then waits on a barrier nothing
+ * arrives at: the first wait to exceed limit_ns records ULY_ERR_TIMEOUT in
+ * the workspace status word and raises the CTA's abort flag, the other
+ * waits return on the flag, the copy is waited for (bounded), TMEM is freed
+ * and the kernel returns.  The stream and context stay usable.
+ *   ws, ws_bytes  device workspace, 256-byte aligned, >= 1280 bytes
+ *                 (ULY_ERR_WORKSPACE otherwise); only its status word is
+ *                 written.
+ *   limit_ns      the waits' time limit, in [1000, 5e9] ns
+ *                 (ULY_ERR_INVALID_ARG otherwise).
+ * Returns once the kernel is enqueued; ulysses_workspace_status(ws, ...)
+ * then reports ULY_ERR_TIMEOUT.
+ */
+uly_status ulysses_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream);
 
 /* Static English text for a status code. */
 const char* ulysses_status_string(uly_status s);

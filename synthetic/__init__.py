@@ -152,11 +152,13 @@ def make_inputs(w: Workload, with_do: Optional[bool] = None) -> Dict[str, np.nda
 
 def custom_inputs(seed: int, b: int, n: int, h_q: int, h_kv: int, d: int,
                   lengths: Optional[List[List[int]]] = None, with_do: bool = True,
-                  scale: float = 1.0) -> Dict[str, np.ndarray]:
+                  scale: float = 1.0, qk_scale: float = 1.0, do_scale: float = 1.0) -> Dict[str, np.ndarray]:
     """Inputs of an arbitrary small shape (for edge-case tests).
 
     ``lengths`` gives each batch row's sample lengths (default: one sample);
-    ``scale`` multiplies the normal draws before bf16 rounding.
+    ``scale`` multiplies the normal draws before bf16 rounding, and
+    ``qk_scale`` multiplies those of q and k once more (large logits with
+    ordinary values), ``do_scale`` those of dO (gradient magnitudes).
     """
     g = streams(10_000 + seed)
     if lengths is None:
@@ -164,19 +166,19 @@ def custom_inputs(seed: int, b: int, n: int, h_q: int, h_kv: int, d: int,
     for ls in lengths:
         assert sum(ls) == n, "sample lengths must cover the row"
 
-    def draw(rng, shape):
-        x = rng.standard_normal(int(np.prod(shape)), dtype=np.float32) * np.float32(scale)
+    def draw(rng, shape, extra=1.0):
+        x = rng.standard_normal(int(np.prod(shape)), dtype=np.float32) * np.float32(scale) * np.float32(extra)
         return f32_to_bf16_bits(x).reshape(shape)
 
     out = {
-        "q": draw(g["q"], (b, n, h_q, d)),
-        "k": draw(g["k"], (b, n, h_kv, d)),
+        "q": draw(g["q"], (b, n, h_q, d), qk_scale),
+        "k": draw(g["k"], (b, n, h_kv, d), qk_scale),
         "v": draw(g["v"], (b, n, h_kv, d)),
         "position_ids": np.stack([position_ids_from_lengths(ls) for ls in lengths]),
         "lengths": lengths,
     }
     if with_do:
-        out["do"] = draw(g["do"], (b, n, h_q, d))
+        out["do"] = draw(g["do"], (b, n, h_q, d), do_scale)
     return out
 
 

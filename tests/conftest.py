@@ -32,3 +32,16 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device on this host")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Every parity comparison's measured error, beside its bound."""
+    mod = sys.modules.get("gpu_util")
+    recs = getattr(mod, "RECORDS", None) if mod else None
+    if not recs:
+        return
+    tr = terminalreporter
+    tr.section("measured errors (max-abs <= bound, mean-rel <= bound)")
+    for what, ma, mr, bma, bmr in recs:
+        rel = "" if mr != mr else f"  mean-rel {mr:.2e} (<= {bmr:g})"
+        tr.write_line(f"{what}: max-abs {ma:.2e} (<= {bma:g}){rel}")

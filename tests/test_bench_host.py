@@ -26,12 +26,12 @@ class _Thread:
         pass
 
 
-def _sampler(lines, window):
+def _record(lines, window):
     s = bench.ClockSampler(0)
     s.proc, s.thread = _Proc(), _Thread()
     s.lines = lines
-    s.mark(*window)
-    return s
+    s.stop()
+    return s.summary(*window)
 
 
 def _line(sm, cap="Not Active", hw="Not Active", mask="0x0000000000000000"):
@@ -46,7 +46,7 @@ def test_clock_record_keeps_only_the_timed_window(monkeypatch):
              (2.0, _line(1610)),
              (2.05, "garbled"),                                        # malformed: skipped
              (3.0, _line(700, hw="Active", mask="0x0000000000000008"))]  # after the window
-    rec = _sampler(lines, (1.0, 2.0)).stop()
+    rec = _record(lines, (1.0, 2.0))
     assert rec["samples"] == 3
     assert rec["sm_mhz"] == 1610.0 and rec["sm_max_mhz"] == 1965.0
     assert (rec["sm_mhz_min"], rec["sm_mhz_max"]) == (1600.0, 1620.0)
@@ -54,26 +54,55 @@ def test_clock_record_keeps_only_the_timed_window(monkeypatch):
     assert rec["active_masks"] == ["0x0", "0x4"]
 
 
+def test_clock_records_of_two_windows(monkeypatch):
+    """One sampler serves several timed windows (the headline and each other workload)."""
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    lines = [(1.0, _line(1900)), (1.5, _line(1880)), (3.0, _line(1500, cap="Active", mask="0x0000000000000004"))]
+    s = bench.ClockSampler(0)
+    s.proc, s.thread = _Proc(), _Thread()
+    s.lines = lines
+    a, b = s.summary(0.9, 1.6), s.summary(2.9, 3.1)
+    assert (a["samples"], a["sm_mhz"], a["reasons"]) == (2, 1890.0, [])
+    assert (b["samples"], b["sm_mhz"], b["reasons"]) == (1, 1500.0, ["sw_power_cap"])
+
+
+def test_clock_peak_is_the_tensor_rate_at_the_sampled_clock():
+    assert bench.clock_peak_tflops(None) is None
+    # 8192 flop per clock per SM x 148 SMs at 1.85 GHz: the nominal 2.24 PFLOP/s dense bf16
+    assert bench.clock_peak_tflops(1850.0) == pytest.approx(8192 * 148 * 1.85e9 / 1e12)
+
+
 def test_clock_record_names_reasons_from_the_mask(monkeypatch):
     monkeypatch.setattr(bench.time, "sleep", lambda s: None)
     lines = [(1.0, _line(1200, mask="0x0000000000000048"))]           # hw_slowdown | hw_thermal_slowdown
-    rec = _sampler(lines, (0.0, 5.0)).stop()
+    rec = _record(lines, (0.0, 5.0))
     assert rec["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
 
 
 def test_clock_record_without_nvidia_smi():
-    rec = bench.ClockSampler(0).stop()
+    s = bench.ClockSampler(0)
+    s.stop()
+    rec = s.summary(0.0, 1.0)
     assert rec["sm_mhz"] is None and rec["reasons"] == ["nvidia-smi unavailable"]
 
 
 def test_recorded_traffic_applies_only_to_its_workload_and_sources(monkeypatch):
-    rec = bench.TRAFFIC["attn_bwd_dkdv_kernel"]
+    rec = {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 123456789,
+           "sources_sha256": bench.sources_sha256("attn_bwd_dkdv_kernel")}
+    monkeypatch.setitem(bench.TRAFFIC, "attn_bwd_dkdv_kernel", rec)
     assert bench.recorded_traffic("attn_bwd_dkdv_kernel", rec["workload"]) == rec["bytes_per_launch"]
-    assert bench.recorded_traffic("attn_bwd_dkdv_kernel", "llama8b_p8_n64k") is None
+    assert bench.recorded_traffic("attn_bwd_dkdv_kernel", "llama8b_p4_n32k") is None
     assert bench.recorded_traffic("attn_bwd_dq_kernel", rec["workload"]) is None
     # once the kernel's sources differ from the ones the counters were taken on
     monkeypatch.setitem(bench.TRAFFIC, "attn_bwd_dkdv_kernel", dict(rec, sources_sha256="0" * 64))
     assert bench.recorded_traffic("attn_bwd_dkdv_kernel", rec["workload"]) is None
+
+
+def test_every_recorded_traffic_matches_the_current_sources():
+    """A committed record whose kernel has changed since the capture would be
+    reported as null: keep only records of the current sources."""
+    for kernel, rec in bench.TRAFFIC.items():
+        assert rec["sources_sha256"] == bench.sources_sha256(kernel), kernel
 
 
 def test_sources_hash_covers_the_kernel_region(tmp_path, monkeypatch):

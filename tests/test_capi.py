@@ -308,3 +308,54 @@ def test_noalloc_forward_refuses_before_touching_the_device():
     assert call(shape(b=1, n=1 << 20)) == WORKSPACE
     assert call(shape(b=2, n=1 << 19)) == WORKSPACE
     assert uly.ulysses_attn_fwd_workspace(shape(b=1, n=1 << 19)) <= 256 + 2 * 4 * (1 << 19)
+
+
+@no_gpu
+def test_selftest_wait_timeout_rejects():
+    import ulysses_head_attention_b200 as uly
+    f = uly.lib.ulysses_selftest_wait_timeout
+    assert f(None, 4096, 1000000, None) == WORKSPACE                 # no workspace
+    assert f(F + 16, 4096, 1000000, None) == WORKSPACE               # not 256-byte aligned
+    assert f(F, 1024, 1000000, None) == WORKSPACE                    # below 256 + 1024 bytes
+    assert f(F, 4096, 999, None) == INVALID                          # limit below 1 us
+    assert f(F, 4096, 5000000001, None) == INVALID                   # limit above 5 s
+
+
+@no_gpu
+def test_push_and_wait_reject():
+    import ulysses_head_attention_b200 as uly
+    P = 4
+    dst = (ctypes.c_void_p * P)(*[F + (i + 1) * (1 << 30) for i in range(P)])
+    flg = (ctypes.c_void_p * P)(*[F + (i + 9) * (1 << 30) for i in range(P)])
+    ws = F + (20 << 30)
+    push = uly.lib.ulysses_seq_to_head_push
+    ok_args = (F, dst, flg, 0, 1, 4096, 32, 128, P, 0, 1, ws, 4096, None)
+
+    def call(**kw):
+        names = ("src", "dst", "flags", "rank", "b", "n", "H", "d", "P", "dt", "epoch", "ws", "ws_bytes", "stream")
+        a = dict(zip(names, ok_args))
+        a.update(kw)
+        return push(*[a[k] for k in names])
+
+    assert call(rank=4) == INVALID                      # rank outside [0, P)
+    assert call(rank=-1) == INVALID
+    assert call(n=4095) == INVALID                      # n % P
+    assert call(H=30) == INVALID                        # H % P
+    assert call(epoch=0) == INVALID                     # 0 means "nothing yet"
+    assert call(P=65, rank=0) == INVALID                # more ranks than the kernel carries
+    assert call(ws=None) == WORKSPACE
+    assert call(ws_bytes=8) == WORKSPACE                # below 4 P bytes
+    assert call(src=F + 8) == INVALID                   # misaligned source
+    assert call(src=F + (1 << 30)) == INVALID           # source overlaps this rank's own destination
+    assert call(d=4, dt=0, H=4) == UNSUPPORTED          # a run of 2 bytes: not a 16-byte multiple
+    bad = (ctypes.c_void_p * P)(*([0] + [F] * (P - 1)))
+    assert call(dst=bad) == INVALID                     # a null destination
+    wait = uly.lib.ulysses_wait_flags
+    assert wait(F, 0, 1, 10**6, ws, None) == INVALID    # no flags
+    assert wait(F, 4, 0, 10**6, ws, None) == INVALID    # epoch 0
+    assert wait(F, 4, 1, 10, ws, None) == INVALID       # limit below 1 us
+    assert wait(F, 4, 1, 10**6, None, None) == WORKSPACE
+    assert uly.lib.ulysses_ipc_handle(None, None) == INVALID
+    assert uly.lib.ulysses_ipc_open(None, None) == INVALID
+    assert uly.lib.ulysses_ipc_close(None) == INVALID
+

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synthetic
-from gpu_util import (LSE_MAX_ABS, MAX_ABS_BF16, MEAN_REL_BF16, assert_close, to_dev_bf16)
+from gpu_util import (LSE_MAX_ABS, MAX_ABS_BF16, MEAN_REL_BF16, assert_close, assert_lse_close, to_dev_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -69,15 +69,15 @@ def test_fwd_matches_oracle(cuda_device, case):
     x = synthetic.custom_inputs(100 + CASES.index(case), b, n, hq, hkv, d, lengths=lengths, with_do=False)
     O, L, heads = gpu_fwd(x, P, cuda_device)
     O_ref, L_ref = oracle_fwd(heads, x["position_ids"], P)
-    assert_close(O, O_ref, f"{case[0]} O")
-    assert np.abs(L - L_ref).max() <= LSE_MAX_ABS, f"{case[0]} LSE {np.abs(L - L_ref).max():.3e}"
+    assert_close(O, O_ref, f"fwd {case[0]} O")
+    assert_lse_close(L, L_ref, f"fwd {case[0]} LSE")
 
 
 def test_fwd_bf16_output(cuda_device):
     x = synthetic.custom_inputs(31, 1, 768, 8, 2, 128, lengths=[[500, 268]], with_do=False)
     O, L, heads = gpu_fwd(x, 2, cuda_device, o_dtype=torch.bfloat16)
     O_ref, L_ref = oracle_fwd(heads, x["position_ids"], 2)
-    assert_close(O, O_ref, "bf16 O", MAX_ABS_BF16, MEAN_REL_BF16)
+    assert_close(O, O_ref, "fwd bf16 storage O", MAX_ABS_BF16, MEAN_REL_BF16)
     assert np.abs(L - L_ref).max() <= LSE_MAX_ABS
 
 
@@ -87,22 +87,22 @@ def test_fwd_single_rank_leaves_others_untouched(cuda_device):
     for rank in (0, 2, 3):
         O, L, heads = gpu_fwd(x, P, cuda_device, rank=rank, sentinel=7.0)
         O_ref, L_ref = oracle_fwd(heads, x["position_ids"], P, rank=rank)
-        assert_close(O[rank], O_ref[rank], f"rank {rank} O")
+        assert_close(O[rank], O_ref[rank], f"fwd rank {rank} O")
         assert np.abs(L[rank] - L_ref[rank]).max() <= LSE_MAX_ABS
         others = [s for s in range(P) if s != rank]
         assert (O[others] == 7.0).all() and (L[others] == 7.0).all()
 
 
 def test_fwd_large_logits_stay_finite(cuda_device):
-    """Inputs scaled x8 give scores in the hundreds: exercises the lazy O
-    rescale and the max subtraction.  The values are 8x larger too, so the
-    absolute bound scales with them: P is rounded to bf16 (2^-8 relative)
-    before the PV product, giving |error| <~ 2^-8 max|v|."""
-    x = synthetic.custom_inputs(33, 1, 1024, 4, 2, 128, with_do=False, scale=8.0)
+    """q and k scaled x8 give scores in the hundreds: exercises the lazy O
+    rescale and the max subtraction (v stays standard normal, so the usual
+    element-wise bounds apply).  LSE is in the hundreds too: its bound is
+    relative."""
+    x = synthetic.custom_inputs(33, 1, 1024, 4, 2, 128, with_do=False, qk_scale=8.0)
     O, L, heads = gpu_fwd(x, 2, cuda_device)
     O_ref, L_ref = oracle_fwd(heads, x["position_ids"], 2)
-    vmax = np.abs(synthetic.bf16_bits_to_f64(heads[2])).max()
-    assert_close(O, O_ref, "scaled O", max_abs=2.0 ** -8 * vmax)
+    assert np.abs(L_ref).max() > 100.0
+    assert_close(O, O_ref, "fwd large logits O")
     assert np.abs(L - L_ref).max() <= 1e-3 * max(1.0, np.abs(L_ref).max())
 
 

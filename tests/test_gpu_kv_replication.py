@@ -7,10 +7,8 @@
   one bf16 rounding for bf16 data.
 * The whole layer with H_kv < P (re-layouts, forward, backward, the reducing
   re-layout of dK and dV) against the oracle's layer, with the tolerances of
-  the other short-row attention tests: fp32 outputs, sum|g-r|/sum|r| <= 2e-3,
-  max-abs <= max(1e-2, 2^-8 max|ref|) (gpu_util.edge_max_abs: P and dS enter
-  the MMAs as bf16, and a replicated kv head's dK / dV sum the whole query
-  group, so their magnitude, and the absolute error with it, grows).
+  the other attention tests: fp32 outputs, every element within 1e-2,
+  sum|g-r|/sum|r| <= 2e-3.
 """
 import numpy as np
 import pytest
@@ -18,7 +16,7 @@ import torch
 
 import oracle
 import synthetic
-from gpu_util import assert_close, edge_max_abs, to_dev_bf16
+from gpu_util import assert_close, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -134,4 +132,4 @@ def test_layer_with_replication_matches_oracle(cuda_device, P, hq, hkv, n, lengt
     refs = oracle.ulysses_layer_bwd(f64["q"], f64["k"], f64["v"], f64["do"], x["position_ids"], P)
     assert_close(o_seq.cpu().numpy(), O_ref, "O")
     for nm, ref in zip(("dq", "dk", "dv"), refs):
-        assert_close(g[nm].cpu().numpy(), ref, nm, max_abs=edge_max_abs(ref))
+        assert_close(g[nm].cpu().numpy(), ref, f"kv replication {nm}")

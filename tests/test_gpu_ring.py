@@ -9,7 +9,8 @@
   full attention (same bounds as the forward tests).
 * ulysses_attn_bwd_kv_range, given the merged O and LSE: each block's dQ
   share, and dK / dV that equal the full gradient on the block's keys and
-  are exactly zero elsewhere; the shares add up to the full dQ.
+  are exactly zero elsewhere; the shares add up to the full dQ (fp32,
+  every element within 1e-2, sum|g-r|/sum|r| <= 2e-3).
 """
 import numpy as np
 import pytest
@@ -17,7 +18,7 @@ import torch
 
 import oracle
 import synthetic
-from gpu_util import LSE_MAX_ABS, assert_close, edge_max_abs, to_dev_bf16
+from gpu_util import LSE_MAX_ABS, assert_close, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -128,11 +129,11 @@ def test_backward_blocks_add_up(cuda_device, cuts):
                                              x["position_ids"], P, a, b)
         got = [x_.cpu().numpy() for x_ in g]
         for nm, gt, rf in zip(("dQ", "dK", "dV"), got, refs):
-            assert_close(gt, rf, f"{nm} block [{a},{b})", max_abs=edge_max_abs(rf))
+            assert_close(gt, rf, f"ring bwd {nm} block [{a},{b})")
         for gt in got[1:]:
             assert not gt[:, :, :a].any() and not gt[:, :, b:].any()   # keys outside the block: exactly 0
         dq_sum += got[0]
-    assert_close(dq_sum, dq_full, "sum of dQ shares", max_abs=edge_max_abs(dq_full))
+    assert_close(dq_sum, dq_full, "ring bwd sum of dQ shares")
 
 
 def test_range_bounds_are_checked(cuda_device):

@@ -6,9 +6,12 @@ seq_to_head(q, k, v) -> forward (fp32 O) -> head_to_seq(O); seq_to_head(dO)
 buffers are byte-identical to unsharded [n][H][d] tensors, so outputs are
 indexed by (token, head) directly.
 
-Compared against the fp64 oracle, element by element, on outputs it can
-compute one at a time (tolerances as everywhere: max-abs <= 1e-2,
-sum|g-r|/sum|r| <= 2e-3 for fp32-stored values, LSE max-abs <= 1e-3):
+Compared against the fp64 oracle, element by element (tolerances as
+everywhere: every element within 1e-2, sum|g-r|/sum|r| <= 2e-3 for
+fp32-stored values, LSE max-abs <= 1e-3):
+  * every element of O, LSE and dQ of all G query heads of one kv group and
+    of that kv head's dK and dV, at full size (the Llama-8B shape and the
+    packed SFT batch; the oracle's per-head work runs in parallel processes);
   * O and LSE of sampled query rows of every head (rows 0 and n-1, the first
     and last row of random 128-row tiles, random rows), each against its
     full visible prefix;
@@ -24,7 +27,8 @@ import torch
 
 import oracle
 import synthetic
-from gpu_util import LSE_MAX_ABS, assert_close, to_dev_bf16
+from gpu_util import LSE_MAX_ABS, assert_close, assert_lse_close, to_dev_bf16
+from oracle_pool import heads_fwd_bwd
 
 pytestmark = [pytest.mark.gpu, pytest.mark.large]
 
@@ -86,6 +90,26 @@ def run_layer(w, x, dev, backward=True):
     return out
 
 
+def check_full_group(w, x, out, g):
+    """Every element of one kv group: O, LSE, dQ of its G query heads and
+    dK, dV of kv head g, against the oracle's blocked fp64 attention."""
+    ss = oracle.segment_starts(x["position_ids"])[0]
+    scale = oracle.default_scale(w.d)
+    k = synthetic.bf16_bits_to_f64(x["k"][0, :, g])
+    v = synthetic.bf16_bits_to_f64(x["v"][0, :, g])
+    hs = list(range(g * w.group, (g + 1) * w.group))
+    jobs = [(synthetic.bf16_bits_to_f64(x["q"][0, :, h]), k, v,
+             synthetic.bf16_bits_to_f64(x["do"][0, :, h]) if w.backward else None, ss, scale) for h in hs]
+    res = heads_fwd_bwd(jobs, backward=w.backward)
+    what = f"{w.name} kv group {g} (all {w.group} query heads, every row)"
+    assert_close(out["o"][:, hs], np.stack([r[0] for r in res], axis=1), f"{what} O")
+    assert_lse_close(out["lse"][hs], np.stack([r[1] for r in res]), f"{what} LSE")
+    if w.backward:
+        assert_close(out["dq"][:, hs], np.stack([r[2] for r in res], axis=1), f"{what} dQ")
+        assert_close(out["dk"][:, g], sum(r[3] for r in res), f"{w.name} kv head {g} dK (every key)")
+        assert_close(out["dv"][:, g], sum(r[4] for r in res), f"{w.name} kv head {g} dV (every key)")
+
+
 def check_forward(w, x, out, rng, rows_per_head):
     ss = oracle.segment_starts(x["position_ids"])[0]
     scale = oracle.default_scale(w.d)
@@ -100,7 +124,7 @@ def check_forward(w, x, out, rng, rows_per_head):
             got.append(out["o"][rows, h]); ref.append(o_r)
             gl.append(out["lse"][h, rows]); rl.append(l_r)
     assert_close(np.concatenate(got), np.concatenate(ref), f"{w.name} O (sampled rows)")
-    assert np.abs(np.concatenate(gl) - np.concatenate(rl)).max() <= LSE_MAX_ABS
+    assert_lse_close(np.concatenate(gl), np.concatenate(rl), f"{w.name} LSE (sampled rows)")
 
 
 def check_backward(w, x, out, rng, rows_per_head):
@@ -139,6 +163,11 @@ def check_backward(w, x, out, rng, rows_per_head):
     assert_close(gk[1], rk[1], f"{w.name} dV (last {W_KEYS} keys of every sample)")
 
 
+# kv group compared in full: the first rank's first group for the Llama-8B
+# shape, the last rank's group for the packed batch
+FULL_GROUP = {"llama8b_p4_n32k": 0, "packed_sft_p8_n64k": 7}
+
+
 @pytest.mark.parametrize("name", ["tiny_p2_n256", "llama8b_p4_n32k", "packed_sft_p8_n64k", "roundtrip_p4_n128k"])
 def test_workload_layer(cuda_device, name):
     w = synthetic.WORKLOADS[name]
@@ -152,6 +181,8 @@ def test_workload_layer(cuda_device, name):
         assert_close(out["o"], oracle.unshard(O_ref)[0], "tiny O (all elements)")
         assert np.abs(out["lse"] - L_ref.transpose(1, 0, 2, 3).reshape(w.h_q, w.n)).max() <= LSE_MAX_ABS
         return
+    if name in FULL_GROUP:
+        check_full_group(w, x, out, FULL_GROUP[name])
     check_forward(w, x, out, rng, rows_per_head=24)
     if w.backward:
         check_backward(w, x, out, rng, rows_per_head=12)

@@ -32,7 +32,11 @@ EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head
            "ulysses_transpose_runs", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_bwd_timed", "ulysses_attn_fwd_noalloc",
            "ulysses_attn_fwd_kv_range", "ulysses_attn_bwd_kv_range", "ulysses_attn_lse_merge",
-           "ulysses_sp_loss_aggregate", "ulysses_workspace_status", "ulysses_status_string")
+           "ulysses_sp_loss_aggregate", "ulysses_workspace_status", "ulysses_selftest_wait_timeout",
+           "ulysses_seq_to_head_push", "ulysses_head_to_seq_push", "ulysses_wait_flags", "ulysses_release_flags",
+           "ulysses_ipc_handle",
+           "ulysses_ipc_open", "ulysses_ipc_close", "ulysses_attn_fwd_block", "ulysses_attn_bwd_block",
+           "ulysses_accumulate", "ulysses_status_string")
 
 
 class UlyShape(ctypes.Structure):
@@ -71,6 +75,20 @@ def _load() -> ctypes.CDLL:
         "ulysses_attn_lse_merge": ([vp, vp, i32, shp, vp, i32, vp, vp], i32),
         "ulysses_sp_loss_aggregate": ([vp, vp, i64, i64, i32, i64, vp, vp, vp, vp], i32),
         "ulysses_workspace_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
+        "ulysses_selftest_wait_timeout": ([vp, sz, ctypes.c_uint64, vp], i32),
+        "ulysses_seq_to_head_push": ([vp, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i64, i64, i64, i64, i32, i32,
+                                      ctypes.c_uint32, vp, sz, vp], i32),
+        "ulysses_head_to_seq_push": ([vp, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i64, i64, i64, i64, i32, i32,
+                                      ctypes.c_uint32, vp, sz, vp], i32),
+        "ulysses_wait_flags": ([vp, i32, ctypes.c_uint32, ctypes.c_uint64, vp, vp], i32),
+        "ulysses_release_flags": ([ctypes.POINTER(vp), i32, ctypes.c_uint32, vp], i32),
+        "ulysses_ipc_handle": ([vp, ctypes.c_char_p], i32),
+        "ulysses_ipc_open": ([ctypes.c_char_p, ctypes.POINTER(vp)], i32),
+        "ulysses_ipc_close": ([vp], i32),
+        "ulysses_attn_fwd_block": ([vp, vp, vp, vp, shp, i64, i64, i64, i64, f32, vp, i32, vp, vp, sz, vp], i32),
+        "ulysses_attn_bwd_block": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i64, i64, i64, i64, f32, vp, vp, vp, i32,
+                                    vp, sz, vp], i32),
+        "ulysses_accumulate": ([vp, vp, i64, vp], i32),
         "ulysses_status_string": ([i32], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -358,6 +376,73 @@ def ulysses_attn_bwd_kv_range(q_head, k_head, v_head, o_head, lse, do_head, posi
                                          _stream(stream)), "ulysses_attn_bwd_kv_range")
 
 
+def _check_block(q_blk, k_blk, v_blk, position_ids, o_blk, lse_blk, stream, do_blk=None, dq_blk=None, dk_blk=None,
+                 dv_blk=None, ws=None):
+    """Layouts of the block calls: Q-side rows q_rows, K-side rows k_rows."""
+    if not isinstance(q_blk, torch.Tensor) or q_blk.dim() != 5 or not isinstance(k_blk, torch.Tensor) \
+            or k_blk.dim() != 5:
+        raise ValueError("q_blk / k_blk must be [P][b][rows][heads][d]")
+    P, b, qr, hq, d = q_blk.shape
+    kr, hkv = k_blk.shape[2], k_blk.shape[3]
+    if not isinstance(position_ids, torch.Tensor) or position_ids.dim() != 2:
+        raise ValueError("position_ids must be [b][n]")
+    n = position_ids.shape[1]
+    _expect(q_blk, (P, b, qr, hq, d), _BF16, "q_blk")
+    _expect(k_blk, (P, b, kr, hkv, d), _BF16, "k_blk")
+    _expect(v_blk, (P, b, kr, hkv, d), _BF16, "v_blk")
+    _expect(position_ids, (b, n), _I64, "position_ids")
+    _expect(o_blk, (P, b, qr, hq, d), _OUT, "o_blk")
+    _expect(lse_blk, (P, b, hq, qr), _F32, "lse_blk")
+    more = {}
+    if do_blk is not None:
+        _expect(do_blk, (P, b, qr, hq, d), _BF16, "do_blk")
+        _expect(dq_blk, (P, b, qr, hq, d), _OUT, "dq_blk")
+        _expect(dk_blk, (P, b, kr, hkv, d), (dq_blk.dtype,), "dk_blk")
+        _expect(dv_blk, (P, b, kr, hkv, d), (dq_blk.dtype,), "dv_blk")
+        more = dict(do_blk=do_blk, dq_blk=dq_blk, dk_blk=dk_blk, dv_blk=dv_blk)
+    if ws is not None:
+        more["ws"] = ws
+    _one_device(stream, q_blk=q_blk, k_blk=k_blk, v_blk=v_blk, position_ids=position_ids, o_blk=o_blk,
+                lse_blk=lse_blk, **more)
+    return UlyShape(b, n, hq * P, hkv * P, d, P), qr, kr
+
+
+def ulysses_attn_fwd_block(q_blk, k_blk, v_blk, position_ids, o_blk, lse_blk, ws, q_base: int, k_base: int,
+                           softmax_scale: float = 0.0, stream=None) -> None:
+    """Partial attention of the query rows [q_base, q_base + q_rows) over the
+    keys [k_base, k_base + k_rows), both stored compactly."""
+    shape, qr, kr = _check_block(q_blk, k_blk, v_blk, position_ids, o_blk, lse_blk, stream, ws=ws)
+    _check(lib.ulysses_attn_fwd_block(_dev(q_blk, "q_blk"), _dev(k_blk, "k_blk"), _dev(v_blk, "v_blk"),
+                                      _dev(position_ids, "position_ids"), ctypes.byref(shape), q_base, qr, k_base, kr,
+                                      softmax_scale, _dev(o_blk, "o_blk"), _dtype_code(o_blk), _dev(lse_blk, "lse_blk"),
+                                      _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+           "ulysses_attn_fwd_block")
+
+
+def ulysses_attn_bwd_block(q_blk, k_blk, v_blk, o_blk, lse_blk, do_blk, position_ids, dq_blk, dk_blk, dv_blk, ws,
+                           q_base: int, k_base: int, softmax_scale: float = 0.0, stream=None) -> None:
+    """The key block's share of dQ and the query block's dK / dV contributions,
+    given the query block's merged O and LSE."""
+    shape, qr, kr = _check_block(q_blk, k_blk, v_blk, position_ids, o_blk, lse_blk, stream, do_blk, dq_blk, dk_blk,
+                                 dv_blk, ws)
+    _check(lib.ulysses_attn_bwd_block(_dev(q_blk, "q_blk"), _dev(k_blk, "k_blk"), _dev(v_blk, "v_blk"),
+                                      _dev(o_blk, "o_blk"), _dtype_code(o_blk), _dev(lse_blk, "lse_blk"),
+                                      _dev(do_blk, "do_blk"), _dev(position_ids, "position_ids"), ctypes.byref(shape),
+                                      q_base, qr, k_base, kr, softmax_scale, _dev(dq_blk, "dq_blk"),
+                                      _dev(dk_blk, "dk_blk"), _dev(dv_blk, "dv_blk"), _dtype_code(dq_blk),
+                                      _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)),
+           "ulysses_attn_bwd_block")
+
+
+def ulysses_accumulate(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
+    """dst += src (float32 tensors of the same shape)."""
+    _expect(src, tuple(dst.shape), _F32, "src")
+    _expect(dst, tuple(dst.shape), _F32, "dst")
+    _one_device(stream, dst=dst, src=src)
+    _check(lib.ulysses_accumulate(_dev(dst, "dst"), _dev(src, "src"), dst.numel(), _stream(stream)),
+           "ulysses_accumulate")
+
+
 def ulysses_attn_lse_merge(o_parts, lse_parts, o_head, lse, h_kv: int, stream=None) -> None:
     """Merge B partial results: o_parts float32 (B, P, b, n, h, d), lse_parts
     float32 (B, P, b, h, n) -> o_head (P, b, n, h, d), lse (P, b, h, n)."""
@@ -382,3 +467,106 @@ def ulysses_workspace_status(ws: torch.Tensor, stream=None) -> int:
     _check(lib.ulysses_workspace_status(_dev(ws, "ws"), _stream(stream), ctypes.byref(code)),
            "ulysses_workspace_status")
     return int(code.value)
+
+
+def ulysses_selftest_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Run the attention kernels' bounded-wait failure path on purpose: one
+    CTA waits on a barrier nothing arrives at, gives up after limit_ns and
+    records ULY_ERR_TIMEOUT in ws's status word (read it with
+    ulysses_workspace_status)."""
+    if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8:
+        raise TypeError("ws must be a uint8 CUDA tensor")
+    _one_device(stream, ws=ws)
+    _check(lib.ulysses_selftest_wait_timeout(_dev(ws, "ws"), ws.numel(), int(limit_ns), _stream(stream)),
+           "ulysses_selftest_wait_timeout")
+
+
+# ----------------------------------------------------------------------------- between GPUs
+def _ptr_array(ptrs):
+    arr = (ctypes.c_void_p * len(ptrs))()
+    for i, p in enumerate(ptrs):
+        arr[i] = int(p)
+    return arr
+
+
+def ulysses_seq_to_head_push(x_seq: torch.Tensor, dst_heads, dst_flags, rank: int, P: int, epoch: int,
+                             ws: torch.Tensor, stream=None) -> None:
+    """Store this rank's seq shard x_seq (b, n/P, H, d) into every rank's head
+    buffer (b, n, H/P, d), then release dst_flags[s][rank] = epoch.  dst_heads /
+    dst_flags: P device addresses (ints; peer-mapped for other GPUs), or
+    tensors on this process's device (one GPU standing in for all ranks)."""
+    b, m, H, d = x_seq.shape
+    _dev(x_seq, "x_seq")
+    _dev(ws, "ws")
+    heads = [t.data_ptr() if isinstance(t, torch.Tensor) else int(t) for t in dst_heads]
+    flags = [t.data_ptr() if isinstance(t, torch.Tensor) else int(t) for t in dst_flags]
+    for t in list(dst_heads) + list(dst_flags):
+        if isinstance(t, torch.Tensor):
+            _one_device(stream, dst=t)
+    if len(heads) != P or len(flags) != P:
+        raise ValueError("dst_heads and dst_flags need one entry per rank")
+    for t in dst_heads:
+        if isinstance(t, torch.Tensor):
+            _expect(t, (b, m * P, H // P, d), (x_seq.dtype,), "dst_heads[s]")
+    _check(lib.ulysses_seq_to_head_push(x_seq.data_ptr(), _ptr_array(heads), _ptr_array(flags), rank, b, m * P, H, d,
+                                        P, _dtype_code(x_seq), epoch, ws.data_ptr(), ws.numel() * ws.element_size(),
+                                        _stream(stream)), "ulysses_seq_to_head_push")
+
+
+def ulysses_head_to_seq_push(x_head: torch.Tensor, dst_seqs, dst_flags, rank: int, P: int, epoch: int,
+                             ws: torch.Tensor, stream=None) -> None:
+    """Store this rank's head slice x_head (b, n, H/P, d) into every rank's seq
+    shard (b, n/P, H, d), then release dst_flags[s][rank] = epoch."""
+    b, n, h, d = x_head.shape
+    _dev(x_head, "x_head")
+    _dev(ws, "ws")
+    seqs = [t.data_ptr() if isinstance(t, torch.Tensor) else int(t) for t in dst_seqs]
+    flags = [t.data_ptr() if isinstance(t, torch.Tensor) else int(t) for t in dst_flags]
+    for t in list(dst_seqs) + list(dst_flags):
+        if isinstance(t, torch.Tensor):
+            _one_device(stream, dst=t)
+    if len(seqs) != P or len(flags) != P:
+        raise ValueError("dst_seqs and dst_flags need one entry per rank")
+    for t in dst_seqs:
+        if isinstance(t, torch.Tensor):
+            _expect(t, (b, n // P, h * P, d), (x_head.dtype,), "dst_seqs[s]")
+    _check(lib.ulysses_head_to_seq_push(x_head.data_ptr(), _ptr_array(seqs), _ptr_array(flags), rank, b, n, h * P, d,
+                                        P, _dtype_code(x_head), epoch, ws.data_ptr(), ws.numel() * ws.element_size(),
+                                        _stream(stream)), "ulysses_head_to_seq_push")
+
+
+def ulysses_wait_flags(flags: torch.Tensor, epoch: int, limit_ns: int, ws: torch.Tensor, stream=None) -> None:
+    """Enqueue a bounded wait until every slot of flags (uint32 as int32) holds epoch."""
+    if flags.dtype not in (torch.int32,) or flags.dim() != 1:
+        raise TypeError("flags must be a 1-D int32 tensor (uint32 slots)")
+    _one_device(stream, flags=flags, ws=ws)
+    _check(lib.ulysses_wait_flags(flags.data_ptr(), flags.numel(), epoch, int(limit_ns), ws.data_ptr(),
+                                  _stream(stream)), "ulysses_wait_flags")
+
+
+def ulysses_release_flags(slot_addrs, epoch: int, stream=None) -> None:
+    """Store epoch into each uint32 slot (device addresses), with release
+    semantics at system scope, after everything enqueued before it."""
+    _check(lib.ulysses_release_flags(_ptr_array(slot_addrs), len(slot_addrs), epoch, _stream(stream)),
+           "ulysses_release_flags")
+
+
+def ulysses_ipc_handle(t: torch.Tensor) -> bytes:
+    """The CUDA IPC handle (64 bytes) of the allocation at t's address."""
+    buf = ctypes.create_string_buffer(64)
+    _check(lib.ulysses_ipc_handle(_dev(t, "t"), buf), "ulysses_ipc_handle")
+    return buf.raw
+
+
+def ulysses_ipc_open(handle: bytes) -> int:
+    """Open another process's allocation; returns its device address here."""
+    if len(handle) != 64:
+        raise ValueError("a CUDA IPC handle is 64 bytes")
+    p = ctypes.c_void_p()
+    _check(lib.ulysses_ipc_open(handle, ctypes.byref(p)), "ulysses_ipc_open")
+    return int(p.value)
+
+
+def ulysses_ipc_close(addr: int) -> None:
+    _check(lib.ulysses_ipc_close(ctypes.c_void_p(addr)), "ulysses_ipc_close")
+

@@ -13,11 +13,27 @@
 //   dK_j  = scale sum_{group heads} sum_i dS_ij q_i
 //   dQ_i  = scale sum_j dS_ij k_j
 //
-// Three kernels, no atomics (results are bitwise reproducible):
+// Operand precision.  The tensor-core products take fp16 copies of q, k, v
+// and dO, each scaled by a power of two chosen from its largest magnitude,
+// so that P and dS (rounded to 16 bits before they feed dV, dK and dQ) carry
+// 11 significant bits instead of bf16's 8: the bf16 rounding of P and dS
+// alone gave dV and dK errors above 1e-2 on short rows and in GQA group
+// sums.  Scaling by 2^-s is exact, so the products are the same numbers up
+// to the known factor, which the kernels fold back in:
+//   q' = q 2^-sq, k' = k 2^-sk, v' = v 2^-sv, dO' = dO 2^-sdo
+//   max|q'|, max|k'| in [2^14, 2^15); max|v'| in [4, 8); max|dO'| in [8, 16)
+// (v and dO are kept small so that dP' - D' = (dP - D) 2^-(sdo+sv) stays
+// below 2 d 8 16 <= 32768, inside fp16's range, for d <= 128).
+//  * bwd_scale: the largest magnitude of each of q, k, v, dO (rows of the
+//               selected ranks), then their fp16 copies and shifts.
+//
+// Three attention kernels, no atomics in them (results are bitwise
+// reproducible):
 //  * bwd_pre:   -LSE_i*log2(e) and -D_i per (rank, head, row), written into
 //               a padded workspace table of 64-row blocks, each holding the
 //               block's 64 values of -LSE*log2e followed by its 64 values of
-//               -D (negated so they feed packed fused multiply-adds).
+//               -D 2^-(sdo+sv) (negated so they feed packed fused
+//               multiply-adds; scaled to the units of dP' = dO' v'^T).
 //  * bwd_dkdv:  one CTA per (rank, batch row, kv head, 128-key tile),
 //               group by group, heaviest key tile first in each.  Loops over
 //               the G query heads of the kv head and the 128-row query tiles
@@ -30,7 +46,7 @@
 //               S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128: the
 //               shape runs the tensor core at full rate, N = 64 does not)
 //               go to TMEM; the softmax frees S^T as soon as it has read it,
-//               then writes P^T and dS^T as bf16 over dP^T, and they feed
+//               then writes P^T and dS^T as fp16 over dP^T, and they feed
 //               dV += P^T dO, dK += dS^T Q as A-from-TMEM MMAs accumulating
 //               in TMEM across the whole group (details at the kernel).
 //               TMEM: dK [0,128) dV [128,256) S^T [256,384) dP^T [384,512).
@@ -40,7 +56,7 @@
 //               dQ reads a K tile one step after S did, so a two-deep ring
 //               would leave no time to load the next one).  S = Q K^T into a
 //               double-buffered TMEM tile, dP = dO V^T, two softmax
-//               warpgroups (64 columns each) turn them into dS (bf16, over S)
+//               warpgroups (64 columns each) turn them into dS (fp16, over S)
 //               and dQ += dS K accumulates in TMEM.
 //               TMEM: S_0 [0,128) S_1 [128,256) dP [256,384) dQ [384,512).
 // Every kernel also takes a key range [k_lo, k_hi) (the whole sequence for
@@ -59,6 +75,78 @@ namespace bwd {
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ============================================================================
+// bwd_scale: per-tensor largest magnitude, then fp16 copies scaled by 2^-s
+// ============================================================================
+// Tensor t of {q, k, v, dO}: elements [off[t], off[t] + cnt[t]) (the rows of
+// the selected ranks; both multiples of 8).  Magnitudes are compared as the
+// bf16 bit patterns with the sign cleared, which order like the values
+// (NaN patterns sort above infinity).
+struct ScaleArgs {
+  const uint16_t* src[4];
+  uint16_t* dst[4];     // fp16 copies, same indexing as src
+  int64_t off[4], cnt[4];
+};
+// Targets: the largest magnitude after scaling lies in [2^T, 2^(T+1)).
+__host__ __device__ constexpr int scale_target(int t) { return t < 2 ? 14 : (t == 2 ? 2 : 3); }
+
+// Tensor t's fields, selected without indexing the parameter arrays at run time.
+template <typename T>
+__device__ __forceinline__ T pick(const T (&x)[4], int t) { return t == 0 ? x[0] : t == 1 ? x[1] : t == 2 ? x[2] : x[3]; }
+
+__global__ void __launch_bounds__(256) bwd_absmax_kernel(const ScaleArgs a, uint32_t* __restrict__ amax) {
+  const int t = blockIdx.y;
+  const uint4* src = reinterpret_cast<const uint4*>(pick(a.src, t) + pick(a.off, t));
+  const int64_t nvec = pick(a.cnt, t) / 8;
+  uint32_t m = 0;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec; i += int64_t(gridDim.x) * blockDim.x) {
+    const uint4 v = src[i];
+    m = __vmaxu2(m, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                             __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+  }
+  m = max(m & 0xFFFFu, m >> 16);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax + t, m);
+}
+
+// Shift s of a tensor whose largest magnitude has bf16 bits `bits`: the
+// scaled maximum 2^(ilogb(max) - s) is 2^T.  All-zero and non-finite
+// tensors keep s = 0; s is clamped so 2^-s stays a normal float.
+__device__ __forceinline__ int scale_shift(uint32_t bits, int target) {
+  if (bits == 0 || bits >= 0x7F80u) return 0;
+  const int e = int(bits >> 7);
+  const int ilog = e > 0 ? e - 127 : (31 - __clz(int(bits & 0x7Fu))) - 133;
+  const int sh = ilog - target;
+  return sh < -120 ? -120 : (sh > 120 ? 120 : sh);
+}
+
+__global__ void __launch_bounds__(256) bwd_to_f16_kernel(const ScaleArgs a, const uint32_t* __restrict__ amax,
+                                                         int32_t* __restrict__ shifts) {
+  const int t = blockIdx.y;
+  const int sh = scale_shift(amax[t], scale_target(t));
+  if (blockIdx.x == 0 && threadIdx.x == 0) shifts[t] = sh;
+  const float f = __int_as_float((127 - sh) << 23);   // 2^-sh
+  const uint4* src = reinterpret_cast<const uint4*>(pick(a.src, t) + pick(a.off, t));
+  uint4* dst = reinterpret_cast<uint4*>(pick(a.dst, t) + pick(a.off, t));
+  const int64_t nvec = pick(a.cnt, t) / 8;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec; i += int64_t(gridDim.x) * blockDim.x) {
+    const uint4 v = src[i];
+    uint4 o;
+    o.x = pack_f16x2(__uint_as_float(v.x << 16) * f, __uint_as_float(v.x & 0xFFFF0000u) * f);
+    o.y = pack_f16x2(__uint_as_float(v.y << 16) * f, __uint_as_float(v.y & 0xFFFF0000u) * f);
+    o.z = pack_f16x2(__uint_as_float(v.z << 16) * f, __uint_as_float(v.z & 0xFFFF0000u) * f);
+    o.w = pack_f16x2(__uint_as_float(v.w << 16) * f, __uint_as_float(v.w & 0xFFFF0000u) * f);
+    dst[i] = o;
+  }
+}
+
+// Shifts of q, k, v, dO as written by bwd_to_f16_kernel.
+enum { kShQ = 0, kShK = 1, kShV = 2, kShDO = 3 };
+
+// 2^e for a shift e in [-120, 120] (a normal float: built from its exponent field).
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// ============================================================================
 // bwd_pre: D = rowsum(dO * O) and LSE*log2(e), one warp per (rank, row, head)
 // ============================================================================
 // stats layout: [P*b][hq][n_pad/64] blocks of {64 x -LSE*log2e, 64 x -D}
@@ -71,8 +159,8 @@ __device__ __forceinline__ int64_t stats_index(int64_t rbh, int64_t n_pad, int64
 template <int D, bool kOF32>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const uint16_t* __restrict__ dO,
                                                       const float* __restrict__ lse, float* __restrict__ stats,
-                                                      int64_t rb0, int64_t n, int64_t n_pad, int32_t hq,
-                                                      int64_t total) {
+                                                      const int32_t* __restrict__ shifts, int64_t rb0, int64_t n,
+                                                      int64_t n_pad, int32_t hq, int64_t total) {
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= total) return;
@@ -104,7 +192,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
     stats[sidx] = -lse[(rb * hq + h) * n + i] * kLog2e;
-    stats[sidx + 64] = -acc;
+    stats[sidx + 64] = -acc * pow2i(-shifts[kShDO]) * pow2i(-shifts[kShV]);
   }
 }
 
@@ -131,10 +219,12 @@ constexpr int kRegsLo = DKDV_REGS_LO, kRegsHi = DKDV_REGS_HI;
 struct Params {
   const int32_t* segend;
   const float* stats;    // see stats_index
-  void* dk;              // [P*b][n][hkv][D]
+  const int32_t* shifts; // q, k, v, dO scale shifts (bwd_to_f16_kernel)
+  void* dk;              // [P*b][k_rows][hkv][D]
   void* dv;
   int* status;
-  int64_t n, n_pad;
+  int64_t n, n_pad;      // tokens of the whole sequence; the statistics table's rows (q_rows rounded up)
+  int64_t q_base, q_rows, k_base, k_rows;   // global rows held by the Q-side and K-side buffers
   int64_t k_lo, k_hi;    // only keys in [k_lo, k_hi) take part (one ring block); 0, n otherwise
   int32_t b, P_sel, rank0, hq, hkv, G;
   float scale, scale_log2;
@@ -168,6 +258,7 @@ struct Bars {
   uint64_t mma_final;
   uint32_t tmem_base;
   int abort_flag;
+  float score_scale;   // scale*log2(e) in the units of the fp16 copies' scores
 };
 static_assert(sizeof(Bars) <= 256, "barrier block outgrew its slot");
 
@@ -202,7 +293,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   // (rank, batch row, kv head) groups run one after another, so the CTAs
   // resident at any time share their query heads' Q / dO tiles in L2; inside
   // a group the key tiles go heaviest (first) to lightest (last)
-  const int nkt = int((p.n + BKV - 1) / BKV);
+  const int nkt = int((p.k_rows + BKV - 1) / BKV);
   const int kt = int(blockIdx.x % nkt);
   int rem = int(blockIdx.x / nkt);
   const int g = rem % p.hkv;
@@ -210,15 +301,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
   const int bb = rem % p.b;
   const int r = p.rank0 + rem / p.b;
   const int rb = r * p.b + bb;
-  const int64_t k0 = int64_t(kt) * BKV;
-  const int64_t last_key = (k0 + BKV - 1 < p.n - 1) ? (k0 + BKV - 1) : (p.n - 1);
+  const int64_t k0 = p.k_base + int64_t(kt) * BKV;   // global key rows [k0, k0 + BKV)
+  const int64_t k_end = p.k_base + p.k_rows, q_blk_end = p.q_base + p.q_rows;
+  const int64_t last_key = (k0 + BKV - 1 < k_end - 1) ? (k0 + BKV - 1) : (k_end - 1);
   const int32_t* se = p.segend + int64_t(bb) * p.n;
-  const int64_t q_end = se[last_key];      // query rows that see this key tile: [k0, q_end)
-  const int qt_first = int(k0 / BQ);
-  const int nqt = int((q_end + BQ - 1) / BQ) - qt_first;
+  // query rows that see this key tile, inside the Q block: [max(k0, q_base), q_end)
+  const int64_t q_end = se[last_key] < q_blk_end ? int64_t(se[last_key]) : q_blk_end;
+  const int qt_first = int((k0 > p.q_base ? k0 : p.q_base) / BQ);
+  const int nqt_raw = int((q_end + BQ - 1) / BQ) - qt_first;
+  const int nqt = nqt_raw > 0 ? nqt_raw : 0;
   // (query head, query tile) pairs, head-major; none when the key tile lies
   // outside [k_lo, k_hi) (its dK, dV are then zero)
-  const int niter = (k0 < p.k_hi && k0 + BKV > p.k_lo) ? nqt * p.G : 0;
+  const int niter = (k0 < p.k_hi && k0 + BKV > p.k_lo && nqt > 0) ? nqt * p.G : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -237,6 +331,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     mbar_init(&bars->ds_ready, 256);
     mbar_init(&bars->mma_final, 1);
     bars->abort_flag = 0;
+    bars->score_scale = p.scale_log2 * pow2i(p.shifts[kShQ]) * pow2i(p.shifts[kShK]);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -264,15 +359,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       if (is_q && niter > 0) {
         mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKV);
         for (int dc = 0; dc < D / 64; ++dc) {
-          tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0), rb);
-          tma_load_4d(&mv, &bars->kv_full, smem + L::oV + dc * BKV * 128, dc * 64, g, int(k0), rb);
+          tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0 - p.k_base), rb);
+          tma_load_4d(&mv, &bars->kv_full, smem + L::oV + dc * BKV * 128, dc * 64, g, int(k0 - p.k_base), rb);
         }
       }
       int issued = 0;
       for (int it = 0; it < niter; ++it) {
         const int st = it % ns, rnd = it / ns;
         const int h = g * p.G + it / nqt;
-        const int q0 = (qt_first + it % nqt) * BQ;
+        const int q0 = int((qt_first + it % nqt) * int64_t(BQ) - p.q_base);   // row in the Q-side buffers
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         if (is_q) {
           mbar_arrive_expect_tx(&full[st], L::kQ);
@@ -295,8 +390,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     }
   } else if (warp == 1) {
     {   // whole warp; the elected lane issues
-      const uint32_t id_s = idesc_bf16(BKV, BQ, false, false);
-      const uint32_t id_g = idesc_bf16(BKV, D, false, true);
+      const uint32_t id_s = idesc_f16(BKV, BQ, false, false);
+      const uint32_t id_g = idesc_f16(BKV, D, false, true);
       const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::oK), 16, 1024);
       const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::oV), 16, 1024);
       auto issue_s = [&](int it) {   // S^T = K Q^T into X
@@ -377,11 +472,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t kj = k0 + row;
     // query rows [kj, kj_end) see key kj (none for a key outside [k_lo, k_hi))
-    const int64_t kj_end = (kj < p.n && kj >= p.k_lo && kj < p.k_hi) ? int64_t(se[kj]) : kj;
-    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+    const int64_t kj_end = (kj < k_end && kj >= p.k_lo && kj < p.k_hi)
+                               ? (se[kj] < q_blk_end ? int64_t(se[kj]) : q_blk_end) : kj;
     bool ok = true;
     for (int it = 0; it < niter; ++it) {
       const int st = it % NSO;
+      // scores come out of the MMA in units of q'.k' = q.k 2^-(sq+sk); the
+      // factor is re-read from shared memory each step rather than held
+      const float sl = *reinterpret_cast<volatile float*>(&bars->score_scale);
+      const uint64_t sl2 = f2_pack(sl, sl);
       const int64_t q0 = int64_t(qt_first + it % nqt) * BQ;
       if (!mbar_wait(&bars->do_full[st], (it / NSO) & 1, abort_flag, p.status, p.limit_ns) ||
           !mbar_wait(&bars->s_full, it & 1, abort_flag, p.status, p.limit_ns)) {
@@ -421,7 +520,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           }
           pr[j] = p0;
           pr[j + 1] = p1;
-          pw[c] = pack_bf16x2(p0, p1);
+          pw[c] = pack_f16x2(p0, p1);
         }
       }
       if (!mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
@@ -460,7 +559,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
             float d0, d1;
             f2_unpack(f2_mul(f2_pack(pr[j], pr[j + 1]),
                              f2_add(f2_pack(__uint_as_float(a0), __uint_as_float(a1)), f2_pack(nd.x, nd.y))), d0, d1);
-            dw[c] = pack_bf16x2(d0, d1);
+            dw[c] = pack_f16x2(d0, d1);
           }
           tmem_st16(tY + lane_off + 64 * wg + 32 * ch + 16, dw);
         }
@@ -471,12 +570,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     }
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
-      const bool valid = kj < p.n;
-      const int64_t orow = (int64_t(rb) * p.n + kj) * p.hkv + g;
+      const bool valid = kj < k_end;
+      const int64_t orow = (int64_t(rb) * p.k_rows + (kj - p.k_base)) * p.hkv + g;
       {
         const int which = wg;   // warpgroup 0 stores dK, warpgroup 1 stores dV
         const uint32_t base = which == 0 ? tDK : tDV;
-        const float mul = which == 0 ? p.scale : 1.f;
+        // dK' = dS'^T q' = scale^-1 dK 2^-(sdo+sv+sq), dV' = P^T dO' = dV 2^-sdo
+        const float mul = which == 0 ? p.scale * pow2i(p.shifts[kShDO]) * pow2i(p.shifts[kShV]) * pow2i(p.shifts[kShQ])
+                                     : pow2i(p.shifts[kShDO]);
         void* out = which == 0 ? p.dk : p.dv;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -534,9 +635,11 @@ constexpr int kThreads = 384;
 struct Params {
   const int32_t* segstart;
   const float* stats;    // see stats_index
-  void* dq;              // [P*b][n][hq][D]
+  const int32_t* shifts; // q, k, v, dO scale shifts (bwd_to_f16_kernel)
+  void* dq;              // [P*b][q_rows][hq][D]
   int* status;
-  int64_t n, n_pad;
+  int64_t n, n_pad;      // tokens of the whole sequence; the statistics table's rows (q_rows rounded up)
+  int64_t q_base, q_rows, k_base, k_rows;   // global rows held by the Q-side and K-side buffers
   int64_t k_lo, k_hi;    // only keys in [k_lo, k_hi) take part (one ring block); 0, n otherwise
   int32_t b, P_sel, rank0, hq, G, ntiles;
   float scale, scale_log2;
@@ -590,8 +693,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
   const int bb = rem % p.b;
   const int r = p.rank0 + rem / p.b;
   const int rb = r * p.b + bb;
-  const int64_t t0 = int64_t(tile) * BM;
-  const int64_t last_row = (t0 + BM - 1 < p.n - 1) ? (t0 + BM - 1) : (p.n - 1);
+  const int64_t t0 = p.q_base + int64_t(tile) * BM;   // global rows [t0, t0 + BM)
+  const int64_t q_blk_end = p.q_base + p.q_rows;
+  const int64_t last_row = (t0 + BM - 1 < q_blk_end - 1) ? (t0 + BM - 1) : (q_blk_end - 1);
   const int32_t* ss = p.segstart + int64_t(bb) * p.n;
   const int64_t seg_lo = ss[t0];
   const int64_t seg_hi = ss[last_row];
@@ -646,8 +750,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       if (is_k) {
         mbar_arrive_expect_tx(&bars->qdo_full, 2 * L::kTile);
         for (int dc = 0; dc < D / 64; ++dc) {
-          tma_load_4d(&mq, &bars->qdo_full, smem + L::oQ + dc * BM * 128, dc * 64, h, int(t0), rb);
-          tma_load_4d(&mdo, &bars->qdo_full, smem + L::oDO + dc * BM * 128, dc * 64, h, int(t0), rb);
+          tma_load_4d(&mq, &bars->qdo_full, smem + L::oQ + dc * BM * 128, dc * 64, h, int(t0 - p.q_base), rb);
+          tma_load_4d(&mdo, &bars->qdo_full, smem + L::oDO + dc * BM * 128, dc * 64, h, int(t0 - p.q_base), rb);
         }
       }
       int issued = 0;
@@ -657,7 +761,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         mbar_arrive_expect_tx(&full[st], L::kTile);
         for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(map, &full[st], smem + base + st * L::kTile + dc * BN * 128, dc * 64, g, k0, rb);
+          tma_load_4d(map, &full[st], smem + base + st * L::kTile + dc * BN * 128, dc * 64, g, int(k0 - p.k_base), rb);
         issued = it + 1;
       }
       if (*abort_flag) {
@@ -668,8 +772,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     }
   } else if (warp == 1) {
     {   // whole warp; the elected lane issues
-      const uint32_t id_s = idesc_bf16(BM, BN, false, false);
-      const uint32_t id_q = idesc_bf16(BM, D, false, true);
+      const uint32_t id_s = idesc_f16(BM, BN, false, false);
+      const uint32_t id_q = idesc_f16(BM, D, false, true);
       const uint32_t q_addr = smem_u32(smem + L::oQ), do_addr = smem_u32(smem + L::oDO);
       bool ok = mbar_wait_warp(&bars->qdo_full, 0, abort_flag, p.status, p.limit_ns);
       tc_fence_after();
@@ -720,19 +824,20 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     const int wg = (warp - 4) >> 2;                 // column half handled by this warpgroup
     const int row = ((warp - 4) & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
-    const int64_t i = t0 + row;
-    const bool valid = i < p.n;
+    const int64_t i = t0 + row;                  // global row
+    const bool valid = i < q_blk_end;
     const int64_t s_i = valid ? ss[i] : seg_hi;
     // this row's keys: [row_lo, row_hi) = its sample's keys up to i, inside [k_lo, k_hi)
     const int64_t row_lo = s_i > p.k_lo ? s_i : p.k_lo;
     const int64_t row_hi = i + 1 < p.k_hi ? i + 1 : p.k_hi;
     float nl = 0.f, nd = 0.f;   // -LSE*log2e, -D of this row
     if (valid) {
-      const int64_t si = stats_index(int64_t(rb) * p.hq + h, p.n_pad, i);
+      const int64_t si = stats_index(int64_t(rb) * p.hq + h, p.n_pad, i - p.q_base);
       nl = p.stats[si];
       nd = p.stats[si + 64];
     }
-    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(nl, nl), nd2 = f2_pack(nd, nd);
+    const float sl = p.scale_log2 * pow2i(p.shifts[kShQ]) * pow2i(p.shifts[kShK]);   // q'.k' units, as dK/dV
+    const uint64_t sl2 = f2_pack(sl, sl), nl2 = f2_pack(nl, nl), nd2 = f2_pack(nd, nd);
     bool ok = true;
     for (int it = 0; it < nkv; ++it) {
       const int b = it & 1;
@@ -772,7 +877,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         }
         float ga, gb;
         f2_unpack(f2_mul(f2_pack(pa, pb), f2_add(f2_pack(__uint_as_float(da), __uint_as_float(db)), nd2)), ga, gb);
-        w[c] = pack_bf16x2(ga, gb);
+        w[c] = pack_f16x2(ga, gb);
       }
       tmem_st32(tS(b) + lane_off + 64 * wg, w);
       tmem_st_wait();
@@ -781,7 +886,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     }
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
-      const int64_t orow = (int64_t(rb) * p.n + i) * p.hq + h;
+      const int64_t orow = (int64_t(rb) * p.q_rows + (i - p.q_base)) * p.hq + h;
+      // dQ' = dS' k' = scale^-1 dQ 2^-(sdo+sv+sk)
+      const float mq = p.scale * pow2i(p.shifts[kShDO]) * pow2i(p.shifts[kShV]) * pow2i(p.shifts[kShK]);
       for (int c = 64 * wg; c < D; c += 128) {
         // warpgroup wg stores head-dim columns [64 wg, 64 wg + 64) (D = 64: wg 0 only)
 #pragma unroll
@@ -798,17 +905,17 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.dq) + orow * D + c + c2);
 #pragma unroll
               for (int e = 0; e < 8; ++e)
-                dst[e] = make_float4(__uint_as_float(o[4 * e]) * p.scale, __uint_as_float(o[4 * e + 1]) * p.scale,
-                                     __uint_as_float(o[4 * e + 2]) * p.scale, __uint_as_float(o[4 * e + 3]) * p.scale);
+                dst[e] = make_float4(__uint_as_float(o[4 * e]) * mq, __uint_as_float(o[4 * e + 1]) * mq,
+                                     __uint_as_float(o[4 * e + 2]) * mq, __uint_as_float(o[4 * e + 3]) * mq);
             } else {
               uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.dq) + orow * D + c + c2);
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 dst[e] = make_uint4(
-                    pack_bf16x2(__uint_as_float(o[8 * e]) * p.scale, __uint_as_float(o[8 * e + 1]) * p.scale),
-                    pack_bf16x2(__uint_as_float(o[8 * e + 2]) * p.scale, __uint_as_float(o[8 * e + 3]) * p.scale),
-                    pack_bf16x2(__uint_as_float(o[8 * e + 4]) * p.scale, __uint_as_float(o[8 * e + 5]) * p.scale),
-                    pack_bf16x2(__uint_as_float(o[8 * e + 6]) * p.scale, __uint_as_float(o[8 * e + 7]) * p.scale));
+                    pack_bf16x2(__uint_as_float(o[8 * e]) * mq, __uint_as_float(o[8 * e + 1]) * mq),
+                    pack_bf16x2(__uint_as_float(o[8 * e + 2]) * mq, __uint_as_float(o[8 * e + 3]) * mq),
+                    pack_bf16x2(__uint_as_float(o[8 * e + 4]) * mq, __uint_as_float(o[8 * e + 5]) * mq),
+                    pack_bf16x2(__uint_as_float(o[8 * e + 6]) * mq, __uint_as_float(o[8 * e + 7]) * mq));
             }
           }
         }
@@ -829,10 +936,23 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
 
 }  // namespace bwd
 
-// Backward workspace: the segment tables (as the forward), then the padded
-// row-statistics table (see stats_index; n_pad = n rounded up to 128).
+// Backward workspace:
+//   [0, 256)      status word (bytes 0-3); the four largest magnitudes as
+//                 bf16 bits (uint32, bytes 64-79) and the four shifts
+//                 (int32, bytes 96-111) of q, k, v, dO
+//   the segment tables (as the forward)
+//   the padded row-statistics table (see stats_index; n_pad = n rounded up to 128)
+//   the fp16 copies q', k', v', dO' (head layout, 256-byte aligned each)
 static int64_t bwd_n_pad(int64_t n) { return (n + 127) / 128 * 128; }
 static size_t bwd_ws_stats_off(const uly_shape* s) { return seg_workspace_bytes(s->b, s->n); }
+static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+static size_t bwd_ws_copies_off(const uly_shape* s) {
+  return bwd_ws_stats_off(s) + round256(size_t(s->b) * size_t(s->h_q) * size_t(bwd_n_pad(s->n)) * 8);
+}
+// bytes of one fp16 copy of a head-layout tensor with h heads per rank
+static size_t bwd_copy_bytes(const uly_shape* s, int64_t h) {
+  return round256(size_t(s->P) * size_t(s->b) * size_t(s->n) * size_t(h) * size_t(s->d) * 2);
+}
 
 }  // namespace uly
 
@@ -840,21 +960,27 @@ using namespace uly;
 
 extern "C" size_t ulysses_attn_bwd_workspace(const uly_shape* s, uly_dtype g_dtype) {
   if (check_shape(s) != ULY_OK || !dtype_ok(g_dtype)) return 0;
-  return bwd_ws_stats_off(s) + size_t(s->b) * size_t(s->h_q) * size_t(bwd_n_pad(s->n)) * 8;
+  const int64_t hq = s->h_q / s->P, hkv = kv_heads_per_rank(*s);
+  return bwd_ws_copies_off(s) + 2 * bwd_copy_bytes(s, hq) + 2 * bwd_copy_bytes(s, hkv);
 }
 
 // events: null, or five caller-owned cudaEvent_t recorded on the stream
-// before the segment-table, statistics, dK/dV and dQ kernels and after dQ.
+// before the segment-table kernel, before the preparation kernels (largest
+// magnitudes, fp16 copies, row statistics), before dK/dV, before dQ and
+// after dQ.
 // k_lo, k_hi: the key range taking part ([0, n) for the plain backward).
+// rows: the global rows the Q-side buffers (q, O, LSE, dO, dQ) and the K-side
+// buffers (k, v, dK, dV) hold.
 static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const void* v_head, const void* o_head,
                                 uly_dtype o_dtype, const float* lse, const void* do_head, const int64_t* position_ids,
                                 const uly_shape* shape, int32_t rank, float softmax_scale, int64_t k_lo,
-                                int64_t k_hi, void* dq_head, void* dk_head, void* dv_head, uly_dtype g_dtype,
-                                void* ws, size_t ws_bytes, void* stream, void* const* events) {
+                                int64_t k_hi, const RowBlocks& rows, void* dq_head, void* dk_head, void* dv_head,
+                                uly_dtype g_dtype, void* ws, size_t ws_bytes, void* stream, void* const* events) {
   uly_status st = validate_attn(q_head, k_head, v_head, position_ids, shape, rank, ws, ws_bytes,
                                 shape ? ulysses_attn_bwd_workspace(shape, g_dtype) : 0);
   if (st != ULY_OK) return st;
-  if (k_lo < 0 || k_hi <= k_lo || k_hi > shape->n) return ULY_ERR_INVALID_ARG;
+  if (!rows_ok(rows, shape->n, 128)) return ULY_ERR_INVALID_ARG;
+  if (k_lo < rows.k_base || k_hi <= k_lo || k_hi > rows.k_base + rows.k_rows) return ULY_ERR_INVALID_ARG;
   if (!o_head || !lse || !do_head || !dq_head || !dk_head || !dv_head) return ULY_ERR_INVALID_ARG;
   if (!dtype_ok(o_dtype) || !dtype_ok(g_dtype)) return ULY_ERR_INVALID_ARG;
   if (!aligned(o_head, 16) || !aligned(lse, 16) || !aligned(do_head, 16) || !aligned(dq_head, 16) ||
@@ -863,9 +989,10 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
   const uly_shape& s = *shape;
   const int64_t hq = s.h_q / s.P, hkv = kv_heads_per_rank(s), Pb = int64_t(s.P) * s.b;
   const size_t gsz = dtype_size(g_dtype);
-  const size_t dqb = size_t(Pb * s.n * hq * s.d) * gsz, dkb = size_t(Pb * s.n * hkv * s.d) * gsz;
-  const size_t qb = size_t(Pb * s.n * hq * s.d) * 2, kb = size_t(Pb * s.n * hkv * s.d) * 2;
-  const size_t ob = size_t(Pb * s.n * hq * s.d) * dtype_size(o_dtype), lb = size_t(Pb * hq * s.n) * 4;
+  const int64_t qr = rows.q_rows, kr = rows.k_rows;
+  const size_t dqb = size_t(Pb * qr * hq * s.d) * gsz, dkb = size_t(Pb * kr * hkv * s.d) * gsz;
+  const size_t qb = size_t(Pb * qr * hq * s.d) * 2, kb = size_t(Pb * kr * hkv * s.d) * 2;
+  const size_t ob = size_t(Pb * qr * hq * s.d) * dtype_size(o_dtype), lb = size_t(Pb * hq * qr) * 4;
   const void* ins[6] = {q_head, k_head, v_head, o_head, lse, do_head};
   const size_t insz[6] = {qb, kb, kb, ob, lb, qb};
   void* outs[3] = {dq_head, dk_head, dv_head};
@@ -877,19 +1004,28 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
       if (overlaps(outs[a], outsz[a], outs[b2], outsz[b2])) return ULY_ERR_INVALID_ARG;
     if (overlaps(outs[a], outsz[a], ws, ws_bytes)) return ULY_ERR_INVALID_ARG;
   }
-
-  CUtensorMap mk128, mv128, mq128, mdo128;
-  if (!make_head_map(&mk128, k_head, Pb, s.n, hkv, s.d, 128) || !make_head_map(&mv128, v_head, Pb, s.n, hkv, s.d, 128) ||
-      !make_head_map(&mq128, q_head, Pb, s.n, hq, s.d, 128) || !make_head_map(&mdo128, do_head, Pb, s.n, hq, s.d, 128))
-    return ULY_ERR_CUDA;
+  for (int b2 = 0; b2 < 6; ++b2)   // the workspace receives the fp16 copies of the inputs
+    if (overlaps(ins[b2], insz[b2], ws, ws_bytes)) return ULY_ERR_INVALID_ARG;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint32_t* amax = reinterpret_cast<uint32_t*>(wsb + 64);
+  int32_t* shifts = reinterpret_cast<int32_t*>(wsb + 96);
+  uint16_t* q16 = reinterpret_cast<uint16_t*>(wsb + bwd_ws_copies_off(&s));
+  uint16_t* do16 = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(q16) + bwd_copy_bytes(&s, hq));
+  uint16_t* k16 = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(do16) + bwd_copy_bytes(&s, hq));
+  uint16_t* v16 = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(k16) + bwd_copy_bytes(&s, hkv));
+
+  // the attention kernels read the fp16 copies
+  CUtensorMap mk128, mv128, mq128, mdo128;
+  if (!make_head_map(&mk128, k16, Pb, kr, hkv, s.d, 128) || !make_head_map(&mv128, v16, Pb, kr, hkv, s.d, 128) ||
+      !make_head_map(&mq128, q16, Pb, qr, hq, s.d, 128) || !make_head_map(&mdo128, do16, Pb, qr, hq, s.d, 128))
+    return ULY_ERR_CUDA;
   const size_t tab = (size_t(s.b) * size_t(s.n) * 4 + 255) & ~size_t(255);
   int32_t* segstart = reinterpret_cast<int32_t*>(wsb + 256);
   int32_t* segend = reinterpret_cast<int32_t*>(wsb + 256 + tab);
   float* stats = reinterpret_cast<float*>(wsb + bwd_ws_stats_off(&s));
-  const int64_t n_pad = bwd_n_pad(s.n);
+  const int64_t n_pad = bwd_n_pad(qr);   // statistics rows of the Q-side block
 
   auto mark = [&](int i) { return !events || cudaEventRecord(static_cast<cudaEvent_t>(events[i]), cs) == cudaSuccess; };
   if (!mark(0)) return ULY_ERR_CUDA;
@@ -901,6 +1037,29 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
   const int64_t rank0 = rank < 0 ? 0 : rank;
   const int64_t rb0 = rank0 * s.b, nrb = P_sel * s.b;
   {
+    // fp16 copies of the selected ranks' rows, each scaled by its own power of two
+    bwd::ScaleArgs a;
+    const void* srcs[4] = {q_head, k_head, v_head, do_head};
+    uint16_t* dsts[4] = {q16, k16, v16, do16};
+    const int64_t heads[4] = {hq, hkv, hkv, hq};
+    const int64_t nrows[4] = {qr, kr, kr, qr};
+    int64_t most = 0;
+    for (int t = 0; t < 4; ++t) {
+      a.src[t] = static_cast<const uint16_t*>(srcs[t]);
+      a.dst[t] = dsts[t];
+      a.off[t] = rb0 * nrows[t] * heads[t] * s.d;
+      a.cnt[t] = nrb * nrows[t] * heads[t] * s.d;
+      most = a.cnt[t] > most ? a.cnt[t] : most;
+    }
+    // a few waves of 256-thread blocks per tensor; each thread strides over 16-byte vectors
+    const int64_t want = (most / 8 + 255) / 256;
+    const unsigned gx = unsigned(want < 4 * 148 ? (want > 0 ? want : 1) : 4 * 148);
+    if (cudaMemsetAsync(amax, 0, 4 * sizeof(uint32_t), cs) != cudaSuccess) return ULY_ERR_CUDA;
+    bwd::bwd_absmax_kernel<<<dim3(gx, 4), 256, 0, cs>>>(a, amax);
+    bwd::bwd_to_f16_kernel<<<dim3(gx, 4), 256, 0, cs>>>(a, amax, shifts);
+    if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
+  }
+  {
     const int64_t total = nrb * n_pad * hq;
     const int64_t blocks = (total * 32 + 255) / 256;
     if (blocks > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
@@ -908,11 +1067,11 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     const uint16_t* dop = static_cast<const uint16_t*>(do_head);
     const unsigned nb = unsigned(blocks);
     if (s.d == 128) {
-      if (of32) bwd::bwd_pre_kernel<128, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
-      else bwd::bwd_pre_kernel<128, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
+      if (of32) bwd::bwd_pre_kernel<128, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
+      else bwd::bwd_pre_kernel<128, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
     } else {
-      if (of32) bwd::bwd_pre_kernel<64, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
-      else bwd::bwd_pre_kernel<64, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, rb0, s.n, n_pad, int32_t(hq), total);
+      if (of32) bwd::bwd_pre_kernel<64, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
+      else bwd::bwd_pre_kernel<64, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
     }
     if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
@@ -924,11 +1083,16 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     bwd::dkdv::Params p;
     p.segend = segend;
     p.stats = stats;
+    p.shifts = shifts;
     p.dk = dk_head;
     p.dv = dv_head;
     p.status = reinterpret_cast<int*>(wsb);
     p.n = s.n;
     p.n_pad = n_pad;
+    p.q_base = rows.q_base;
+    p.q_rows = qr;
+    p.k_base = rows.k_base;
+    p.k_rows = kr;
     p.k_lo = k_lo;
     p.k_hi = k_hi;
     p.b = int32_t(s.b);
@@ -941,7 +1105,7 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.scale_log2 = scale * bwd::kLog2e;
     p.g_f32 = g_dtype == ULY_F32;
     p.limit_ns = 2000000000ull;
-    const int64_t grid = (s.n + bwd::dkdv::BKV - 1) / bwd::dkdv::BKV * P_sel * s.b * hkv;
+    const int64_t grid = (kr + bwd::dkdv::BKV - 1) / bwd::dkdv::BKV * P_sel * s.b * hkv;
     if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
     if (s.d == 128) {
       auto kern = bwd::dkdv::attn_bwd_dkdv_kernel<128>;
@@ -962,10 +1126,15 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     bwd::dq::Params p;
     p.segstart = segstart;
     p.stats = stats;
+    p.shifts = shifts;
     p.dq = dq_head;
     p.status = reinterpret_cast<int*>(wsb);
     p.n = s.n;
     p.n_pad = n_pad;
+    p.q_base = rows.q_base;
+    p.q_rows = qr;
+    p.k_base = rows.k_base;
+    p.k_rows = kr;
     p.k_lo = k_lo;
     p.k_hi = k_hi;
     p.b = int32_t(s.b);
@@ -973,7 +1142,7 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.rank0 = int32_t(rank0);
     p.hq = int32_t(hq);
     p.G = int32_t(group_per_rank(s));
-    p.ntiles = int32_t((s.n + bwd::dq::BM - 1) / bwd::dq::BM);
+    p.ntiles = int32_t((qr + bwd::dq::BM - 1) / bwd::dq::BM);
     p.scale = scale;
     p.scale_log2 = scale * bwd::kLog2e;
     p.g_f32 = g_dtype == ULY_F32;
@@ -1004,7 +1173,8 @@ extern "C" uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, c
                                        uly_dtype g_dtype, void* ws, size_t ws_bytes, void* stream) {
   if (check_shape(shape) != ULY_OK) return check_shape(shape);
   return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
-                       softmax_scale, 0, shape->n, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, nullptr);
+                       softmax_scale, 0, shape->n, whole_rows(shape->n), dq_head, dk_head, dv_head, g_dtype, ws,
+                       ws_bytes, stream, nullptr);
 }
 
 extern "C" uly_status ulysses_attn_bwd_kv_range(const void* q_head, const void* k_head, const void* v_head,
@@ -1016,7 +1186,21 @@ extern "C" uly_status ulysses_attn_bwd_kv_range(const void* q_head, const void* 
                                                 void* stream) {
   if (check_shape(shape) != ULY_OK) return check_shape(shape);
   return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
-                       softmax_scale, k_lo, k_hi, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, nullptr);
+                       softmax_scale, k_lo, k_hi, whole_rows(shape->n), dq_head, dk_head, dv_head, g_dtype, ws,
+                       ws_bytes, stream, nullptr);
+}
+
+extern "C" uly_status ulysses_attn_bwd_block(const void* q_blk, const void* k_blk, const void* v_blk,
+                                             const void* o_blk, uly_dtype o_dtype, const float* lse_blk,
+                                             const void* do_blk, const int64_t* position_ids, const uly_shape* shape,
+                                             int64_t q_base, int64_t q_rows, int64_t k_base, int64_t k_rows,
+                                             float softmax_scale, void* dq_blk, void* dk_blk, void* dv_blk,
+                                             uly_dtype g_dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (check_shape(shape) != ULY_OK) return check_shape(shape);
+  const RowBlocks rows{q_base, q_rows, k_base, k_rows};
+  if (!rows_ok(rows, shape->n, 128)) return ULY_ERR_INVALID_ARG;
+  return attn_bwd_impl(q_blk, k_blk, v_blk, o_blk, o_dtype, lse_blk, do_blk, position_ids, shape, -1, softmax_scale,
+                       k_base, k_base + k_rows, rows, dq_blk, dk_blk, dv_blk, g_dtype, ws, ws_bytes, stream, nullptr);
 }
 
 extern "C" uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_head, const void* v_head,
@@ -1030,5 +1214,6 @@ extern "C" uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_h
     if (!events[i]) return ULY_ERR_INVALID_ARG;
   if (check_shape(shape) != ULY_OK) return check_shape(shape);
   return attn_bwd_impl(q_head, k_head, v_head, o_head, o_dtype, lse, do_head, position_ids, shape, rank,
-                       softmax_scale, 0, shape->n, dq_head, dk_head, dv_head, g_dtype, ws, ws_bytes, stream, events);
+                       softmax_scale, 0, shape->n, whole_rows(shape->n), dq_head, dk_head, dv_head, g_dtype, ws,
+                       ws_bytes, stream, events);
 }

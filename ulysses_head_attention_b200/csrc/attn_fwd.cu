@@ -57,10 +57,12 @@ constexpr int kMufuPairs = FWD_MUFU_PAIRS;  // of the 64 column pairs per row, t
 
 struct Params {
   const int32_t* segstart;   // [b][n]
-  float* lse;                // [P][b][hq][n]
-  void* o;                   // [P][b][n][hq][D]
+  float* lse;                // [P][b][hq][q_rows]
+  void* o;                   // [P][b][q_rows][hq][D]
   int* status;
-  int64_t n;
+  int64_t n;                 // tokens of the whole sequence (the segment tables')
+  int64_t q_base, q_rows;    // Q, O, LSE hold the global rows [q_base, q_base + q_rows); 0, n for whole tensors
+  int64_t k_base;            // K, V hold the global keys from k_base on (a multiple of BN); 0 for whole tensors
   int64_t k_lo, k_hi;        // keys outside [k_lo, k_hi) are not attended (one ring block); 0, n otherwise
   int32_t b, P_sel, rank0, hq, G, ntiles, npairs;
   float scale_log2;
@@ -98,14 +100,15 @@ struct TileRange {
 };
 
 // Key tiles are also clipped to [k_lo, k_hi); first > last means the query
-// tile sees no key there (0 <= k_lo < k_hi <= n).
-__device__ __forceinline__ TileRange tile_range(const int32_t* ss, int64_t n, int tile, int ntiles, int64_t k_lo,
-                                                int64_t k_hi) {
+// tile sees no key there (0 <= k_lo < k_hi <= n).  `tile` counts query tiles
+// from q_base (a multiple of BM); rows end at q_end.
+__device__ __forceinline__ TileRange tile_range(const int32_t* ss, int64_t q_base, int64_t q_end, int tile, int ntiles,
+                                                int64_t k_lo, int64_t k_hi) {
   TileRange tr;
   tr.valid = tile < ntiles;
   const int tl = tr.valid ? tile : ntiles - 1;
-  tr.t0 = int64_t(tl) * BM;
-  const int64_t last_row = (tr.t0 + BM - 1 < n - 1) ? (tr.t0 + BM - 1) : (n - 1);
+  tr.t0 = q_base + int64_t(tl) * BM;
+  const int64_t last_row = (tr.t0 + BM - 1 < q_end - 1) ? (tr.t0 + BM - 1) : (q_end - 1);
   const int64_t key_lo = int64_t(ss[tr.t0]) > k_lo ? int64_t(ss[tr.t0]) : k_lo;
   const int64_t key_hi = last_row < k_hi - 1 ? last_row : k_hi - 1;   // last key, inclusive
   tr.first = int(key_lo / BN);
@@ -141,8 +144,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   const int r = p.rank0 + rem / p.b;
   const int rb = r * p.b + bb;
   const int32_t* ss = p.segstart + int64_t(bb) * p.n;
-  const TileRange tr0 = tile_range(ss, p.n, 2 * pair, p.ntiles, p.k_lo, p.k_hi);
-  const TileRange tr1 = tile_range(ss, p.n, 2 * pair + 1, p.ntiles, p.k_lo, p.k_hi);
+  const int64_t q_end = p.q_base + p.q_rows;
+  const TileRange tr0 = tile_range(ss, p.q_base, q_end, 2 * pair, p.ntiles, p.k_lo, p.k_hi);
+  const TileRange tr1 = tile_range(ss, p.q_base, q_end, 2 * pair + 1, p.ntiles, p.k_lo, p.k_hi);
   const bool has0 = tr0.valid && tr0.last >= tr0.first, has1 = tr1.valid && tr1.last >= tr1.first;
   // key tiles of the pair: tile 1 starts no earlier and ends no earlier than tile 0
   const int j_lo = has0 ? tr0.first : (has1 ? tr1.first : 0);
@@ -190,7 +194,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         for (int q = 0; q < (tr1.valid ? 2 : 1); ++q)
           for (int dc = 0; dc < D / 64; ++dc)
             tma_load_4d(&mq, &bars->q_full, smem + L::kQ + q * L::kTileBytes + dc * BM * 128, dc * 64, j,
-                        int((q ? tr1 : tr0).t0), rb);
+                        int((q ? tr1 : tr0).t0 - p.q_base), rb);
       }
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
@@ -199,7 +203,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         mbar_arrive_expect_tx(&full[st], L::kTileBytes);
         for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(map, &full[st], smem + base + st * L::kTileBytes + dc * BN * 128, dc * 64, g, k0, rb);
+          tma_load_4d(map, &full[st], smem + base + st * L::kTileBytes + dc * BN * 128, dc * 64, g,
+                      int(k0 - p.k_base), rb);
         issued = it + 1;
       }
       // Error path only: let every copy this thread started land before exit.
@@ -274,8 +279,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     const uint32_t tS = tmem + 128u * q, tO = tmem + 256u + 128u * q;
     const int row = ((warp - 4) & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
-    const int64_t i = tr.t0 + row;
-    const bool valid = tr.valid && i < p.n;
+    const int64_t i = tr.t0 + row;                 // global row
+    const bool valid = tr.valid && i < q_end;
+    const int64_t il = i - p.q_base;               // row in the Q / O / LSE buffers
     const int64_t s_i = valid ? ss[i] : tr.seg_hi;
     // this row's keys: [row_lo, row_hi) = its sample's keys up to i, inside [k_lo, k_hi)
     const int64_t row_lo = s_i > p.k_lo ? s_i : p.k_lo;
@@ -387,7 +393,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     if (ntile > 0 && mbar_wait(&bars->o_final[q], 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
       const float inv_l = row_vis ? 1.f / l : 0.f;   // a row that saw no key gets O = 0
-      const int64_t orow = (int64_t(rb) * p.n + i) * p.hq + j;
+      const int64_t orow = (int64_t(rb) * p.q_rows + il) * p.hq + j;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
@@ -415,10 +421,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         }
       }
       if (valid)
-        p.lse[(int64_t(rb) * p.hq + j) * p.n + i] = row_vis ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        p.lse[(int64_t(rb) * p.hq + j) * p.q_rows + il] = row_vis ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
     } else if (ntile == 0 && valid) {
       // no key of [k_lo, k_hi) is visible to this query tile: O = 0, LSE = -inf
-      const int64_t orow = (int64_t(rb) * p.n + i) * p.hq + j;
+      const int64_t orow = (int64_t(rb) * p.q_rows + il) * p.hq + j;
       if (p.o_f32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D);
         for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -426,7 +432,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D);
         for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
       }
-      p.lse[(int64_t(rb) * p.hq + j) * p.n + i] = -INFINITY;
+      p.lse[(int64_t(rb) * p.hq + j) * p.q_rows + il] = -INFINITY;
     }
   }
 
@@ -486,27 +492,31 @@ extern "C" size_t ulysses_attn_fwd_workspace(const uly_shape* s) {
   return seg_workspace_bytes(s->b, s->n);
 }
 
-// k_lo, k_hi: the key range attended ([0, n) for the plain forward).
+// k_lo, k_hi: the key range attended ([0, n) for the plain forward).  rows:
+// the global rows the Q / O / LSE buffers and the K / V buffers hold (the
+// whole sequence for the head-layout calls, one block for the block calls).
 static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const void* v_head,
                                 const int64_t* position_ids, const uly_shape* shape, int32_t rank,
-                                float softmax_scale, int64_t k_lo, int64_t k_hi, void* o_head, uly_dtype o_dtype,
-                                float* lse, void* ws, size_t ws_bytes, void* stream) {
+                                float softmax_scale, int64_t k_lo, int64_t k_hi, const RowBlocks& rows,
+                                void* o_head, uly_dtype o_dtype, float* lse, void* ws, size_t ws_bytes, void* stream) {
   uly_status st = validate_attn(q_head, k_head, v_head, position_ids, shape, rank, ws, ws_bytes,
                                 shape ? ulysses_attn_fwd_workspace(shape) : 0);
   if (st != ULY_OK) return st;
-  if (k_lo < 0 || k_hi <= k_lo || k_hi > shape->n) return ULY_ERR_INVALID_ARG;
+  if (!rows_ok(rows, shape->n, fwd::BM)) return ULY_ERR_INVALID_ARG;
+  if (k_lo < rows.k_base || k_hi <= k_lo || k_hi > rows.k_base + rows.k_rows) return ULY_ERR_INVALID_ARG;
   if (!o_head || !lse || !dtype_ok(o_dtype)) return ULY_ERR_INVALID_ARG;
   if (!aligned(o_head, 16) || !aligned(lse, 16)) return ULY_ERR_INVALID_ARG;
   const uly_shape& s = *shape;
   const int64_t hq = s.h_q / s.P, hkv = kv_heads_per_rank(s), Pb = int64_t(s.P) * s.b;
-  const int64_t ntiles = (s.n + fwd::BM - 1) / fwd::BM;
+  const int64_t ntiles = (rows.q_rows + fwd::BM - 1) / fwd::BM;
   const int64_t npairs = (ntiles + 1) / 2;
   const int64_t P_sel = rank < 0 ? s.P : 1;
   const int64_t grid = npairs * P_sel * s.b * hq;
   if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
   // Outputs must not overlap inputs.
-  const size_t qbytes = size_t(Pb * s.n * hq * s.d) * 2, kvbytes = size_t(Pb * s.n * hkv * s.d) * 2;
-  const size_t obytes = size_t(Pb * s.n * hq * s.d) * dtype_size(o_dtype), lbytes = size_t(Pb * hq * s.n) * 4;
+  const size_t qbytes = size_t(Pb * rows.q_rows * hq * s.d) * 2, kvbytes = size_t(Pb * rows.k_rows * hkv * s.d) * 2;
+  const size_t obytes = size_t(Pb * rows.q_rows * hq * s.d) * dtype_size(o_dtype);
+  const size_t lbytes = size_t(Pb * hq * rows.q_rows) * 4;
   if (overlaps(o_head, obytes, q_head, qbytes) || overlaps(o_head, obytes, k_head, kvbytes) ||
       overlaps(o_head, obytes, v_head, kvbytes) || overlaps(o_head, obytes, lse, lbytes) ||
       overlaps(lse, lbytes, q_head, qbytes) || overlaps(lse, lbytes, ws, ws_bytes) ||
@@ -514,8 +524,9 @@ static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const vo
     return ULY_ERR_INVALID_ARG;
 
   CUtensorMap mq, mk, mv;
-  if (!make_head_map(&mq, q_head, Pb, s.n, hq, s.d, fwd::BM) || !make_head_map(&mk, k_head, Pb, s.n, hkv, s.d, fwd::BN) ||
-      !make_head_map(&mv, v_head, Pb, s.n, hkv, s.d, fwd::BN))
+  if (!make_head_map(&mq, q_head, Pb, rows.q_rows, hq, s.d, fwd::BM) ||
+      !make_head_map(&mk, k_head, Pb, rows.k_rows, hkv, s.d, fwd::BN) ||
+      !make_head_map(&mv, v_head, Pb, rows.k_rows, hkv, s.d, fwd::BN))
     return ULY_ERR_CUDA;
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -531,6 +542,9 @@ static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const vo
   p.o = o_head;
   p.status = reinterpret_cast<int*>(wsb);
   p.n = s.n;
+  p.q_base = rows.q_base;
+  p.q_rows = rows.q_rows;
+  p.k_base = rows.k_base;
   p.k_lo = k_lo;
   p.k_hi = k_hi;
   p.b = int32_t(s.b);
@@ -553,8 +567,8 @@ extern "C" uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, c
                                        float softmax_scale, void* o_head, uly_dtype o_dtype, float* lse, void* ws,
                                        size_t ws_bytes, void* stream) {
   if (check_shape(shape) != ULY_OK) return check_shape(shape);
-  return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, 0, shape->n, o_head,
-                       o_dtype, lse, ws, ws_bytes, stream);
+  return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, 0, shape->n,
+                       whole_rows(shape->n), o_head, o_dtype, lse, ws, ws_bytes, stream);
 }
 
 extern "C" uly_status ulysses_attn_fwd_kv_range(const void* q_head, const void* k_head, const void* v_head,
@@ -563,8 +577,20 @@ extern "C" uly_status ulysses_attn_fwd_kv_range(const void* q_head, const void* 
                                                 uly_dtype o_dtype, float* lse, void* ws, size_t ws_bytes,
                                                 void* stream) {
   if (check_shape(shape) != ULY_OK) return check_shape(shape);
-  return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, k_lo, k_hi, o_head,
-                       o_dtype, lse, ws, ws_bytes, stream);
+  return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, k_lo, k_hi,
+                       whole_rows(shape->n), o_head, o_dtype, lse, ws, ws_bytes, stream);
+}
+
+extern "C" uly_status ulysses_attn_fwd_block(const void* q_blk, const void* k_blk, const void* v_blk,
+                                             const int64_t* position_ids, const uly_shape* shape, int64_t q_base,
+                                             int64_t q_rows, int64_t k_base, int64_t k_rows, float softmax_scale,
+                                             void* o_blk, uly_dtype o_dtype, float* lse_blk, void* ws,
+                                             size_t ws_bytes, void* stream) {
+  if (check_shape(shape) != ULY_OK) return check_shape(shape);
+  const RowBlocks rows{q_base, q_rows, k_base, k_rows};
+  if (!rows_ok(rows, shape->n, fwd::BM)) return ULY_ERR_INVALID_ARG;
+  return attn_fwd_impl(q_blk, k_blk, v_blk, position_ids, shape, -1, softmax_scale, k_base, k_base + k_rows, rows,
+                       o_blk, o_dtype, lse_blk, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -56,6 +56,20 @@ inline int64_t group_per_rank(const uly_shape& s) { return (s.h_q / s.P) / kv_he
 
 inline uly_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA; }
 
+// The global sequence rows the attention buffers hold: Q (and O, LSE, dO,
+// dQ) rows [q_base, q_base + q_rows), K (and V, dK, dV) rows
+// [k_base, k_base + k_rows).  The head-layout calls pass the whole sequence;
+// the block calls (ring attention) one block of queries and one of keys.
+struct RowBlocks {
+  int64_t q_base, q_rows, k_base, k_rows;
+};
+inline RowBlocks whole_rows(int64_t n) { return RowBlocks{0, n, 0, n}; }
+// Blocks inside [0, n), starting on tile boundaries (multiples of `tile`).
+inline bool rows_ok(const RowBlocks& r, int64_t n, int64_t tile) {
+  return r.q_base >= 0 && r.q_rows >= 1 && r.q_base + r.q_rows <= n && r.q_base % tile == 0 && r.k_base >= 0 &&
+         r.k_rows >= 1 && r.k_base + r.k_rows <= n && r.k_base % tile == 0;
+}
+
 typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                       CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,

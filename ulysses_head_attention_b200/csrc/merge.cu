@@ -115,3 +115,40 @@ extern "C" uly_status ulysses_attn_lse_merge(const float* o_parts, const float* 
             : launch_merge<64, false>(o_parts, lse_parts, nparts, rows, s.n, h, o_head, lse, cs);
   return cuda_status(e);
 }
+
+// ---------------------------------------------------------------------------
+// ulysses_accumulate: dst += src over float32 elements (the ring passes' sums
+// of per-block dQ shares and of the dK / dV that travel with a key block).
+// 16-byte vectors, grid-stride; HBM-bound (two reads, one write per element).
+// ---------------------------------------------------------------------------
+namespace uly {
+namespace {
+
+__global__ void __launch_bounds__(256) accumulate_kernel(float4* __restrict__ dst, const float4* __restrict__ src,
+                                                         int64_t nvec) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec; i += int64_t(gridDim.x) * blockDim.x) {
+    float4 a = dst[i];
+    const float4 b = src[i];
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    dst[i] = a;
+  }
+}
+
+}  // namespace
+}  // namespace uly
+
+extern "C" uly_status ulysses_accumulate(float* dst, const float* src, int64_t count, void* stream) {
+  using namespace uly;
+  if (!dst || !src || count < 1 || count % 4 || !aligned(dst, 16) || !aligned(src, 16)) return ULY_ERR_INVALID_ARG;
+  if (overlaps(dst, size_t(count) * 4, src, size_t(count) * 4) && dst != src) return ULY_ERR_INVALID_ARG;
+  const int64_t nvec = count / 4;
+  const int64_t want = (nvec + 255) / 256;
+  const unsigned grid = unsigned(want < 8 * 148 ? want : 8 * 148);
+  accumulate_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<float4*>(dst),
+                                                                          reinterpret_cast<const float4*>(src), nvec);
+  return cuda_status(cudaGetLastError());
+}
+
