@@ -70,7 +70,8 @@ typedef enum {
   ULY_ERR_UNSUPPORTED = 2,
   ULY_ERR_CUDA = 3,
   ULY_ERR_WORKSPACE = 4,
-  ULY_ERR_TIMEOUT = 5
+  ULY_ERR_TIMEOUT = 5,
+  ULY_ERR_BOUNDS = 6   /* bounds-checked debug build only: an index fell outside its buffer */
 } uly_status;
 
 typedef enum { ULY_BF16 = 0, ULY_F32 = 1 } uly_dtype;
@@ -370,11 +371,25 @@ uly_status ulysses_sp_loss_aggregate(const float* losses, const int64_t* shift_l
  * ulysses_workspace_status -- synchronizes `stream`, then reads and clears
  * the status word kept at the start of an attention workspace.  *code gets
  * ULY_OK, ULY_ERR_TIMEOUT when a kernel gave up waiting on one of its own
- * pipeline stages, or ULY_ERR_CUDA when a kernel found its dynamic shared
- * memory too poorly aligned to lay out its tiles and did nothing (in both
- * error cases the outputs are invalid).
+ * pipeline stages, ULY_ERR_CUDA when a kernel found its dynamic shared
+ * memory too poorly aligned to lay out its tiles and did nothing, or (in
+ * the bounds-checked debug build) ULY_ERR_BOUNDS when an index or a tile
+ * coordinate fell outside its buffer and the access was skipped (in every
+ * error case the outputs are invalid).
  */
 uly_status ulysses_workspace_status(void* ws, void* stream, int32_t* code);
+
+/*
+ * ulysses_debug_status -- the bounds-checked debug build (libulysses_debug.so,
+ * compiled with ULY_DEBUG_BOUNDS) checks every global index and TMA tile
+ * coordinate of its kernels before the access, records one that falls
+ * outside its buffer and skips it.  The attention kernels record into their
+ * workspace status word; the re-layout kernels, which take no workspace,
+ * into a word of the library's own, which this call synchronizes `stream`,
+ * reads and clears: *code = ULY_OK or ULY_ERR_BOUNDS.  The release build
+ * compiles no checks: it sets *code = ULY_OK and returns ULY_ERR_UNSUPPORTED.
+ */
+uly_status ulysses_debug_status(void* stream, int32_t* code);
 
 /*
  * Between GPUs: the two all-to-alls fused with the re-layout

@@ -45,3 +45,14 @@ def pytest_terminal_summary(terminalreporter):
     for what, ma, mr, bma, bmr in recs:
         rel = "" if mr != mr else f"  mean-rel {mr:.2e} (<= {bmr:g})"
         tr.write_line(f"{what}: max-abs {ma:.2e} (<= {bma:g}){rel}")
+
+
+@pytest.fixture(autouse=True)
+def _debug_build_bounds_record(request):
+    """Under the bounds-checked debug build (ULYSSES_DEBUG=1), every GPU test
+    must also leave the re-layout kernels' bounds record clean."""
+    yield
+    mod = sys.modules.get("ulysses_head_attention_b200")
+    if mod is None or not getattr(mod, "DEBUG_BUILD", False) or request.node.get_closest_marker("gpu") is None:
+        return
+    assert mod.ulysses_debug_status() == 0, "an index fell outside its buffer (debug build)"

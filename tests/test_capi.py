@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     import ulysses_head_attention_b200 as uly
-    for code in range(6):
+    for code in range(7):
         assert uly.status_string(code) and uly.status_string(code) != "unknown status"
     assert uly.status_string(99) == "unknown status"
 
@@ -358,4 +358,22 @@ def test_push_and_wait_reject():
     assert uly.lib.ulysses_ipc_handle(None, None) == INVALID
     assert uly.lib.ulysses_ipc_open(None, None) == INVALID
     assert uly.lib.ulysses_ipc_close(None) == INVALID
+
+
+def test_release_build_has_no_bounds_checks():
+    import ulysses_head_attention_b200 as uly
+    code = ctypes.c_int32(-1)
+    if uly.DEBUG_BUILD:
+        pytest.skip("the debug build is loaded")
+    assert uly.lib.ulysses_debug_status(None, ctypes.byref(code)) == UNSUPPORTED and code.value == 0
+
+
+def test_debug_build_exports_the_same_symbols():
+    """libulysses_debug.so (built with ULY_DEBUG_BOUNDS) loads and exports what the header declares."""
+    lib = os.path.join(ROOT, "ulysses_head_attention_b200", "libulysses_debug.so")
+    if not os.path.exists(lib):
+        pytest.fail("libulysses_debug.so is missing: build it with `python ulysses_head_attention_b200/build.py --debug`")
+    d = ctypes.CDLL(lib)
+    for n in header_functions():
+        assert hasattr(d, n), n
 

@@ -22,11 +22,14 @@ from typing import Optional
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libulysses.so")
+# ULYSSES_DEBUG=1 loads the bounds-checked build (every global index and TMA
+# tile coordinate checked; see ulysses_debug_status) instead of the release one.
+DEBUG_BUILD = os.environ.get("ULYSSES_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(HERE, "libulysses_debug.so" if DEBUG_BUILD else "libulysses.so")
 
 ULY_BF16, ULY_F32 = 0, 1
 STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED", 3: "ULY_ERR_CUDA",
-                4: "ULY_ERR_WORKSPACE", 5: "ULY_ERR_TIMEOUT"}
+                4: "ULY_ERR_WORKSPACE", 5: "ULY_ERR_TIMEOUT", 6: "ULY_ERR_BOUNDS"}
 # Every symbol include/ulysses.h declares.
 EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head", "ulysses_kv_head_to_seq",
            "ulysses_transpose_runs", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
@@ -36,7 +39,7 @@ EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head
            "ulysses_seq_to_head_push", "ulysses_head_to_seq_push", "ulysses_wait_flags", "ulysses_release_flags",
            "ulysses_ipc_handle",
            "ulysses_ipc_open", "ulysses_ipc_close", "ulysses_attn_fwd_block", "ulysses_attn_bwd_block",
-           "ulysses_accumulate", "ulysses_status_string")
+           "ulysses_accumulate", "ulysses_debug_status", "ulysses_status_string")
 
 
 class UlyShape(ctypes.Structure):
@@ -89,6 +92,7 @@ def _load() -> ctypes.CDLL:
         "ulysses_attn_bwd_block": ([vp, vp, vp, vp, i32, vp, vp, vp, shp, i64, i64, i64, i64, f32, vp, vp, vp, i32,
                                     vp, sz, vp], i32),
         "ulysses_accumulate": ([vp, vp, i64, vp], i32),
+        "ulysses_debug_status": ([vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "ulysses_status_string": ([i32], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -459,6 +463,15 @@ def ulysses_attn_lse_merge(o_parts, lse_parts, o_head, lse, h_kv: int, stream=No
     _check(lib.ulysses_attn_lse_merge(_dev(o_parts, "o_parts"), _dev(lse_parts, "lse_parts"), B,
                                       ctypes.byref(shape), _dev(o_head, "o_head"), _dtype_code(o_head),
                                       _dev(lse, "lse"), _stream(stream)), "ulysses_attn_lse_merge")
+
+
+def ulysses_debug_status(stream=None) -> int:
+    """Debug build: synchronize, then read and clear the re-layout kernels'
+    bounds record (0 = no index outside its buffer, 6 = ULY_ERR_BOUNDS).
+    The release build has no checks and raises UlyssesError(ULY_ERR_UNSUPPORTED)."""
+    code = ctypes.c_int32(-1)
+    _check(lib.ulysses_debug_status(_stream(stream), ctypes.byref(code)), "ulysses_debug_status")
+    return int(code.value)
 
 
 def ulysses_workspace_status(ws: torch.Tensor, stream=None) -> int:

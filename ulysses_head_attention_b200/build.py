@@ -1,6 +1,8 @@
-"""Build libulysses.so (all CUDA sources under csrc/) for sm_100a, in-tree.
+"""Build libulysses.so (all CUDA sources under csrc/) for sm_100a, in-tree,
+and its bounds-checked debug twin libulysses_debug.so (ULY_DEBUG_BOUNDS:
+every global index and TMA tile coordinate checked before the access).
 
-    python ulysses_head_attention_b200/build.py [--force]
+    python ulysses_head_attention_b200/build.py [--force] [--debug]
 
 (Run by path: importing the package itself loads the library, which may be
 missing or stale before a build.)
@@ -22,7 +24,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libulysses.so")
+LIB_DEBUG = os.path.join(HERE, "libulysses_debug.so")
 OBJ_DIR = os.path.join(ROOT, "_build", "obj")
+OBJ_DIR_DEBUG = os.path.join(ROOT, "_build", "obj_debug")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
@@ -43,22 +47,24 @@ def _deps():
     return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "ulysses.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OBJ_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib, obj_dir = (LIB_DEBUG, OBJ_DIR_DEBUG) if debug else (LIB, OBJ_DIR)
+    extra = ["-DULY_DEBUG_BOUNDS"] if debug else []
+    if not force and up_to_date(lib):
+        return lib
+    os.makedirs(obj_dir, exist_ok=True)
     cc = nvcc()
 
     def compile_one(src):
-        obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
-        cmd = [cc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
+        cmd = [cc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
@@ -68,14 +74,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-lrt", "-lpthread", "-ldl"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    force, verbose = "--force" in sys.argv, "-v" in sys.argv
+    print(build(force=force, verbose=verbose))
+    if "--debug" in sys.argv:
+        print(build(force=force, verbose=verbose, debug=True))

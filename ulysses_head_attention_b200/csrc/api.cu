@@ -47,6 +47,7 @@ extern "C" const char* ulysses_status_string(uly_status s) {
     case ULY_ERR_CUDA: return "CUDA error";
     case ULY_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
     case ULY_ERR_TIMEOUT: return "a kernel gave up waiting on its own pipeline";
+    case ULY_ERR_BOUNDS: return "debug build: an index fell outside its buffer";
   }
   return "unknown status";
 }
@@ -59,6 +60,9 @@ extern "C" uly_status ulysses_workspace_status(void* ws, void* stream, int32_t* 
   if (cudaStreamSynchronize(s) != cudaSuccess) return ULY_ERR_CUDA;
   if (cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return ULY_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return ULY_ERR_CUDA;
-  *code = word == 0 ? ULY_OK : word == uly::kDevSmemAlign ? ULY_ERR_CUDA : ULY_ERR_TIMEOUT;
+  *code = word == 0                    ? ULY_OK
+          : word == uly::kDevSmemAlign ? ULY_ERR_CUDA
+          : word == uly::kDevBounds    ? ULY_ERR_BOUNDS
+                                       : ULY_ERR_TIMEOUT;
   return ULY_OK;
 }

@@ -160,7 +160,8 @@ template <int D, bool kOF32>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o, const uint16_t* __restrict__ dO,
                                                       const float* __restrict__ lse, float* __restrict__ stats,
                                                       const int32_t* __restrict__ shifts, int64_t rb0, int64_t n,
-                                                      int64_t n_pad, int32_t hq, int64_t total) {
+                                                      int64_t n_pad, int32_t hq, int64_t total, int64_t elems,
+                                                      int64_t stats_elems, int* status) {
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= total) return;
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
   const int64_t i = rem / hq;          // token (head fastest: consecutive warps read adjacent rows)
   const int64_t h = rem % hq;
   const int64_t sidx = stats_index(rb * hq + h, n_pad, i);
+  if (!in_bounds(sidx >= 0 && sidx + 64 < stats_elems, status)) return;
   if (i >= n) {
     if (lane == 0) {
       stats[sidx] = 0.f;
@@ -178,6 +180,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const void* __restrict__ o
     return;
   }
   const int64_t row = (rb * n + i) * hq + h;
+  if (!in_bounds((row + 1) * D <= elems, status)) return;
   constexpr int E = D / 32;
   float acc = 0.f;
 #pragma unroll
@@ -230,6 +233,7 @@ struct Params {
   float scale, scale_log2;
   int32_t g_f32;
   uint64_t limit_ns;
+  int64_t g_elems, stats_elems, se_elems;   // dK/dV, statistics and segment-table extents (debug build checks)
 };
 
 template <int D>
@@ -358,10 +362,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       tma_prefetch_desc(is_q ? &mq : &mdo);
       if (is_q && niter > 0) {
         mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKV);
-        for (int dc = 0; dc < D / 64; ++dc) {
-          tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0 - p.k_base), rb);
-          tma_load_4d(&mv, &bars->kv_full, smem + L::oV + dc * BKV * 128, dc * 64, g, int(k0 - p.k_base), rb);
-        }
+        if (in_bounds(k0 - p.k_base >= 0 && k0 - p.k_base < p.k_rows, p.status))
+          for (int dc = 0; dc < D / 64; ++dc) {
+            tma_load_4d(&mk, &bars->kv_full, smem + L::oK + dc * BKV * 128, dc * 64, g, int(k0 - p.k_base), rb);
+            tma_load_4d(&mv, &bars->kv_full, smem + L::oV + dc * BKV * 128, dc * 64, g, int(k0 - p.k_base), rb);
+          }
       }
       int issued = 0;
       for (int it = 0; it < niter; ++it) {
@@ -369,16 +374,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         const int h = g * p.G + it / nqt;
         const int q0 = int((qt_first + it % nqt) * int64_t(BQ) - p.q_base);   // row in the Q-side buffers
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
+        const bool q_in = in_bounds(q0 >= 0 && q0 < p.q_rows, p.status);
         if (is_q) {
           mbar_arrive_expect_tx(&full[st], L::kQ);
-          for (int dc = 0; dc < D / 64; ++dc)
-            tma_load_4d(&mq, &full[st], smem + L::oQ + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
+          if (q_in)
+            for (int dc = 0; dc < D / 64; ++dc)
+              tma_load_4d(&mq, &full[st], smem + L::oQ + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
         } else {
           mbar_arrive_expect_tx(&full[st], L::kQ + L::kSt);
-          for (int dc = 0; dc < D / 64; ++dc)
-            tma_load_4d(&mdo, &full[st], smem + L::oDO + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
-          bulk_load(smem + L::oSt + st * L::kSt, p.stats + stats_index(int64_t(rb) * p.hq + h, p.n_pad, q0), L::kSt,
-                    &full[st]);
+          const int64_t si = stats_index(int64_t(rb) * p.hq + h, p.n_pad, q0);
+          if (q_in && in_bounds(si >= 0 && si + L::kSt / 4 <= p.stats_elems, p.status)) {
+            for (int dc = 0; dc < D / 64; ++dc)
+              tma_load_4d(&mdo, &full[st], smem + L::oDO + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
+            bulk_load(smem + L::oSt + st * L::kSt, p.stats + si, L::kSt, &full[st]);
+          }
         }
         issued = it + 1;
       }
@@ -472,7 +481,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t kj = k0 + row;
     // query rows [kj, kj_end) see key kj (none for a key outside [k_lo, k_hi))
-    const int64_t kj_end = (kj < k_end && kj >= p.k_lo && kj < p.k_hi)
+    const int64_t kj_end = (kj < k_end && kj >= p.k_lo && kj < p.k_hi &&
+                            in_bounds(int64_t(bb) * p.n + kj < p.se_elems, p.status))
                                ? (se[kj] < q_blk_end ? int64_t(se[kj]) : q_blk_end) : kj;
     bool ok = true;
     for (int it = 0; it < niter; ++it) {
@@ -570,8 +580,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     }
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
-      const bool valid = kj < k_end;
       const int64_t orow = (int64_t(rb) * p.k_rows + (kj - p.k_base)) * p.hkv + g;
+      const bool valid = kj < k_end && in_bounds(orow >= 0 && (orow + 1) * D <= p.g_elems, p.status);
       {
         const int which = wg;   // warpgroup 0 stores dK, warpgroup 1 stores dV
         const uint32_t base = which == 0 ? tDK : tDV;
@@ -645,6 +655,7 @@ struct Params {
   float scale, scale_log2;
   int32_t g_f32;
   uint64_t limit_ns;
+  int64_t g_elems, stats_elems, ss_elems;   // dQ, statistics and segment-table extents (debug build checks)
 };
 
 template <int D>
@@ -750,8 +761,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       if (is_k) {
         mbar_arrive_expect_tx(&bars->qdo_full, 2 * L::kTile);
         for (int dc = 0; dc < D / 64; ++dc) {
-          tma_load_4d(&mq, &bars->qdo_full, smem + L::oQ + dc * BM * 128, dc * 64, h, int(t0 - p.q_base), rb);
-          tma_load_4d(&mdo, &bars->qdo_full, smem + L::oDO + dc * BM * 128, dc * 64, h, int(t0 - p.q_base), rb);
+          if (in_bounds(t0 - p.q_base >= 0 && t0 - p.q_base < p.q_rows, p.status)) {
+            tma_load_4d(&mq, &bars->qdo_full, smem + L::oQ + dc * BM * 128, dc * 64, h, int(t0 - p.q_base), rb);
+            tma_load_4d(&mdo, &bars->qdo_full, smem + L::oDO + dc * BM * 128, dc * 64, h, int(t0 - p.q_base), rb);
+          }
         }
       }
       int issued = 0;
@@ -760,8 +773,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const int k0 = (kv_first + it) * BN;
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         mbar_arrive_expect_tx(&full[st], L::kTile);
-        for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(map, &full[st], smem + base + st * L::kTile + dc * BN * 128, dc * 64, g, int(k0 - p.k_base), rb);
+        if (in_bounds(k0 - p.k_base >= 0 && k0 - p.k_base < p.k_rows, p.status))
+          for (int dc = 0; dc < D / 64; ++dc)
+            tma_load_4d(map, &full[st], smem + base + st * L::kTile + dc * BN * 128, dc * 64, g, int(k0 - p.k_base),
+                        rb);
         issued = it + 1;
       }
       if (*abort_flag) {
@@ -826,15 +841,17 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t i = t0 + row;                  // global row
     const bool valid = i < q_blk_end;
-    const int64_t s_i = valid ? ss[i] : seg_hi;
+    const int64_t s_i = valid && in_bounds(int64_t(bb) * p.n + i < p.ss_elems, p.status) ? ss[i] : seg_hi;
     // this row's keys: [row_lo, row_hi) = its sample's keys up to i, inside [k_lo, k_hi)
     const int64_t row_lo = s_i > p.k_lo ? s_i : p.k_lo;
     const int64_t row_hi = i + 1 < p.k_hi ? i + 1 : p.k_hi;
     float nl = 0.f, nd = 0.f;   // -LSE*log2e, -D of this row
     if (valid) {
       const int64_t si = stats_index(int64_t(rb) * p.hq + h, p.n_pad, i - p.q_base);
-      nl = p.stats[si];
-      nd = p.stats[si + 64];
+      if (in_bounds(si >= 0 && si + 64 < p.stats_elems, p.status)) {
+        nl = p.stats[si];
+        nd = p.stats[si + 64];
+      }
     }
     const float sl = p.scale_log2 * pow2i(p.shifts[kShQ]) * pow2i(p.shifts[kShK]);   // q'.k' units, as dK/dV
     const uint64_t sl2 = f2_pack(sl, sl), nl2 = f2_pack(nl, nl), nd2 = f2_pack(nd, nd);
@@ -887,6 +904,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     if (mbar_wait(&bars->mma_final, 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
       const int64_t orow = (int64_t(rb) * p.q_rows + (i - p.q_base)) * p.hq + h;
+      const bool store = valid && in_bounds(orow >= 0 && (orow + 1) * D <= p.g_elems, p.status);
       // dQ' = dS' k' = scale^-1 dQ 2^-(sdo+sv+sk)
       const float mq = p.scale * pow2i(p.shifts[kShDO]) * pow2i(p.shifts[kShV]) * pow2i(p.shifts[kShK]);
       for (int c = 64 * wg; c < D; c += 128) {
@@ -900,7 +918,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = 0u;
           }
-          if (valid) {
+          if (store) {
             if (p.g_f32) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.dq) + orow * D + c + c2);
 #pragma unroll
@@ -1059,6 +1077,9 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     bwd::bwd_to_f16_kernel<<<dim3(gx, 4), 256, 0, cs>>>(a, amax, shifts);
     if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
+  const int64_t qelems = Pb * qr * hq * s.d;                       // Q-side buffer elements
+  const int64_t stats_elems = int64_t(s.b) * s.h_q * bwd_n_pad(s.n) * 2;   // the workspace's statistics table
+  int* st_word = reinterpret_cast<int*>(wsb);
   {
     const int64_t total = nrb * n_pad * hq;
     const int64_t blocks = (total * 32 + 255) / 256;
@@ -1067,11 +1088,11 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     const uint16_t* dop = static_cast<const uint16_t*>(do_head);
     const unsigned nb = unsigned(blocks);
     if (s.d == 128) {
-      if (of32) bwd::bwd_pre_kernel<128, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
-      else bwd::bwd_pre_kernel<128, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
+      if (of32) bwd::bwd_pre_kernel<128, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total, qelems, stats_elems, st_word);
+      else bwd::bwd_pre_kernel<128, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total, qelems, stats_elems, st_word);
     } else {
-      if (of32) bwd::bwd_pre_kernel<64, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
-      else bwd::bwd_pre_kernel<64, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total);
+      if (of32) bwd::bwd_pre_kernel<64, true><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total, qelems, stats_elems, st_word);
+      else bwd::bwd_pre_kernel<64, false><<<nb, 256, 0, cs>>>(o_head, dop, lse, stats, shifts, rb0, qr, n_pad, int32_t(hq), total, qelems, stats_elems, st_word);
     }
     if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
@@ -1105,6 +1126,9 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.scale_log2 = scale * bwd::kLog2e;
     p.g_f32 = g_dtype == ULY_F32;
     p.limit_ns = 2000000000ull;
+    p.g_elems = Pb * kr * hkv * s.d;
+    p.stats_elems = stats_elems;
+    p.se_elems = s.b * s.n;
     const int64_t grid = (kr + bwd::dkdv::BKV - 1) / bwd::dkdv::BKV * P_sel * s.b * hkv;
     if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
     if (s.d == 128) {
@@ -1147,6 +1171,9 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
     p.scale_log2 = scale * bwd::kLog2e;
     p.g_f32 = g_dtype == ULY_F32;
     p.limit_ns = 2000000000ull;
+    p.g_elems = qelems;
+    p.stats_elems = stats_elems;
+    p.ss_elems = s.b * s.n;
     const int64_t grid = int64_t(p.ntiles) * P_sel * s.b * hq;
     if (grid > 0x7FFFFFFF) return ULY_ERR_UNSUPPORTED;
     if (s.d == 128) {

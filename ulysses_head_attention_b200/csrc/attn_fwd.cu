@@ -62,12 +62,13 @@ struct Params {
   int* status;
   int64_t n;                 // tokens of the whole sequence (the segment tables')
   int64_t q_base, q_rows;    // Q, O, LSE hold the global rows [q_base, q_base + q_rows); 0, n for whole tensors
-  int64_t k_base;            // K, V hold the global keys from k_base on (a multiple of BN); 0 for whole tensors
+  int64_t k_base, k_rows;    // K, V hold the global keys [k_base, k_base + k_rows) (k_base a multiple of BN)
   int64_t k_lo, k_hi;        // keys outside [k_lo, k_hi) are not attended (one ring block); 0, n otherwise
   int32_t b, P_sel, rank0, hq, G, ntiles, npairs;
   float scale_log2;
   int32_t o_f32;
   uint64_t limit_ns;
+  int64_t o_elems, lse_elems, ss_elems;   // buffer extents, for the debug build's bounds checks
 };
 
 template <int D>
@@ -191,10 +192,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       if (is_k) {
         tma_prefetch_desc(&mq);
         mbar_arrive_expect_tx(&bars->q_full, (tr1.valid ? 2 : 1) * L::kTileBytes);
-        for (int q = 0; q < (tr1.valid ? 2 : 1); ++q)
-          for (int dc = 0; dc < D / 64; ++dc)
-            tma_load_4d(&mq, &bars->q_full, smem + L::kQ + q * L::kTileBytes + dc * BM * 128, dc * 64, j,
-                        int((q ? tr1 : tr0).t0 - p.q_base), rb);
+        for (int q = 0; q < (tr1.valid ? 2 : 1); ++q) {
+          const int64_t qc = (q ? tr1 : tr0).t0 - p.q_base;
+          if (in_bounds(qc >= 0 && qc < p.q_rows && rb < p.P_sel * p.b + p.rank0 * p.b, p.status))
+            for (int dc = 0; dc < D / 64; ++dc)
+              tma_load_4d(&mq, &bars->q_full, smem + L::kQ + q * L::kTileBytes + dc * BM * 128, dc * 64, j, int(qc),
+                          rb);
+        }
       }
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
@@ -202,9 +206,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         const int k0 = (j_lo + it) * BN;
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         mbar_arrive_expect_tx(&full[st], L::kTileBytes);
-        for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(map, &full[st], smem + base + st * L::kTileBytes + dc * BN * 128, dc * 64, g,
-                      int(k0 - p.k_base), rb);
+        if (in_bounds(k0 - p.k_base >= 0 && k0 - p.k_base < p.k_rows, p.status))
+          for (int dc = 0; dc < D / 64; ++dc)
+            tma_load_4d(map, &full[st], smem + base + st * L::kTileBytes + dc * BN * 128, dc * 64, g,
+                        int(k0 - p.k_base), rb);
         issued = it + 1;
       }
       // Error path only: let every copy this thread started land before exit.
@@ -282,7 +287,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     const int64_t i = tr.t0 + row;                 // global row
     const bool valid = tr.valid && i < q_end;
     const int64_t il = i - p.q_base;               // row in the Q / O / LSE buffers
-    const int64_t s_i = valid ? ss[i] : tr.seg_hi;
+    const int64_t s_i = valid && in_bounds(int64_t(bb) * p.n + i < p.ss_elems, p.status) ? ss[i] : tr.seg_hi;
     // this row's keys: [row_lo, row_hi) = its sample's keys up to i, inside [k_lo, k_hi)
     const int64_t row_lo = s_i > p.k_lo ? s_i : p.k_lo;
     const int64_t row_hi = i + 1 < p.k_hi ? i + 1 : p.k_hi;
@@ -399,7 +404,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         uint32_t o[32];
         tmem_ld32(tO + lane_off + c, o);
         tmem_ld_wait();
-        if (valid) {
+        if (valid && in_bounds(orow >= 0 && (orow + 1) * D <= p.o_elems, p.status)) {
           if (p.o_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D + c);
 #pragma unroll
@@ -420,19 +425,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           }
         }
       }
-      if (valid)
-        p.lse[(int64_t(rb) * p.hq + j) * p.q_rows + il] = row_vis ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const int64_t li = (int64_t(rb) * p.hq + j) * p.q_rows + il;
+      if (valid && in_bounds(li >= 0 && li < p.lse_elems, p.status))
+        p.lse[li] = row_vis ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
     } else if (ntile == 0 && valid) {
       // no key of [k_lo, k_hi) is visible to this query tile: O = 0, LSE = -inf
       const int64_t orow = (int64_t(rb) * p.q_rows + il) * p.hq + j;
-      if (p.o_f32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D);
-        for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D);
-        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      const int64_t li = (int64_t(rb) * p.hq + j) * p.q_rows + il;
+      if (in_bounds(orow >= 0 && (orow + 1) * D <= p.o_elems && li >= 0 && li < p.lse_elems, p.status)) {
+        if (p.o_f32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow * D);
+          for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.o) + orow * D);
+          for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        p.lse[li] = -INFINITY;
       }
-      p.lse[(int64_t(rb) * p.hq + j) * p.q_rows + il] = -INFINITY;
     }
   }
 
@@ -545,6 +554,7 @@ static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const vo
   p.q_base = rows.q_base;
   p.q_rows = rows.q_rows;
   p.k_base = rows.k_base;
+  p.k_rows = rows.k_rows;
   p.k_lo = k_lo;
   p.k_hi = k_hi;
   p.b = int32_t(s.b);
@@ -558,6 +568,9 @@ static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const vo
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_f32 = o_dtype == ULY_F32;
   p.limit_ns = 2000000000ull;
+  p.o_elems = Pb * rows.q_rows * hq * s.d;
+  p.lse_elems = Pb * hq * rows.q_rows;
+  p.ss_elems = s.b * s.n;
   e = s.d == 128 ? fwd::launch<128>(mq, mk, mv, p, grid, cs) : fwd::launch<64>(mq, mk, mv, p, grid, cs);
   return cuda_status(e);
 }

@@ -17,9 +17,19 @@
 #include <cstdint>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace uly {
 namespace {
+
+#ifdef ULY_DEBUG_BOUNDS
+// The debug build's record of a re-layout index outside its buffer (read and
+// cleared by ulysses_debug_status).
+__device__ int g_relayout_bounds;
+#define ULY_RELAYOUT_STATUS (&g_relayout_bounds)
+#else
+#define ULY_RELAYOUT_STATUS nullptr
+#endif
 
 struct RelayoutArgs {
   int64_t b, m, n;        // batch rows, tokens per rank (n/P), tokens
@@ -28,6 +38,7 @@ struct RelayoutArgs {
   int32_t vpr_shift;      // log2(vpr) when vpr is a power of two, else -1
   int32_t tile_tokens;    // T
   int32_t tiles_per_rank; // ceil(m / T)
+  int64_t total_vecs;     // vectors in either buffer (debug build checks)
 };
 
 constexpr int kThreads = 256;
@@ -64,12 +75,13 @@ __global__ void __launch_bounds__(kThreads) relayout_kernel(const V* __restrict_
         col = i - row * a.vpr;
       }
       seq_idx[u] = seq_base + row * a.vrow + col;
-      if (i < total) val[u] = kToHead ? src[seq_idx[u]] : src[head_base + i];
+      if (i < total && in_bounds(seq_idx[u] < a.total_vecs && head_base + i < a.total_vecs, ULY_RELAYOUT_STATUS))
+        val[u] = kToHead ? src[seq_idx[u]] : src[head_base + i];
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t i = i0 + int64_t(u) * kThreads;
-      if (i < total) {
+      if (i < total && in_bounds(seq_idx[u] < a.total_vecs && head_base + i < a.total_vecs, ULY_RELAYOUT_STATUS)) {
         if (kToHead)
           dst[head_base + i] = val[u];
         else
@@ -99,6 +111,7 @@ cudaError_t launch_typed(const void* src, void* dst, int64_t b, int64_t n, int64
   if (T > a.m) T = a.m;
   a.tile_tokens = int32_t(T);
   a.tiles_per_rank = int32_t((a.m + T - 1) / T);
+  a.total_vecs = b * n * H * d * int64_t(esize) / int64_t(sizeof(V));
   const int64_t gx = int64_t(P) * b * a.tiles_per_rank;
   if (gx > 0x7FFFFFFF || P > 65535) return cudaErrorInvalidConfiguration;
   const dim3 grid{unsigned(gx), unsigned(P), 1u};
@@ -356,3 +369,29 @@ extern "C" uly_status ulysses_transpose_runs(const void* src, void* dst, int64_t
   else e = launch_transpose<uint8_t>(src, dst, A, B, run_bytes, cs);
   return cuda_status(e);
 }
+
+// Debug build: reads and clears the re-layout kernels' bounds record.  The
+// release build compiles no checks and answers ULY_ERR_UNSUPPORTED.
+extern "C" uly_status ulysses_debug_status(void* stream, int32_t* code) {
+  if (!code) return ULY_ERR_INVALID_ARG;
+#ifdef ULY_DEBUG_BOUNDS
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyFromSymbolAsync(&word, uly::g_relayout_bounds, sizeof(int), 0, cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return ULY_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ULY_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbolAsync(uly::g_relayout_bounds, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s) !=
+      cudaSuccess)
+    return ULY_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ULY_ERR_CUDA;
+  *code = word == 0 ? ULY_OK : ULY_ERR_BOUNDS;
+  return ULY_OK;
+#else
+  (void)stream;
+  *code = ULY_OK;
+  return ULY_ERR_UNSUPPORTED;
+#endif
+}
+

@@ -55,13 +55,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Error words written to the caller's status slot: a wait gave up, or a
-// kernel found its dynamic shared memory too poorly aligned for its tiles.
+// Error words written to the caller's status slot: a wait gave up, a
+// kernel found its dynamic shared memory too poorly aligned for its tiles,
+// or (debug build only) an index fell outside its buffer.
 enum : int {
   kDevOk = 0,
   kDevTimeout = 1,
   kDevSmemAlign = 2,
+  kDevBounds = 3,
 };
+
+// The bounds-checked debug build (compiled with ULY_DEBUG_BOUNDS) checks every
+// global index and TMA tile coordinate before the access: one outside its
+// buffer is recorded as kDevBounds in the status word (the first error code
+// wins) and the access is skipped, so a wait that then never completes gives
+// up on its time limit instead of reading or writing stray memory.  The
+// release build compiles every check away.
+#ifdef ULY_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+
+__device__ __forceinline__ bool in_bounds(bool ok, int* status) {
+  if constexpr (!kDebugBounds) {
+    return true;
+  } else {
+    if (!ok && status) atomicCAS(status, 0, kDevBounds);
+    return ok;
+  }
+}
 
 // Bounded wait on an mbarrier phase.  Repeats the (suspending) try_wait;
 // every 16 tries it checks the CTA-wide abort flag (set by any warp that gave
