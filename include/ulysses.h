@@ -323,8 +323,11 @@ uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_head, const 
  *   enqueue nothing.  The call allocates nothing (no cudaMalloc, no
  *   allocating library routine).
  *   First call per device: looks up the scratch's device address
- *   (cudaGetSymbolAddress) with that device current and caches it; make that
- *   first call before any stream capture.
+ *   (cudaGetSymbolAddress) with that device current and caches it for the
+ *   life of the process; make that first call before any stream capture.
+ *   cudaDeviceReset (which reloads the module and may move the array) is not
+ *   supported while this library is loaded: the cached address would be
+ *   stale.
  *   Sharing: every call on a device uses the same scratch and it keeps the
  *   last call's contents (nothing in it needs to start at zero).  Calls whose
  *   work overlaps on the GPU (e.g. on two concurrently running streams) race
