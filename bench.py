@@ -517,73 +517,33 @@ def run_ours(args, w):
 
 
 def measure_e2e(layer, steps, barrier, world, dev):
-    """The same metric with every step's inputs copied in from pinned host
-    memory and its outputs (O, dQ, dK, dV) copied back, inside the timed
-    region.  Host-to-device copies run on one side stream and device-to-host
-    copies on another, each ordered against the compute stream by events, so
-    that step i+1's inputs arrive and step i's outputs leave while attention
-    runs."""
+    """The same metric through the C ABI's host-buffer call
+    (ulysses_layer_step_host): every step copies its inputs in from pinned
+    host memory and its outputs (O, dQ, dK, dV) back, inside the timed
+    region.  The library runs the copies on two side streams, ordered by
+    events against the kernels, so that dO arrives during the forward, O
+    leaves during the backward, and one step's gradients leave while the
+    next step's inputs arrive."""
     import torch
+    uly, w = layer.uly, layer.w
+    P, b, m, d = w.P, w.b, w.n // w.P, w.d
     f32 = torch.float32
+    step = uly.LayerStepHost(b, w.n, w.h_q, w.h_kv, d, P, dev)
+    h_out = [torch.empty((P, b, m, h, d), dtype=f32).pin_memory() for h in (w.h_q, w.h_q, w.h_kv, w.h_kv)]
+    ins = [layer.host[k] for k in ("q", "k", "v", "do")]
+    h2d = sum(t.numel() * t.element_size() for t in ins) + layer.host_pos.numel() * 8
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
     main = torch.cuda.current_stream()
-    up, down = torch.cuda.Stream(), torch.cuda.Stream()
-    h_out = {"o": torch.empty(layer.o_seq.shape, dtype=f32, pin_memory=True)}
-    for k in layer.g_seq:
-        h_out[k] = torch.empty(layer.g_seq[k].shape, dtype=f32, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in layer.host.values()) + layer.host_pos.numel() * 8
-    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
-    uly, h, s, g = layer.uly, layer.head, layer.seq, layer.g_head
-    # position_ids are read by the backward too, which still runs when the
-    # next step's inputs arrive: two buffers, used by alternate steps
-    pos = [layer.pos, torch.empty_like(layer.pos)]
-    ev = lambda: torch.cuda.Event()   # noqa: E731
 
     def run(n_steps):
-        # state carried between steps: the events the next copies wait on
-        inputs_free, o_free, g_free = ev(), ev(), ev()
-        inputs_free.record(main), o_free.record(main), g_free.record(main)
-        for i in range(n_steps):
-            p_i = pos[i % 2]   # last read by step i - 2, whose backward finished before inputs_free
-            up.wait_event(inputs_free)
-            with torch.cuda.stream(up):
-                for k in ("q", "k", "v"):
-                    s[k].copy_(layer.host[k], non_blocking=True)
-                p_i.copy_(layer.host_pos, non_blocking=True)
-                qkv_in = ev(); qkv_in.record(up)
-                s["do"].copy_(layer.host["do"], non_blocking=True)
-                do_in = ev(); do_in.record(up)
-            main.wait_event(qkv_in)
-            uly.ulysses_seq_to_head(s["q"], h["q"])
-            for k in ("k", "v"):
-                uly.ulysses_kv_seq_to_head(s[k], h[k])
-            uly.ulysses_attn_fwd(h["q"], h["k"], h["v"], p_i, layer.o_head, layer.lse, layer.ws_f)
-            main.wait_event(o_free)
-            uly.ulysses_head_to_seq(layer.o_head, layer.o_seq)
-            o_ready = ev(); o_ready.record(main)
-            main.wait_event(do_in)
-            uly.ulysses_seq_to_head(s["do"], h["do"])
-            inputs_free = ev(); inputs_free.record(main)   # q, k, v, dO consumed: next inputs may land
-            down.wait_event(o_ready)
-            with torch.cuda.stream(down):
-                h_out["o"].copy_(layer.o_seq, non_blocking=True)
-                o_free = ev(); o_free.record(down)
-            uly.ulysses_attn_bwd(h["q"], h["k"], h["v"], layer.o_head, layer.lse, h["do"], p_i,
-                                 g["q"], g["k"], g["v"], layer.ws_b)
-            main.wait_event(g_free)
-            uly.ulysses_head_to_seq(g["q"], layer.g_seq["q"])
-            for k in ("k", "v"):
-                uly.ulysses_kv_head_to_seq(g[k], layer.g_seq[k])
-            g_ready = ev(); g_ready.record(main)
-            down.wait_event(g_ready)
-            with torch.cuda.stream(down):
-                for k in layer.g_seq:
-                    h_out[k].copy_(layer.g_seq[k], non_blocking=True)
-                g_free = ev(); g_free.record(down)
-        main.wait_event(o_free)
-        main.wait_event(g_free)
+        for _ in range(n_steps):
+            step.step(*ins, layer.host_pos, *h_out)
+        main.wait_event(step.done_event())
 
     run(1)
     torch.cuda.synchronize()
+    if step.status() != 0:
+        raise RuntimeError("a kernel reported a pipeline timeout in the end-to-end warm-up")
     barrier()
     torch.cuda.synchronize()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -592,11 +552,15 @@ def measure_e2e(layer, steps, barrier, world, dev):
     e2.record(main)
     torch.cuda.synchronize()
     barrier()
-    layer.check_status("in the end-to-end region")
+    if step.status() != 0:
+        raise RuntimeError("a kernel reported a pipeline timeout in the end-to-end region")
     e2e_ms = max_over_ranks(s2.elapsed_time(e2), world, dev) / steps
+    del step
+    torch.cuda.empty_cache()
     return {"value": whole_job_tflops(world, layer.fwd_flops + layer.bwd_flops, e2e_ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-            "copies": "pinned host; H2D and D2H on two side streams ordered by events, overlapping attention"}
+            "api": "ulysses_layer_step_host (C ABI, pinned host buffers in and out)",
+            "copies": "H2D and D2H on two side streams ordered by events, overlapping attention"}
 
 
 # the other workloads timed in the same run: (name, steps, warm-up)

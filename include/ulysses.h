@@ -460,6 +460,43 @@ uly_status ulysses_ipc_open(const void* handle, void** dev_ptr_out);
 uly_status ulysses_ipc_close(void* dev_ptr);
 
 /*
+ * ulysses_layer_step_host -- one whole Ulysses layer step, forward and
+ * backward, from host memory to host memory ("How Ulysses works", steps
+ * 1-6): the seq-sharded inputs are copied in, seq_to_head(q, k, v) ->
+ * ulysses_attn_fwd -> head_to_seq(O); seq_to_head(dO) -> ulysses_attn_bwd ->
+ * head_to_seq(dQ, dK, dV) run for all P virtual ranks, and the seq-sharded
+ * outputs are copied out.  A convenience over the calls above, with the
+ * copies overlapping the attention kernels:
+ *   inputs   q_seq, do_seq [P][b][n/P][h_q][d] bf16; k_seq, v_seq
+ *            [P][b][n/P][h_kv][d] bf16; position_ids [b][n] int64: host
+ *            memory, page-locked for the copies to run asynchronously
+ *   outputs  o_seq, dq_seq [P][b][n/P][h_q][d] float; dk_seq, dv_seq
+ *            [P][b][n/P][h_kv][d] float: host memory, page-locked
+ *   dev      caller-owned device memory of ulysses_layer_step_host_bytes()
+ *            bytes, 256-byte aligned (ULY_ERR_WORKSPACE otherwise): device
+ *            staging, head-layout buffers and both attention workspaces;
+ *            reused by every call with the same shape
+ *   streams  `stream` runs the kernels, `h2d_stream` the host-to-device and
+ *            `d2h_stream` the device-to-host copies (three distinct streams
+ *            of the current device)
+ *   events   three caller-created cudaEvent_t (as void*), the same for every
+ *            call on `dev`, that order consecutive calls: events[0] "this
+ *            call's inputs are consumed" (the next call's input copies wait
+ *            for it), events[1] "O is on the host", events[2] "the gradients
+ *            are on the host".  All outputs of a call are on the host once
+ *            the events[2] it recorded has completed (cudaEventSynchronize).
+ * Errors as for the calls it makes; ulysses_layer_status reads (and
+ * clears) the attention workspaces' status words inside `dev`.
+ */
+size_t ulysses_layer_step_host_bytes(const uly_shape* shape);
+uly_status ulysses_layer_step_host(const void* q_seq, const void* k_seq, const void* v_seq, const void* do_seq,
+                                   const int64_t* position_ids, const uly_shape* shape, float softmax_scale,
+                                   float* o_seq, float* dq_seq, float* dk_seq, float* dv_seq, void* dev,
+                                   size_t dev_bytes, void* stream, void* h2d_stream, void* d2h_stream,
+                                   void* const* events);
+uly_status ulysses_layer_status(void* dev, const uly_shape* shape, void* stream, int32_t* code);
+
+/*
  * ulysses_selftest_wait_timeout -- runs the failure path of the attention
  * kernels' bounded waits on purpose, so that it can be checked on a GPU.
  * (Not a step of the method: the pages have no counterpart; it tests the

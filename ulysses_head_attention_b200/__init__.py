@@ -39,7 +39,8 @@ EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head
            "ulysses_seq_to_head_push", "ulysses_head_to_seq_push", "ulysses_wait_flags", "ulysses_release_flags",
            "ulysses_ipc_handle",
            "ulysses_ipc_open", "ulysses_ipc_close", "ulysses_attn_fwd_block", "ulysses_attn_bwd_block",
-           "ulysses_accumulate", "ulysses_debug_status", "ulysses_status_string")
+           "ulysses_accumulate", "ulysses_debug_status", "ulysses_layer_step_host_bytes", "ulysses_layer_step_host",
+           "ulysses_layer_status", "ulysses_status_string")
 
 
 class UlyShape(ctypes.Structure):
@@ -93,6 +94,10 @@ def _load() -> ctypes.CDLL:
                                     vp, sz, vp], i32),
         "ulysses_accumulate": ([vp, vp, i64, vp], i32),
         "ulysses_debug_status": ([vp, ctypes.POINTER(ctypes.c_int32)], i32),
+        "ulysses_layer_step_host_bytes": ([shp], sz),
+        "ulysses_layer_step_host": ([vp, vp, vp, vp, vp, shp, f32, vp, vp, vp, vp, vp, sz, vp, vp, vp,
+                                     ctypes.POINTER(vp)], i32),
+        "ulysses_layer_status": ([vp, shp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "ulysses_status_string": ([i32], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
@@ -582,4 +587,66 @@ def ulysses_ipc_open(handle: bytes) -> int:
 
 def ulysses_ipc_close(addr: int) -> None:
     _check(lib.ulysses_ipc_close(ctypes.c_void_p(addr)), "ulysses_ipc_close")
+
+
+# ----------------------------------------------------------------------------- host to host
+def _host(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+class LayerStepHost:
+    """ulysses_layer_step_host with its device buffer, streams and events:
+    one layer step from (pinned) host tensors to host tensors."""
+
+    def __init__(self, b: int, n: int, h_q: int, h_kv: int, d: int, P: int, device=None):
+        self.shape = UlyShape(b, n, h_q, h_kv, d, P)
+        self.device = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        nbytes = int(lib.ulysses_layer_step_host_bytes(ctypes.byref(self.shape)))
+        if nbytes == 0:
+            raise ValueError("shape not accepted by the library")
+        self.dev = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.h2d, self.d2h = torch.cuda.Stream(self.device), torch.cuda.Stream(self.device)
+        self.events = [torch.cuda.Event() for _ in range(3)]
+
+    def step(self, q_seq, k_seq, v_seq, do_seq, position_ids, o_seq, dq_seq, dk_seq, dv_seq,
+             softmax_scale: float = 0.0, stream=None) -> None:
+        P, b, n, hq, hkv, d = (self.shape.P, self.shape.b, self.shape.n, self.shape.h_q, self.shape.h_kv,
+                               self.shape.d)
+        m = n // P
+        _expect(q_seq, (P, b, m, hq, d), _BF16, "q_seq")
+        _expect(k_seq, (P, b, m, hkv, d), _BF16, "k_seq")
+        _expect(v_seq, (P, b, m, hkv, d), _BF16, "v_seq")
+        _expect(do_seq, (P, b, m, hq, d), _BF16, "do_seq")
+        _expect(position_ids, (b, n), _I64, "position_ids")
+        _expect(o_seq, (P, b, m, hq, d), _F32, "o_seq")
+        _expect(dq_seq, (P, b, m, hq, d), _F32, "dq_seq")
+        _expect(dk_seq, (P, b, m, hkv, d), _F32, "dk_seq")
+        _expect(dv_seq, (P, b, m, hkv, d), _F32, "dv_seq")
+        for e in self.events:   # record once so the handles exist (a never-recorded event is complete)
+            if e.cuda_event == 0:
+                e.record(self.d2h)
+        evs = (ctypes.c_void_p * 3)(*[e.cuda_event for e in self.events])
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        _check(lib.ulysses_layer_step_host(_host(q_seq, "q_seq"), _host(k_seq, "k_seq"), _host(v_seq, "v_seq"),
+                                           _host(do_seq, "do_seq"), _host(position_ids, "position_ids"),
+                                           ctypes.byref(self.shape), softmax_scale, _host(o_seq, "o_seq"),
+                                           _host(dq_seq, "dq_seq"), _host(dk_seq, "dk_seq"), _host(dv_seq, "dv_seq"),
+                                           self.dev.data_ptr(), self.dev.numel(), ctypes.c_void_p(s.cuda_stream),
+                                           ctypes.c_void_p(self.h2d.cuda_stream), ctypes.c_void_p(self.d2h.cuda_stream),
+                                           evs), "ulysses_layer_step_host")
+
+    def done_event(self) -> torch.cuda.Event:
+        """Completes once every output of the last step is on the host."""
+        return self.events[2]
+
+    def status(self) -> int:
+        code = ctypes.c_int32(-1)
+        _check(lib.ulysses_layer_status(self.dev.data_ptr(), ctypes.byref(self.shape),
+                                        ctypes.c_void_p(torch.cuda.current_stream(self.device).cuda_stream),
+                                        ctypes.byref(code)), "ulysses_layer_status")
+        return int(code.value)
 
