@@ -40,7 +40,7 @@ def test_status_strings():
 
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake-pointer checks run only without a GPU")
 F = 0x100000          # fake, 256-byte aligned "device" addresses, never dereferenced
-INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 4
+INVALID, UNSUPPORTED, CUDA, WORKSPACE = 1, 2, 3, 4
 
 
 @no_gpu
@@ -307,7 +307,9 @@ def test_noalloc_forward_refuses_before_touching_the_device():
     assert call(shape(n=1000, P=16)) == INVALID
     assert call(shape(b=1, n=1 << 20)) == WORKSPACE
     assert call(shape(b=2, n=1 << 19)) == WORKSPACE
-    assert uly.ulysses_attn_fwd_workspace(shape(b=1, n=1 << 19)) <= 256 + 2 * 4 * (1 << 19)
+    # the largest accepted size passes the size check and stops at the device
+    # lookup, which has no device to find here
+    assert call(shape(b=1, n=1 << 19)) == CUDA
 
 
 @no_gpu

@@ -4,7 +4,8 @@ The GPU forward produces O (fp32) and LSE; the GPU backward then produces
 dQ, dK, dV.  The oracle's backward recomputes everything in fp64 from the
 same bf16 inputs (its own O, not the GPU's).  Tolerance for fp32-stored
 gradients: every element within 1e-2 of the oracle, and
-sum|g-r|/sum|r| <= 2e-3; bf16-stored gradients at twice those bounds.
+sum|g-r|/sum|r| <= 2e-3; bf16-stored gradients: every element within
+1e-2 + 2^-8 |ref| (one more bf16 rounding), sum|g-r|/sum|r| <= 4e-3.
 """
 import numpy as np
 import pytest
@@ -12,7 +13,7 @@ import torch
 
 import oracle
 import synthetic
-from gpu_util import MAX_ABS_BF16, MEAN_REL_BF16, assert_close, to_dev_bf16
+from gpu_util import assert_close, assert_close_bf16_storage, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -86,7 +87,7 @@ def test_bwd_bf16_storage(cuda_device):
     (dq, dk, dv), heads = gpu_fwd_bwd(x, 2, cuda_device, g_dtype=torch.bfloat16, o_dtype=torch.bfloat16)
     dq_r, dk_r, dv_r = oracle_bwd(heads, x["position_ids"], 2)
     for got, ref, nm in ((dq, dq_r, "dQ"), (dk, dk_r, "dK"), (dv, dv_r, "dV")):
-        assert_close(got, ref, f"bwd bf16 storage {nm}", MAX_ABS_BF16, MEAN_REL_BF16)
+        assert_close_bf16_storage(got, ref, f"bwd bf16 storage {nm}")
 
 
 @pytest.mark.parametrize("do_scale", [1e-6, 1e3], ids=["tiny_dO", "large_dO"])

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synthetic
-from gpu_util import (LSE_MAX_ABS, MAX_ABS_BF16, MEAN_REL_BF16, assert_close, assert_lse_close, to_dev_bf16)
+from gpu_util import (LSE_MAX_ABS, assert_close, assert_close_bf16_storage, assert_lse_close, to_dev_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -77,7 +77,7 @@ def test_fwd_bf16_output(cuda_device):
     x = synthetic.custom_inputs(31, 1, 768, 8, 2, 128, lengths=[[500, 268]], with_do=False)
     O, L, heads = gpu_fwd(x, 2, cuda_device, o_dtype=torch.bfloat16)
     O_ref, L_ref = oracle_fwd(heads, x["position_ids"], 2)
-    assert_close(O, O_ref, "fwd bf16 storage O", MAX_ABS_BF16, MEAN_REL_BF16)
+    assert_close_bf16_storage(O, O_ref, "fwd bf16 storage O")
     assert np.abs(L - L_ref).max() <= LSE_MAX_ABS
 
 

@@ -74,77 +74,8 @@ namespace bwd {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// ============================================================================
-// bwd_scale: per-tensor largest magnitude, then fp16 copies scaled by 2^-s
-// ============================================================================
-// Tensor t of {q, k, v, dO}: elements [off[t], off[t] + cnt[t]) (the rows of
-// the selected ranks; both multiples of 8).  Magnitudes are compared as the
-// bf16 bit patterns with the sign cleared, which order like the values
-// (NaN patterns sort above infinity).
-struct ScaleArgs {
-  const uint16_t* src[4];
-  uint16_t* dst[4];     // fp16 copies, same indexing as src
-  int64_t off[4], cnt[4];
-};
-// Targets: the largest magnitude after scaling lies in [2^T, 2^(T+1)).
-__host__ __device__ constexpr int scale_target(int t) { return t < 2 ? 14 : (t == 2 ? 2 : 3); }
-
-// Tensor t's fields, selected without indexing the parameter arrays at run time.
-template <typename T>
-__device__ __forceinline__ T pick(const T (&x)[4], int t) { return t == 0 ? x[0] : t == 1 ? x[1] : t == 2 ? x[2] : x[3]; }
-
-__global__ void __launch_bounds__(256) bwd_absmax_kernel(const ScaleArgs a, uint32_t* __restrict__ amax) {
-  const int t = blockIdx.y;
-  const uint4* src = reinterpret_cast<const uint4*>(pick(a.src, t) + pick(a.off, t));
-  const int64_t nvec = pick(a.cnt, t) / 8;
-  uint32_t m = 0;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec; i += int64_t(gridDim.x) * blockDim.x) {
-    const uint4 v = src[i];
-    m = __vmaxu2(m, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                             __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
-  }
-  m = max(m & 0xFFFFu, m >> 16);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax + t, m);
-}
-
-// Shift s of a tensor whose largest magnitude has bf16 bits `bits`: the
-// scaled maximum 2^(ilogb(max) - s) is 2^T.  All-zero and non-finite
-// tensors keep s = 0; s is clamped so 2^-s stays a normal float.
-__device__ __forceinline__ int scale_shift(uint32_t bits, int target) {
-  if (bits == 0 || bits >= 0x7F80u) return 0;
-  const int e = int(bits >> 7);
-  const int ilog = e > 0 ? e - 127 : (31 - __clz(int(bits & 0x7Fu))) - 133;
-  const int sh = ilog - target;
-  return sh < -120 ? -120 : (sh > 120 ? 120 : sh);
-}
-
-__global__ void __launch_bounds__(256) bwd_to_f16_kernel(const ScaleArgs a, const uint32_t* __restrict__ amax,
-                                                         int32_t* __restrict__ shifts) {
-  const int t = blockIdx.y;
-  const int sh = scale_shift(amax[t], scale_target(t));
-  if (blockIdx.x == 0 && threadIdx.x == 0) shifts[t] = sh;
-  const float f = __int_as_float((127 - sh) << 23);   // 2^-sh
-  const uint4* src = reinterpret_cast<const uint4*>(pick(a.src, t) + pick(a.off, t));
-  uint4* dst = reinterpret_cast<uint4*>(pick(a.dst, t) + pick(a.off, t));
-  const int64_t nvec = pick(a.cnt, t) / 8;
-  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec; i += int64_t(gridDim.x) * blockDim.x) {
-    const uint4 v = src[i];
-    uint4 o;
-    o.x = pack_f16x2(__uint_as_float(v.x << 16) * f, __uint_as_float(v.x & 0xFFFF0000u) * f);
-    o.y = pack_f16x2(__uint_as_float(v.y << 16) * f, __uint_as_float(v.y & 0xFFFF0000u) * f);
-    o.z = pack_f16x2(__uint_as_float(v.z << 16) * f, __uint_as_float(v.z & 0xFFFF0000u) * f);
-    o.w = pack_f16x2(__uint_as_float(v.w << 16) * f, __uint_as_float(v.w & 0xFFFF0000u) * f);
-    dst[i] = o;
-  }
-}
-
-// Shifts of q, k, v, dO as written by bwd_to_f16_kernel.
+// Shifts of q, k, v, dO as written by the fp16-copy kernels (f16copy.cu).
 enum { kShQ = 0, kShK = 1, kShV = 2, kShDO = 3 };
-
-// 2^e for a shift e in [-120, 120] (a normal float: built from its exponent field).
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 
 // ============================================================================
 // bwd_pre: D = rowsum(dO * O) and LSE*log2(e), one warp per (rank, row, head)
@@ -222,7 +153,7 @@ constexpr int kRegsLo = DKDV_REGS_LO, kRegsHi = DKDV_REGS_HI;
 struct Params {
   const int32_t* segend;
   const float* stats;    // see stats_index
-  const int32_t* shifts; // q, k, v, dO scale shifts (bwd_to_f16_kernel)
+  const int32_t* shifts; // q, k, v, dO scale shifts (launch_f16_copies)
   void* dk;              // [P*b][k_rows][hkv][D]
   void* dv;
   int* status;
@@ -645,7 +576,7 @@ constexpr int kThreads = 384;
 struct Params {
   const int32_t* segstart;
   const float* stats;    // see stats_index
-  const int32_t* shifts; // q, k, v, dO scale shifts (bwd_to_f16_kernel)
+  const int32_t* shifts; // q, k, v, dO scale shifts (launch_f16_copies)
   void* dq;              // [P*b][q_rows][hq][D]
   int* status;
   int64_t n, n_pad;      // tokens of the whole sequence; the statistics table's rows (q_rows rounded up)
@@ -1055,26 +986,23 @@ static uly_status attn_bwd_impl(const void* q_head, const void* k_head, const vo
   const int64_t rank0 = rank < 0 ? 0 : rank;
   const int64_t rb0 = rank0 * s.b, nrb = P_sel * s.b;
   {
-    // fp16 copies of the selected ranks' rows, each scaled by its own power of two
-    bwd::ScaleArgs a;
+    // fp16 copies of the selected ranks' rows, each scaled by its own power of
+    // two: q, k to [2^14, 2^15), v to [4, 8), dO to [8, 16) (dP' - D' in range)
+    F16Copies a;
     const void* srcs[4] = {q_head, k_head, v_head, do_head};
     uint16_t* dsts[4] = {q16, k16, v16, do16};
     const int64_t heads[4] = {hq, hkv, hkv, hq};
     const int64_t nrows[4] = {qr, kr, kr, qr};
-    int64_t most = 0;
+    const int32_t targets[4] = {14, 14, 2, 3};
+    a.count = 4;
     for (int t = 0; t < 4; ++t) {
       a.src[t] = static_cast<const uint16_t*>(srcs[t]);
       a.dst[t] = dsts[t];
       a.off[t] = rb0 * nrows[t] * heads[t] * s.d;
       a.cnt[t] = nrb * nrows[t] * heads[t] * s.d;
-      most = a.cnt[t] > most ? a.cnt[t] : most;
+      a.target[t] = targets[t];
     }
-    // a few waves of 256-thread blocks per tensor; each thread strides over 16-byte vectors
-    const int64_t want = (most / 8 + 255) / 256;
-    const unsigned gx = unsigned(want < 4 * 148 ? (want > 0 ? want : 1) : 4 * 148);
-    if (cudaMemsetAsync(amax, 0, 4 * sizeof(uint32_t), cs) != cudaSuccess) return ULY_ERR_CUDA;
-    bwd::bwd_absmax_kernel<<<dim3(gx, 4), 256, 0, cs>>>(a, amax);
-    bwd::bwd_to_f16_kernel<<<dim3(gx, 4), 256, 0, cs>>>(a, amax, shifts);
+    if (launch_f16_copies(a, amax, shifts, cs) != cudaSuccess) return ULY_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return ULY_ERR_CUDA;
   }
   const int64_t qelems = Pb * qr * hq * s.d;                       // Q-side buffer elements

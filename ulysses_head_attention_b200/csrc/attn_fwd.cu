@@ -55,6 +55,14 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when t
 #endif
 constexpr int kMufuPairs = FWD_MUFU_PAIRS;  // of the 64 column pairs per row, the rest use exp2_poly
 
+// P as the A operand of PV: fp16 (11 significant bits, V read from its scaled
+// fp16 copy) in the workspace forward; bf16 with bf16 V in the no-workspace
+// forward, which has no room for a V copy.
+template <bool kF16>
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+  return kF16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+}
+
 struct Params {
   const int32_t* segstart;   // [b][n]
   float* lse;                // [P][b][hq][q_rows]
@@ -69,6 +77,7 @@ struct Params {
   int32_t o_f32;
   uint64_t limit_ns;
   int64_t o_elems, lse_elems, ss_elems;   // buffer extents, for the debug build's bounds checks
+  const int32_t* v_shift;    // fp16 P: V' = V 2^-s, s here (written by the copy kernel); null for bf16 P
 };
 
 template <int D>
@@ -118,7 +127,7 @@ __device__ __forceinline__ TileRange tile_range(const int32_t* ss, int64_t q_bas
   return tr;
 }
 
-template <int D>
+template <int D, bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                 const __grid_constant__ CUtensorMap mv, const Params p) {
@@ -221,7 +230,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer (whole warp, elected lane issues)
       const uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
-      const uint32_t idesc_o = idesc_bf16(BM, D, false, true);
+      const uint32_t idesc_o = kF16 ? idesc_f16(BM, D, false, true) : idesc_bf16(BM, D, false, true);
       bool ok = mbar_wait_warp(&bars->q_full, 0, abort_flag, p.status, p.limit_ns);
       int npv[2] = {0, 0};
       for (int it = 0; ok && it <= nkv; ++it) {
@@ -371,19 +380,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           const int c2 = 32 * half + c;
           float e0, e1;
           f2_unpack(f2_fma(f2_pack(x[2 * c2], x[2 * c2 + 1]), sl2, nms2), e0, e1);
-          if (c2 < kMufuPairs) {
-            e0 = ex2_approx(e0);
-            e1 = ex2_approx(e1);
-          } else {
-            e0 = exp2_poly(e0);
-            e1 = exp2_poly(e1);
+#ifdef FWD_EX2_F16X2
+          if (kF16 && c2 < kMufuPairs) {   // one MUFU op for both exponentials, in fp16
+            pk[c] = ex2_f16x2(pack_f16x2(e0, e1));
+            unpack_f16x2(pk[c], e0, e1);
+          } else
+#endif
+          {
+            if (c2 < kMufuPairs) {
+              e0 = ex2_approx(e0);
+              e1 = ex2_approx(e1);
+            } else {
+              e0 = exp2_poly(e0);
+              e1 = exp2_poly(e1);
+            }
+            pk[c] = pack_p<kF16>(e0, e1);
           }
           const uint64_t ee = f2_pack(e0, e1);
           if ((c & 3) == 0) sum0 = f2_add(sum0, ee);
           else if ((c & 3) == 1) sum1 = f2_add(sum1, ee);
           else if ((c & 3) == 2) sum2 = f2_add(sum2, ee);
           else sum3 = f2_add(sum3, ee);
-          pk[c] = pack_bf16x2(e0, e1);
         }
         tmem_st32(tS + lane_off + 32 * half, pk);
       }
@@ -397,7 +414,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
     // ---- epilogue: O / l and LSE
     if (ntile > 0 && mbar_wait(&bars->o_final[q], 0, abort_flag, p.status, p.limit_ns) && ok && !*abort_flag) {
       tc_fence_after();
-      const float inv_l = row_vis ? 1.f / l : 0.f;   // a row that saw no key gets O = 0
+      // a row that saw no key gets O = 0; the fp16 path folds V's scale 2^s back in
+      const float inv_l = row_vis ? (kF16 ? pow2i(*p.v_shift) : 1.f) / l : 0.f;
       const int64_t orow = (int64_t(rb) * p.q_rows + il) * p.hq + j;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
@@ -458,10 +476,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   }
 }
 
-template <int D>
+template <int D, bool kF16>
 cudaError_t launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const Params& p,
                    int64_t grid, cudaStream_t s) {
-  auto kern = attn_fwd_kernel<D>;
+  auto kern = attn_fwd_kernel<D, kF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<D>::kDynamic);
   if (e != cudaSuccess) return e;
   kern<<<unsigned(grid), kThreads, Layout<D>::kDynamic, s>>>(mq, mk, mv, p);
@@ -496,20 +514,32 @@ uly_status validate_attn(const void* q, const void* k, const void* v, const int6
 
 using namespace uly;
 
+// Forward workspace: the segment tables (seg_workspace_bytes; bytes 64-67 of
+// the status block hold V's largest magnitude, 96-99 its shift), then the
+// scaled fp16 copy of V in the head layout, 256-byte aligned.
+static size_t fwd_v_copy_bytes(const uly_shape* s) {
+  return (size_t(s->P) * size_t(s->b) * size_t(s->n) * size_t(kv_heads_per_rank(*s)) * size_t(s->d) * 2 + 255) &
+         ~size_t(255);
+}
+
 extern "C" size_t ulysses_attn_fwd_workspace(const uly_shape* s) {
   if (check_shape(s) != ULY_OK) return 0;
-  return seg_workspace_bytes(s->b, s->n);
+  return seg_workspace_bytes(s->b, s->n) + fwd_v_copy_bytes(s);
 }
 
 // k_lo, k_hi: the key range attended ([0, n) for the plain forward).  rows:
 // the global rows the Q / O / LSE buffers and the K / V buffers hold (the
 // whole sequence for the head-layout calls, one block for the block calls).
+// f16_p: P and V enter the PV product as fp16 (V from a scaled fp16 copy in
+// the workspace); otherwise as bf16 (the no-workspace forward).
 static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const void* v_head,
                                 const int64_t* position_ids, const uly_shape* shape, int32_t rank,
                                 float softmax_scale, int64_t k_lo, int64_t k_hi, const RowBlocks& rows,
-                                void* o_head, uly_dtype o_dtype, float* lse, void* ws, size_t ws_bytes, void* stream) {
-  uly_status st = validate_attn(q_head, k_head, v_head, position_ids, shape, rank, ws, ws_bytes,
-                                shape ? ulysses_attn_fwd_workspace(shape) : 0);
+                                void* o_head, uly_dtype o_dtype, float* lse, void* ws, size_t ws_bytes, void* stream,
+                                bool f16_p = true) {
+  const size_t need = shape == nullptr || check_shape(shape) != ULY_OK ? 0
+                      : f16_p ? ulysses_attn_fwd_workspace(shape) : seg_workspace_bytes(shape->b, shape->n);
+  uly_status st = validate_attn(q_head, k_head, v_head, position_ids, shape, rank, ws, ws_bytes, need);
   if (st != ULY_OK) return st;
   if (!rows_ok(rows, shape->n, fwd::BM)) return ULY_ERR_INVALID_ARG;
   if (k_lo < rows.k_base || k_hi <= k_lo || k_hi > rows.k_base + rows.k_rows) return ULY_ERR_INVALID_ARG;
@@ -532,18 +562,34 @@ static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const vo
       overlaps(o_head, obytes, ws, ws_bytes))
     return ULY_ERR_INVALID_ARG;
 
-  CUtensorMap mq, mk, mv;
-  if (!make_head_map(&mq, q_head, Pb, rows.q_rows, hq, s.d, fwd::BM) ||
-      !make_head_map(&mk, k_head, Pb, rows.k_rows, hkv, s.d, fwd::BN) ||
-      !make_head_map(&mv, v_head, Pb, rows.k_rows, hkv, s.d, fwd::BN))
-    return ULY_ERR_CUDA;
+  if (overlaps(ws, ws_bytes, q_head, qbytes) || overlaps(ws, ws_bytes, k_head, kvbytes) ||
+      overlaps(ws, ws_bytes, v_head, kvbytes))
+    return ULY_ERR_INVALID_ARG;   // the workspace receives a copy of V
 
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* v16 = reinterpret_cast<uint16_t*>(wsb + seg_workspace_bytes(s.b, s.n));
+  int32_t* v_shift = reinterpret_cast<int32_t*>(wsb + 96);
+  CUtensorMap mq, mk, mv;
+  if (!make_head_map(&mq, q_head, Pb, rows.q_rows, hq, s.d, fwd::BM) ||
+      !make_head_map(&mk, k_head, Pb, rows.k_rows, hkv, s.d, fwd::BN) ||
+      !make_head_map(&mv, f16_p ? static_cast<const void*>(v16) : v_head, Pb, rows.k_rows, hkv, s.d, fwd::BN))
+    return ULY_ERR_CUDA;
   int32_t* segstart = reinterpret_cast<int32_t*>(wsb + 256);
   int32_t* segend = reinterpret_cast<int32_t*>(wsb + 256 + ((size_t(s.b) * size_t(s.n) * 4 + 255) & ~size_t(255)));
   cudaError_t e = launch_segments(position_ids, segstart, segend, s.b, s.n, cs);
   if (e != cudaSuccess) return ULY_ERR_CUDA;
+  if (f16_p) {   // V' = V 2^-s in fp16, the selected ranks' rows, largest magnitude in [2^14, 2^15)
+    F16Copies a{};
+    const int64_t rb0 = int64_t(rank < 0 ? 0 : rank) * s.b, nrb = int64_t(rank < 0 ? s.P : 1) * s.b;
+    a.src[0] = static_cast<const uint16_t*>(v_head);
+    a.dst[0] = v16;
+    a.off[0] = rb0 * rows.k_rows * hkv * s.d;
+    a.cnt[0] = nrb * rows.k_rows * hkv * s.d;
+    a.target[0] = 14;
+    a.count = 1;
+    if (launch_f16_copies(a, reinterpret_cast<uint32_t*>(wsb + 64), v_shift, cs) != cudaSuccess) return ULY_ERR_CUDA;
+  }
 
   fwd::Params p;
   p.segstart = segstart;
@@ -568,10 +614,14 @@ static uly_status attn_fwd_impl(const void* q_head, const void* k_head, const vo
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o_f32 = o_dtype == ULY_F32;
   p.limit_ns = 2000000000ull;
+  p.v_shift = f16_p ? v_shift : nullptr;
   p.o_elems = Pb * rows.q_rows * hq * s.d;
   p.lse_elems = Pb * hq * rows.q_rows;
   p.ss_elems = s.b * s.n;
-  e = s.d == 128 ? fwd::launch<128>(mq, mk, mv, p, grid, cs) : fwd::launch<64>(mq, mk, mv, p, grid, cs);
+  if (f16_p)
+    e = s.d == 128 ? fwd::launch<128, true>(mq, mk, mv, p, grid, cs) : fwd::launch<64, true>(mq, mk, mv, p, grid, cs);
+  else
+    e = s.d == 128 ? fwd::launch<128, false>(mq, mk, mv, p, grid, cs) : fwd::launch<64, false>(mq, mk, mv, p, grid, cs);
   return cuda_status(e);
 }
 
@@ -654,13 +704,15 @@ extern "C" uly_status ulysses_attn_fwd_noalloc(const void* q_head, const void* k
   const uly_status sst = check_shape(shape);
   if (sst != ULY_OK) return sst;
   // Sizes beyond the fixed scratch are refused before anything is enqueued.
-  if (ulysses_attn_fwd_workspace(shape) > kNoAllocScratchBytes) return ULY_ERR_WORKSPACE;
+  if (seg_workspace_bytes(shape->b, shape->n) > kNoAllocScratchBytes) return ULY_ERR_WORKSPACE;
   void* scratch = nullptr;
   const uly_status st = scratch_on_current_device(&scratch);
   if (st != ULY_OK) return st;
   // Nothing in the scratch has to start at zero: every call rewrites both
   // segment tables before reading them, and the status word is only written
   // (on a pipeline timeout), never read, on this path.
-  return ulysses_attn_fwd(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, o_head, o_dtype, lse,
-                          scratch, kNoAllocScratchBytes, stream);
+  // The scratch holds the segment tables only, so P and V enter the PV
+  // product as bf16 (no room for the fp16 copy of V the workspace forward uses).
+  return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, 0, shape->n,
+                       whole_rows(shape->n), o_head, o_dtype, lse, scratch, kNoAllocScratchBytes, stream, false);
 }

@@ -56,6 +56,31 @@ inline int64_t group_per_rank(const uly_shape& s) { return (s.h_q / s.P) / kv_he
 
 inline uly_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ULY_OK : ULY_ERR_CUDA; }
 
+// fp16 copies of up to four bf16 tensors (f16copy.cu): tensor t's elements
+// [off[t], off[t] + cnt[t]) (multiples of 8) of src[t] go, scaled by 2^-s_t,
+// to the same elements of dst[t]; s_t puts the tensor's largest magnitude in
+// [2^target[t], 2^(target[t]+1)).  amax (count words) receives the largest
+// magnitudes as bf16 bits and shifts (count words) the s_t; both device memory.
+struct F16Copies {
+  const uint16_t* src[4];
+  uint16_t* dst[4];
+  int64_t off[4], cnt[4];
+  int32_t target[4];
+  int32_t count;
+};
+cudaError_t launch_f16_copies(const F16Copies& a, uint32_t* amax, int32_t* shifts, cudaStream_t s);
+
+// 2^e for a shift e in [-120, 120] (a normal float: built from its exponent field).
+__host__ __device__ __forceinline__ float pow2i(int e) {
+#ifdef __CUDA_ARCH__
+  return __int_as_float((e + 127) << 23);
+#else
+  union { uint32_t u; float f; } x;
+  x.u = uint32_t(e + 127) << 23;
+  return x.f;
+#endif
+}
+
 // The global sequence rows the attention buffers hold: Q (and O, LSE, dO,
 // dQ) rows [q_base, q_base + q_rows), K (and V, dK, dV) rows
 // [k_base, k_base + k_rows).  The head-layout calls pass the whole sequence;
