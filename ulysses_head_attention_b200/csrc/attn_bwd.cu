@@ -454,14 +454,26 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           const float2 nl = *reinterpret_cast<const float2*>(stt + j);   // -LSE*log2e
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(s0), __uint_as_float(s1)), sl2, f2_pack(nl.x, nl.y)), x0, x1);
+#ifdef BWD_EX2_F16X2
+          // both exponentials in one MUFU operation, in fp16 (the precision P^T is stored in)
+          uint32_t ph = ex2_f16x2(pack_f16x2(x0, x1));
+          if (need_mask) {
+            if (unsigned(j - lo) >= unsigned(hi - lo)) ph &= 0xFFFF0000u;
+            if (unsigned(j + 1 - lo) >= unsigned(hi - lo)) ph &= 0x0000FFFFu;
+          }
+          float p0, p1;
+          unpack_f16x2(ph, p0, p1);
+          pw[c] = ph;
+#else
           float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           if (need_mask) {
             if (unsigned(j - lo) >= unsigned(hi - lo)) p0 = 0.f;
             if (unsigned(j + 1 - lo) >= unsigned(hi - lo)) p1 = 0.f;
           }
+          pw[c] = pack_f16x2(p0, p1);
+#endif
           pr[j] = p0;
           pr[j + 1] = p1;
-          pw[c] = pack_f16x2(p0, p1);
         }
       }
       if (!mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
@@ -818,7 +830,12 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const uint32_t db = c < 16 ? d0[2 * c + 1] : d1[2 * c - 31];
         float xa, xb;
         f2_unpack(f2_fma(f2_pack(__uint_as_float(sa), __uint_as_float(sb)), sl2, nl2), xa, xb);
+#ifdef BWD_EX2_F16X2
+        float pa, pb;
+        unpack_f16x2(ex2_f16x2(pack_f16x2(xa, xb)), pa, pb);   // one MUFU operation, fp16 precision
+#else
         float pa = ex2_approx(xa), pb = ex2_approx(xb);
+#endif
         if (need_mask) {
           if (unsigned(2 * c - lo) >= unsigned(hi - lo)) pa = 0.f;
           if (unsigned(2 * c + 1 - lo) >= unsigned(hi - lo)) pb = 0.f;
