@@ -379,3 +379,44 @@ def test_debug_build_exports_the_same_symbols():
     for n in header_functions():
         assert hasattr(d, n), n
 
+
+@no_gpu
+def test_layer_step_host_rejects():
+    import ulysses_head_attention_b200 as uly
+    f = uly.lib.ulysses_layer_step_host
+    s = shape()
+    need = uly.lib.ulysses_layer_step_host_bytes(ctypes.byref(s))
+    assert need > 0 and uly.lib.ulysses_layer_step_host_bytes(ctypes.byref(shape(n=1001))) == 0
+    ev = (ctypes.c_void_p * 3)(F, F + 64, F + 128)
+    host = [F + (i + 1) * (1 << 30) for i in range(9)]
+
+    def call(dev=F + (20 << 30), dev_bytes=need, events=ev, sh=s):
+        return f(*host[:5], ctypes.byref(sh), 0.0, *host[5:], dev, dev_bytes, None, None, None, events)
+    assert call(dev_bytes=need - 1) == WORKSPACE            # device buffer too small
+    assert call(dev=F + (20 << 30) + 16) == WORKSPACE       # not 256-byte aligned
+    assert call(events=None) == INVALID                      # no ordering events
+    assert call(events=(ctypes.c_void_p * 3)(F, 0, F)) == INVALID
+    assert call(sh=shape(n=1001)) == INVALID                 # n % P
+
+
+@no_gpu
+def test_block_calls_and_accumulate_reject():
+    import ulysses_head_attention_b200 as uly
+    G = 1 << 30
+    s = shape(b=1, n=4096, hq=8, hkv=2, d=128, P=1)
+    ws = uly.lib.ulysses_attn_fwd_workspace(ctypes.byref(s))
+    fb = uly.lib.ulysses_attn_fwd_block
+
+    def fwd(q_base, q_rows, k_base, k_rows):
+        return fb(F, F + G, F + 2 * G, F + 3 * G, ctypes.byref(s), q_base, q_rows, k_base, k_rows, 0.0,
+                  F + 4 * G, 1, F + 5 * G, F + 6 * G, ws, None)
+    assert fwd(64, 128, 0, 128) == INVALID         # query block off a tile edge
+    assert fwd(0, 128, 100, 128) == INVALID        # key block off a tile edge
+    assert fwd(4096, 128, 0, 128) == INVALID       # query block past the sequence
+    assert fwd(0, 128, 3968, 256) == INVALID       # key block past the sequence
+    assert fwd(0, 0, 0, 128) == INVALID            # empty block
+    acc = uly.lib.ulysses_accumulate
+    assert acc(F, F + G, 6, None) == INVALID       # not a multiple of 4
+    assert acc(F, F + 64, 1024, None) == INVALID   # overlapping, not identical
+    assert acc(F + 4, F + G, 8, None) == INVALID   # misaligned
+
