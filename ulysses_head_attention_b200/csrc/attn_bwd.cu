@@ -583,7 +583,17 @@ constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int NSK = 3;   // K ring: a K tile is read by S and, one step later, by dQ
 constexpr int NSV = 2;   // V ring: read by dP only
-constexpr int kThreads = 384;
+#ifndef DQ_NWG
+#define DQ_NWG 2
+#endif
+constexpr int kNWG = DQ_NWG;           // softmax warpgroups, each taking kCW key columns of a tile
+constexpr int kCW = BN / kNWG;
+constexpr int kThreads = 128 + 128 * kNWG;
+static_assert(kNWG == 2 || kNWG == 4, "two or four softmax warpgroups");
+// with four softmax warpgroups (640 threads, 96 registers each at launch) the
+// first warpgroup hands registers to the softmax warpgroups
+constexpr int kRegsLo = 56, kRegsHi = 104;
+static_assert(kNWG == 2 || 128 * kRegsLo + 512 * kRegsHi <= 640 * 96, "register split over budget");
 
 struct Params {
   const int32_t* segstart;
@@ -671,10 +681,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->ds_ready[s], 256);
+      mbar_init(&bars->ds_ready[s], 128 * kNWG);
     }
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->dp_free, 256);
+    mbar_init(&bars->dp_free, 128 * kNWG);
     mbar_init(&bars->mma_final, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -691,6 +701,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
   const uint32_t tDP = tmem + 256, tDQ = tmem + 384;
 
   if (warp == 0 || warp == 2) {
+    if constexpr (kNWG > 2) regs_split_n<kRegsLo, kRegsHi, kThreads, 96>(false);
     // producers: warp 0 loads Q, dO and the K ring, warp 2 the V ring, so a
     // K load never waits behind a V stage that is still being read
     if (lane == 0) {
@@ -729,6 +740,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       }
     }
   } else if (warp == 1) {
+    if constexpr (kNWG > 2) regs_split_n<kRegsLo, kRegsHi, kThreads, 96>(false);
     {   // whole warp; the elected lane issues
       const uint32_t id_s = idesc_f16(BM, BN, false, false);
       const uint32_t id_q = idesc_f16(BM, D, false, true);
@@ -742,9 +754,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         const uint32_t k_addr = smem_u32(smem + L::oK + st * L::kTile);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // dS of keys [16kk, 16kk+16): the first 64 keys' bf16 pairs sit in S
-          // columns [0,32), the last 64 keys' in [64,96) (one half per warpgroup).
-          const uint32_t a_col = kk < 4 ? kk * 8 : 64 + (kk - 4) * 8;
+          // dS of keys [16kk, 16kk+16): warpgroup w's kCW keys sit, as fp16
+          // pairs, in the first kCW/2 of its own kCW S columns
+          const uint32_t a_col = kCW * ((16 * kk) / kCW) + 8 * (kk % (kCW / 16));
           umma_ts_warp(tDQ, tS(b) + a_col, sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), id_q,
                   (jt > 0 || kk > 0) ? 1u : 0u);
         }
@@ -778,8 +790,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       if (ok && nkv > 0) issue_dq(nkv - 1);
       umma_commit_warp(&bars->mma_final);
     }
+  } else if (warp == 3) {
+    if constexpr (kNWG > 2) regs_split_n<kRegsLo, kRegsHi, kThreads, 96>(false);
   } else if (warp >= 4) {
-    const int wg = (warp - 4) >> 2;                 // column half handled by this warpgroup
+    if constexpr (kNWG > 2) regs_split_n<kRegsLo, kRegsHi, kThreads, 96>(true);
+    const int wg = (warp - 4) >> 2;                 // key columns [kCW wg, kCW wg + kCW) of every tile
     const int row = ((warp - 4) & 3) * 32 + lane;
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t i = t0 + row;                  // global row
@@ -801,33 +816,33 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
     bool ok = true;
     for (int it = 0; it < nkv; ++it) {
       const int b = it & 1;
-      const int64_t k0 = int64_t(kv_first + it) * BN + 64 * wg;   // first key column of this warpgroup
+      const int64_t k0 = int64_t(kv_first + it) * BN + kCW * wg;   // first key column of this warpgroup
       if (!mbar_wait(&bars->s_full[b], (it >> 1) & 1, abort_flag, p.status, p.limit_ns) ||
           !mbar_wait(&bars->dp_full, it & 1, abort_flag, p.status, p.limit_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t s0[32], s1[32], d0[32], d1[32];
-      tmem_ld32(tS(b) + lane_off + 64 * wg, s0);
-      tmem_ld32(tS(b) + lane_off + 64 * wg + 32, s1);
-      tmem_ld32(tDP + lane_off + 64 * wg, d0);
-      tmem_ld32(tDP + lane_off + 64 * wg + 32, d1);
+      constexpr int NC = kCW / 32;   // 32-column chunks of this warpgroup
+      uint32_t sv[NC][32], dv_[NC][32];
+#pragma unroll
+      for (int ch = 0; ch < NC; ++ch) {
+        tmem_ld32(tS(b) + lane_off + kCW * wg + 32 * ch, sv[ch]);
+        tmem_ld32(tDP + lane_off + kCW * wg + 32 * ch, dv_[ch]);
+      }
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->dp_free);
       // visible key columns c of this warpgroup: lo <= c < hi (keys row_lo .. row_hi - 1)
       const int64_t lo64 = row_lo - k0, hi64 = valid ? row_hi - k0 : lo64;
-      const bool need_mask = lo64 > 0 || hi64 < 64;
-      const int lo = int(lo64 < 0 ? 0 : (lo64 > 64 ? 64 : lo64));
-      const int hi = int(hi64 < lo ? lo : (hi64 > 64 ? 64 : hi64));
-      uint32_t w[32];
+      const bool need_mask = lo64 > 0 || hi64 < kCW;
+      const int lo = int(lo64 < 0 ? 0 : (lo64 > kCW ? kCW : lo64));
+      const int hi = int(hi64 < lo ? lo : (hi64 > kCW ? kCW : hi64));
+      uint32_t w[kCW / 2];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const uint32_t sa = c < 16 ? s0[2 * c] : s1[2 * c - 32];
-        const uint32_t sb = c < 16 ? s0[2 * c + 1] : s1[2 * c - 31];
-        const uint32_t da = c < 16 ? d0[2 * c] : d1[2 * c - 32];
-        const uint32_t db = c < 16 ? d0[2 * c + 1] : d1[2 * c - 31];
+      for (int c = 0; c < kCW / 2; ++c) {
+        const uint32_t sa = sv[(2 * c) / 32][(2 * c) % 32], sb = sv[(2 * c) / 32][(2 * c + 1) % 32];
+        const uint32_t da = dv_[(2 * c) / 32][(2 * c) % 32], db = dv_[(2 * c) / 32][(2 * c + 1) % 32];
         float xa, xb;
         f2_unpack(f2_fma(f2_pack(__uint_as_float(sa), __uint_as_float(sb)), sl2, nl2), xa, xb);
 #ifdef BWD_EX2_F16X2
@@ -844,7 +859,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         f2_unpack(f2_mul(f2_pack(pa, pb), f2_add(f2_pack(__uint_as_float(da), __uint_as_float(db)), nd2)), ga, gb);
         w[c] = pack_f16x2(ga, gb);
       }
-      tmem_st32(tS(b) + lane_off + 64 * wg, w);
+      if constexpr (kCW == 64) {
+        tmem_st32(tS(b) + lane_off + kCW * wg, w);
+      } else {
+        tmem_st16(tS(b) + lane_off + kCW * wg, w);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->ds_ready[b]);
@@ -855,10 +874,11 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
       const bool store = valid && in_bounds(orow >= 0 && (orow + 1) * D <= p.g_elems, p.status);
       // dQ' = dS' k' = scale^-1 dQ 2^-(sdo+sv+sk)
       const float mq = p.scale * pow2i(p.shifts[kShDO]) * pow2i(p.shifts[kShV]) * pow2i(p.shifts[kShK]);
-      for (int c = 64 * wg; c < D; c += 128) {
-        // warpgroup wg stores head-dim columns [64 wg, 64 wg + 64) (D = 64: wg 0 only)
+      for (int c = kCW * wg; c < D; c += 128) {
+        // warpgroup wg stores head-dim columns [kCW wg, kCW wg + kCW) (and the
+        // same 128 further on); a warpgroup past D stores nothing
 #pragma unroll
-        for (int c2 = 0; c2 < 64; c2 += 32) {
+        for (int c2 = 0; c2 < kCW; c2 += 32) {
           uint32_t o[32];
           tmem_ld32(tDQ + lane_off + c + c2, o);
           tmem_ld_wait();

@@ -297,6 +297,15 @@ __device__ __forceinline__ void regs_split(bool softmax_warpgroup) {
   else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(LO) : "memory");
 }
 
+// The same for NT threads launched at RL registers each: the first warpgroup
+// takes LO, the other NT - 128 threads HI, with 128 LO + (NT - 128) HI <= NT RL.
+template <int LO, int HI, int NT, int RL>
+__device__ __forceinline__ void regs_split_n(bool softmax_warpgroup) {
+  static_assert(LO % 8 == 0 && HI % 8 == 0 && 128 * LO + (NT - 128) * HI <= NT * RL, "register split over budget");
+  if (softmax_warpgroup) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(HI) : "memory");
+  else asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(LO) : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // tcgen05: TMEM <-> registers (warp-collective; warp w touches lanes 32*(w%4)..)
 // ----------------------------------------------------------------------------
