@@ -13,6 +13,7 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200) and the built library")
     config.addinivalue_line("markers", "large: full-size workload parity (slow)")
+    config.addinivalue_line("markers", "oracle_heavy: minutes of fp64 oracle work on the host (n = 131072 in full)")
 
 
 def read_golden(name):

@@ -10,8 +10,9 @@ Compared against the fp64 oracle, element by element (tolerances as
 everywhere: every element within 1e-2, sum|g-r|/sum|r| <= 2e-3 for
 fp32-stored values, LSE max-abs <= 1e-3):
   * every element of O, LSE and dQ of all G query heads of one kv group and
-    of that kv head's dK and dV, at full size (the Llama-8B shape and the
-    packed SFT batch; the oracle's per-head work runs in parallel processes);
+    of that kv head's dK and dV, at full size (the Llama-8B shape, the packed
+    SFT batch and the n = 131072 round trip; the oracle's per-head work runs
+    in parallel processes);
   * O and LSE of sampled query rows of every head (rows 0 and n-1, the first
     and last row of random 128-row tiles, random rows), each against its
     full visible prefix;
@@ -186,6 +187,17 @@ def test_workload_layer(cuda_device, name):
     check_forward(w, x, out, rng, rows_per_head=24)
     if w.backward:
         check_backward(w, x, out, rng, rows_per_head=12)
+
+
+@pytest.mark.oracle_heavy
+def test_roundtrip_full_kv_group_0(cuda_device):
+    """The full layer round trip at n = 131072: every element of O, LSE, dQ of
+    kv group 0's four query heads and of kv head 0's dK, dV against the
+    oracle (about 5e13 flops of fp64 on the host, spread over its cores)."""
+    w = synthetic.WORKLOADS["roundtrip_p4_n128k"]
+    x = synthetic.make_inputs(w)
+    out = run_layer(w, x, cuda_device, backward=True)
+    check_full_group(w, x, out, 0)
 
 
 def test_workload_long_context_rank_by_rank(cuda_device):
