@@ -142,11 +142,19 @@ constexpr int BQ = 128;    // query rows per inner tile (N = 128 MMAs)
 // latency every step); dO and the row statistics live one step less.
 constexpr int NSQ = 3;     // Q stages
 constexpr int NSO = 2;     // dO + row-statistics stages
-constexpr int kThreads = 384;
+#ifndef DKDV_NWG
+#define DKDV_NWG 2
+#endif
+constexpr int kNWG = DKDV_NWG;         // softmax warpgroups, each taking kCW query columns of a tile
+constexpr int kCW = BQ / kNWG;
+constexpr int kThreads = 128 + 128 * kNWG;
+static_assert(kNWG == 2 || kNWG == 4, "two or four softmax warpgroups");
 constexpr uint32_t kSmemOptin = 232448;   // per-CTA dynamic shared memory limit (227 KB)
+// register split: 384 threads at 168 registers, or 640 at 96
+constexpr int kRegsLaunch = kNWG == 2 ? 168 : 96;
 #ifndef DKDV_REGS_LO
 #define DKDV_REGS_LO 72
-#define DKDV_REGS_HI 216
+#define DKDV_REGS_HI (DKDV_NWG == 2 ? 216 : 96)
 #endif
 constexpr int kRegsLo = DKDV_REGS_LO, kRegsHi = DKDV_REGS_HI;
 
@@ -261,9 +269,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->x_free, 256);
-    mbar_init(&bars->p_ready, 256);
-    mbar_init(&bars->ds_ready, 256);
+    mbar_init(&bars->x_free, 128 * kNWG);
+    mbar_init(&bars->p_ready, 128 * kNWG);
+    mbar_init(&bars->ds_ready, 128 * kNWG);
     mbar_init(&bars->mma_final, 1);
     bars->abort_flag = 0;
     bars->score_scale = p.scale_log2 * pow2i(p.shifts[kShQ]) * pow2i(p.shifts[kShK]);
@@ -281,7 +289,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 
 
   if (warp < 4) {
-  regs_split<kRegsLo, kRegsHi>(false);   // producers, MMA issuer, idle warp 3
+  regs_split_n<kRegsLo, kRegsHi, kThreads, kRegsLaunch>(false);   // producers, MMA issuer, idle warp 3
   if (warp == 0 || warp == 2) {
     // producers: warp 0 loads K, V and the Q ring, warp 2 the dO + statistics
     // ring, so neither ring's loads wait behind the other's free slots
@@ -406,8 +414,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     }
   }
   } else {
-    regs_split<kRegsLo, kRegsHi>(true);   // softmax warpgroups and epilogue
-    const int wg = (warp - 4) >> 2;                  // query columns [64 wg, 64 wg + 64) of each tile
+    regs_split_n<kRegsLo, kRegsHi, kThreads, kRegsLaunch>(true);   // softmax warpgroups and epilogue
+    const int wg = (warp - 4) >> 2;                  // query columns [kCW wg, kCW wg + kCW) of each tile
     const int row = ((warp - 4) & 3) * 32 + lane;    // key row within the tile
     const uint32_t lane_off = uint32_t(((warp - 4) & 3) * 32) << 16;
     const int64_t kj = k0 + row;
@@ -429,28 +437,31 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
         break;
       }
       tc_fence_after();
-      // this warpgroup's 64 columns are statistics block wg: {64 x -LSE*log2e, 64 x -D}
-      const float* stt = reinterpret_cast<const float*>(smem + L::oSt + st * L::kSt) + 128 * wg;
+      // this warpgroup's query columns [c0, c0 + kCW) sit in statistics block
+      // c0 / 64 ({64 x -LSE*log2e, 64 x -D}) from offset c0 % 64
+      constexpr int NC = kCW / 32;   // 32-column chunks of this warpgroup
+      const int c0 = kCW * wg;
+      const float* stt = reinterpret_cast<const float*>(smem + L::oSt + st * L::kSt) + 128 * (c0 / 64) + (c0 % 64);
       // visible query columns c of this warpgroup: lo <= c < hi (queries kj .. kj_end-1)
-      const int64_t qb = q0 + 64 * wg;
+      const int64_t qb = q0 + c0;
       const int64_t lo64 = kj - qb, hi64 = kj_end - qb;
-      const bool need_mask = lo64 > 0 || hi64 < 64;
-      const int lo = int(lo64 < 0 ? 0 : (lo64 > 64 ? 64 : lo64));
-      const int hi = int(hi64 < lo ? lo : (hi64 > 64 ? 64 : hi64));
-      float pr[64];
-      uint32_t pw[32];
+      const bool need_mask = lo64 > 0 || hi64 < kCW;
+      const int lo = int(lo64 < 0 ? 0 : (lo64 > kCW ? kCW : lo64));
+      const int hi = int(hi64 < lo ? lo : (hi64 > kCW ? kCW : hi64));
+      float pr[kCW];
+      uint32_t pw[kCW / 2];
       {
-        // both S^T chunks in one round trip, then X may be rewritten
-        uint32_t sv0[32], sv1[32];
-        tmem_ld32(tX + lane_off + 64 * wg, sv0);
-        tmem_ld32(tX + lane_off + 64 * wg + 32, sv1);
+        // all S^T chunks in one round trip, then X may be rewritten
+        uint32_t sv[NC][32];
+#pragma unroll
+        for (int ch = 0; ch < NC; ++ch) tmem_ld32(tX + lane_off + c0 + 32 * ch, sv[ch]);
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&bars->x_free);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
+        for (int c = 0; c < kCW / 2; ++c) {
           const int j = 2 * c;
-          const uint32_t s0 = c < 16 ? sv0[j] : sv1[j - 32], s1 = c < 16 ? sv0[j + 1] : sv1[j - 31];
+          const uint32_t s0 = sv[j / 32][j % 32], s1 = sv[j / 32][(j + 1) % 32];
           const float2 nl = *reinterpret_cast<const float2*>(stt + j);   // -LSE*log2e
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(s0), __uint_as_float(s1)), sl2, f2_pack(nl.x, nl.y)), x0, x1);
@@ -482,39 +493,37 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       }
       tc_fence_after();
       {
-        uint32_t dp0[32], dp1[32];
-        tmem_ld32(tY + lane_off + 64 * wg, dp0);
-        tmem_ld32(tY + lane_off + 64 * wg + 32, dp1);
+        uint32_t dp[NC][32];
+#pragma unroll
+        for (int ch = 0; ch < NC; ++ch) tmem_ld32(tY + lane_off + c0 + 32 * ch, dp[ch]);
         tmem_ld_wait();
         // each 32-query chunk goes back over the 32 columns it came from:
         // 16 columns of P^T, then 16 of dS^T.  P^T first, so dV can start
         // while dS is computed.
-        {
+#pragma unroll
+        for (int ch = 0; ch < NC; ++ch) {
           uint32_t pc[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) pc[c] = pw[c];
-          tmem_st16(tY + lane_off + 64 * wg, pc);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) pc[c] = pw[16 + c];
-          tmem_st16(tY + lane_off + 64 * wg + 32, pc);
+          for (int c = 0; c < 16; ++c) pc[c] = pw[16 * ch + c];
+          tmem_st16(tY + lane_off + c0 + 32 * ch, pc);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
+        for (int ch = 0; ch < NC; ++ch) {
           uint32_t dw[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int j = 32 * ch + 2 * c;
-            const uint32_t a0 = ch == 0 ? dp0[2 * c] : dp1[2 * c], a1 = ch == 0 ? dp0[2 * c + 1] : dp1[2 * c + 1];
+            const uint32_t a0 = dp[ch][2 * c], a1 = dp[ch][2 * c + 1];
             const float2 nd = *reinterpret_cast<const float2*>(stt + 64 + j);   // -D
             float d0, d1;
             f2_unpack(f2_mul(f2_pack(pr[j], pr[j + 1]),
                              f2_add(f2_pack(__uint_as_float(a0), __uint_as_float(a1)), f2_pack(nd.x, nd.y))), d0, d1);
             dw[c] = pack_f16x2(d0, d1);
           }
-          tmem_st16(tY + lane_off + 64 * wg + 32 * ch + 16, dw);
+          tmem_st16(tY + lane_off + c0 + 32 * ch + 16, dw);
         }
       }
       tmem_st_wait();
@@ -526,14 +535,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       const int64_t orow = (int64_t(rb) * p.k_rows + (kj - p.k_base)) * p.hkv + g;
       const bool valid = kj < k_end && in_bounds(orow >= 0 && (orow + 1) * D <= p.g_elems, p.status);
       {
-        const int which = wg;   // warpgroup 0 stores dK, warpgroup 1 stores dV
+        // the first half of the warpgroups stores dK, the second dV, each
+        // warpgroup D / (kNWG / 2) of the head-dim columns
+        const int which = wg / (kNWG / 2);
+        const int cbeg = (wg % (kNWG / 2)) * (D / (kNWG / 2)), cend = cbeg + D / (kNWG / 2);
         const uint32_t base = which == 0 ? tDK : tDV;
         // dK' = dS'^T q' = scale^-1 dK 2^-(sdo+sv+sq), dV' = P^T dO' = dV 2^-sdo
         const float mul = which == 0 ? p.scale * pow2i(p.shifts[kShDO]) * pow2i(p.shifts[kShV]) * pow2i(p.shifts[kShQ])
                                      : pow2i(p.shifts[kShDO]);
         void* out = which == 0 ? p.dk : p.dv;
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        for (int c = cbeg; c < cend; c += 32) {
           uint32_t o[32];
           tmem_ld32(base + lane_off + c, o);
           tmem_ld_wait();
