@@ -473,9 +473,10 @@ uly_status ulysses_ipc_close(void* dev_ptr);
  *   outputs  o_seq, dq_seq [P][b][n/P][h_q][d] float; dk_seq, dv_seq
  *            [P][b][n/P][h_kv][d] float: host memory, page-locked
  *   dev      caller-owned device memory of ulysses_layer_step_host_bytes()
- *            bytes, 256-byte aligned (ULY_ERR_WORKSPACE otherwise): device
- *            staging, head-layout buffers and both attention workspaces;
- *            reused by every call with the same shape
+ *            bytes, 256-byte aligned (ULY_ERR_WORKSPACE otherwise), zeroed
+ *            once before the first call (it holds the attention workspaces'
+ *            status words): device staging, head-layout buffers and both
+ *            attention workspaces; reused by every call with the same shape
  *   streams  `stream` runs the kernels, `h2d_stream` the host-to-device and
  *            `d2h_stream` the device-to-host copies (three distinct streams
  *            of the current device)

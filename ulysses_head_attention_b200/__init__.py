@@ -608,7 +608,8 @@ class LayerStepHost:
         nbytes = int(lib.ulysses_layer_step_host_bytes(ctypes.byref(self.shape)))
         if nbytes == 0:
             raise ValueError("shape not accepted by the library")
-        self.dev = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        # zeroed once: the attention workspaces' status words inside it start clear
+        self.dev = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         self.h2d, self.d2h = torch.cuda.Stream(self.device), torch.cuda.Stream(self.device)
         self.events = [torch.cuda.Event() for _ in range(3)]
 

@@ -54,6 +54,11 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when t
 #define FWD_MUFU_PAIRS 48
 #endif
 constexpr int kMufuPairs = FWD_MUFU_PAIRS;  // of the 64 column pairs per row, the rest use exp2_poly
+#ifndef FWD_REGS_LO
+#define FWD_REGS_LO 72
+#define FWD_REGS_HI 216
+#endif
+constexpr int kRegsLo = FWD_REGS_LO, kRegsHi = FWD_REGS_HI;   // producer/MMA warpgroup, softmax warpgroups
 
 // P as the A operand of PV: fp16 (11 significant bits, V read from its scaled
 // fp16 copy) in the workspace forward; bf16 with bf16 V in the no-workspace
@@ -189,7 +194,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
   const uint32_t tmem = bars->tmem_base;
 
   if (warp < 4) {
-    regs_split<72, 216>(false);
+    regs_split<kRegsLo, kRegsHi>(false);
     if ((warp == 0 || warp == 2) && lane == 0) {
       // ---------------------------------------------------------- producers
       const bool is_k = warp == 0;
@@ -286,7 +291,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       umma_commit_warp(&bars->o_final[1]);
     }
   } else {
-    regs_split<72, 216>(true);
+    regs_split<kRegsLo, kRegsHi>(true);
     // ------------------------------------------------------------ softmax
     const int q = (warp - 4) >> 2;                     // query tile of this warpgroup
     const TileRange tr = q ? tr1 : tr0;
