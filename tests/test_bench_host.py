@@ -92,7 +92,8 @@ def test_recorded_traffic_applies_only_to_its_workload_and_sources(monkeypatch):
     monkeypatch.setitem(bench.TRAFFIC, "attn_bwd_dkdv_kernel", rec)
     assert bench.recorded_traffic("attn_bwd_dkdv_kernel", rec["workload"]) == rec["bytes_per_launch"]
     assert bench.recorded_traffic("attn_bwd_dkdv_kernel", "llama8b_p4_n32k") is None
-    assert bench.recorded_traffic("attn_bwd_dq_kernel", rec["workload"]) is None
+    monkeypatch.delitem(bench.TRAFFIC, "attn_bwd_dq_kernel", raising=False)
+    assert bench.recorded_traffic("attn_bwd_dq_kernel", rec["workload"]) is None   # no record
     # once the kernel's sources differ from the ones the counters were taken on
     monkeypatch.setitem(bench.TRAFFIC, "attn_bwd_dkdv_kernel", dict(rec, sources_sha256="0" * 64))
     assert bench.recorded_traffic("attn_bwd_dkdv_kernel", rec["workload"]) is None
