@@ -30,11 +30,15 @@ def test_kernel_constants_are_the_fit():
     m = _fit_module()
     c = m.fit(3)                                   # c0 + c1 f + c2 f^2 + c3 f^3
     text = open(os.path.join(CSRC, "sm100.cuh")).read()
-    body = text[text.index("float exp2_poly(float x)"):]
-    body = body[:body.index("return __int_as_float")]
-    nums = [np.float32(float(x)) for x in re.findall(r"([0-9]+\.[0-9]+)f", body) if float(x) < 10.0]
-    # Horner order in the kernel: c3, c2 (first fmaf), then c1, then c0
-    assert nums == [np.float32(c[3]), np.float32(c[2]), np.float32(c[1]), np.float32(c[0])], (nums, c)
+    found = {int(i): np.float32(float(v)) for i, v in re.findall(r"kExp2PolyC([0-3]) = ([0-9]+\.[0-9]+)f;", text)}
+    assert found == {i: np.float32(c[i]) for i in range(4)}, (found, c)
+    # both the scalar and the packed evaluation use the named constants, in Horner order
+    for fn in ("float exp2_poly(float x)", "uint64_t exp2_poly2(uint64_t x2)"):
+        body = text[text.index(fn):]
+        body = body[:body.index("return ")]
+        assert not re.findall(r"0\.[0-9]{5,}f", body), fn
+        order = [int(x) for x in re.findall(r"kExp2PolyC([0-3])", body)]
+        assert [x for i, x in enumerate(order) if i == 0 or x != order[i - 1]] == [3, 2, 1, 0], (fn, order)
 
 
 def test_fit_meets_its_error_bound_in_float32():

@@ -149,6 +149,12 @@ constexpr int kNWG = DKDV_NWG;         // softmax warpgroups, each taking kCW qu
 constexpr int kCW = BQ / kNWG;
 constexpr int kThreads = 128 + 128 * kNWG;
 static_assert(kNWG == 2 || kNWG == 4, "two or four softmax warpgroups");
+// of each thread's kCW / 2 column pairs per tile, the first kMufuPairs take
+// their exponentials on the MUFU unit, the rest on the FMA pipe (exp2_poly)
+#ifndef DKDV_MUFU_PAIRS
+#define DKDV_MUFU_PAIRS 32
+#endif
+constexpr int kMufuPairs = DKDV_MUFU_PAIRS < kCW / 2 ? DKDV_MUFU_PAIRS : kCW / 2;
 constexpr uint32_t kSmemOptin = 232448;   // per-CTA dynamic shared memory limit (227 KB)
 // register split: 384 threads at 168 registers, or 640 at 96
 constexpr int kRegsLaunch = kNWG == 2 ? 168 : 96;
@@ -476,7 +482,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           unpack_f16x2(ph, p0, p1);
           pw[c] = ph;
 #else
-          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          float p0, p1;
+          if (c < kMufuPairs) {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          } else {
+            f2_unpack(exp2_poly2(f2_pack(x0, x1)), p0, p1);
+          }
           if (need_mask) {
             if (unsigned(j - lo) >= unsigned(hi - lo)) p0 = 0.f;
             if (unsigned(j + 1 - lo) >= unsigned(hi - lo)) p1 = 0.f;
@@ -602,6 +614,12 @@ constexpr int kNWG = DQ_NWG;           // softmax warpgroups, each taking kCW ke
 constexpr int kCW = BN / kNWG;
 constexpr int kThreads = 128 + 128 * kNWG;
 static_assert(kNWG == 2 || kNWG == 4, "two or four softmax warpgroups");
+// exponentials of the first kMufuPairs column pairs on MUFU, the rest on the
+// FMA pipe (exp2_poly)
+#ifndef DQ_MUFU_PAIRS
+#define DQ_MUFU_PAIRS 32
+#endif
+constexpr int kMufuPairs = DQ_MUFU_PAIRS < kCW / 2 ? DQ_MUFU_PAIRS : kCW / 2;
 // with four softmax warpgroups (640 threads, 96 registers each at launch) the
 // first warpgroup hands registers to the softmax warpgroups
 constexpr int kRegsLo = 56, kRegsHi = 104;
@@ -861,7 +879,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant
         float pa, pb;
         unpack_f16x2(ex2_f16x2(pack_f16x2(xa, xb)), pa, pb);   // one MUFU operation, fp16 precision
 #else
-        float pa = ex2_approx(xa), pb = ex2_approx(xb);
+        float pa, pb;
+        if (c < kMufuPairs) {
+          pa = ex2_approx(xa);
+          pb = ex2_approx(xb);
+        } else {
+          f2_unpack(exp2_poly2(f2_pack(xa, xb)), pa, pb);
+        }
 #endif
         if (need_mask) {
           if (unsigned(2 * c - lo) >= unsigned(hi - lo)) pa = 0.f;

@@ -47,7 +47,11 @@ namespace fwd {
 
 constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // keys per tile
-constexpr int NS = 2;          // K/V stages
+#ifndef FWD_NSK
+#define FWD_NSK 2
+#endif
+constexpr int NSK = FWD_NSK;   // K stages
+constexpr int NSV = 2;         // V stages
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 #ifndef FWD_MUFU_PAIRS
@@ -90,15 +94,16 @@ struct Layout {
   static constexpr uint32_t kTileBytes = BM * D * 2;   // a Q, K or V tile
   static constexpr uint32_t kQ = 0;                     // two query tiles
   static constexpr uint32_t kK = kQ + 2 * kTileBytes;
-  static constexpr uint32_t kV = kK + NS * kTileBytes;
-  static constexpr uint32_t kBar = kV + NS * kTileBytes;
+  static constexpr uint32_t kV = kK + NSK * kTileBytes;
+  static constexpr uint32_t kBar = kV + NSV * kTileBytes;
   static constexpr uint32_t kBytes = kBar + 256;
   static constexpr uint32_t kDynamic = kBytes + 1024;  // alignment slack
+  static_assert(kDynamic <= 232448, "dynamic shared memory above the per-CTA limit");
 };
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[NS], v_full[NS], k_empty[NS], v_empty[NS];
+  uint64_t k_full[NSK], k_empty[NSK], v_full[NSV], v_empty[NSV];
   uint64_t s_full[2], p_full[2];
   uint64_t o_final[2];
   uint32_t tmem_base;
@@ -170,10 +175,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
+      mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -202,6 +209,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       uint64_t* full = is_k ? bars->k_full : bars->v_full;
       uint64_t* empty = is_k ? bars->k_empty : bars->v_empty;
       const uint32_t base = is_k ? L::kK : L::kV;
+      const int ns = is_k ? NSK : NSV;
       tma_prefetch_desc(map);
       if (is_k) {
         tma_prefetch_desc(&mq);
@@ -216,7 +224,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       }
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
-        const int st = it % NS, rnd = it / NS;
+        const int st = it % ns, rnd = it / ns;
         const int k0 = (j_lo + it) * BN;
         if (rnd > 0 && !mbar_wait(&empty[st], (rnd - 1) & 1, abort_flag, p.status, p.limit_ns)) break;
         mbar_arrive_expect_tx(&full[st], L::kTileBytes);
@@ -229,8 +237,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       // Error path only: let every copy this thread started land before exit.
       if (*abort_flag) {
         if (is_k) mbar_wait(&bars->q_full, 0, nullptr, nullptr, p.limit_ns);
-        for (int x = max(0, issued - NS); x < issued; ++x)
-          mbar_wait(&full[x % NS], (x / NS) & 1, nullptr, nullptr, p.limit_ns);
+        for (int x = max(0, issued - ns); x < issued; ++x)
+          mbar_wait(&full[x % ns], (x / ns) & 1, nullptr, nullptr, p.limit_ns);
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer (whole warp, elected lane issues)
@@ -251,11 +259,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           // stage waits ride along with tile 0's P wait.
           if (do_pv && !mbar_wait_warp(&bars->p_full[q], npv[q] & 1, abort_flag, p.status, p.limit_ns)) { ok = false; break; }
           if (q == 0) {
-            if (it >= 1 && !mbar_wait_warp(&bars->v_full[(it - 1) % NS], ((it - 1) / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+            if (it >= 1 && !mbar_wait_warp(&bars->v_full[(it - 1) % NSV], ((it - 1) / NSV) & 1, abort_flag, p.status, p.limit_ns)) {
               ok = false;
               break;
             }
-            if (it < nkv && !mbar_wait_warp(&bars->k_full[it % NS], (it / NS) & 1, abort_flag, p.status, p.limit_ns)) {
+            if (it < nkv && !mbar_wait_warp(&bars->k_full[it % NSK], (it / NSK) & 1, abort_flag, p.status, p.limit_ns)) {
               ok = false;
               break;
             }
@@ -265,7 +273,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           // Descriptors: base once, then + compile-time offsets (16-byte units)
           // so the issue loop is a few instructions per MMA.
           if (do_pv) {
-            const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::kV + ((it - 1) % NS) * L::kTileBytes), BN * 128, 1024);
+            const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::kV + ((it - 1) % NSV) * L::kTileBytes), BN * 128, 1024);
             umma_ts_warp(tO, tS, v_desc, idesc_o, npv[q] > 0 ? 1u : 0u);
 #pragma unroll
             for (int kk = 1; kk < BN / 16; ++kk)
@@ -274,7 +282,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           }
           if (do_s) {
             const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::kQ + q * L::kTileBytes), 16, 1024);
-            const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::kK + (it % NS) * L::kTileBytes), 16, 1024);
+            const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::kK + (it % NSK) * L::kTileBytes), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t off = uint64_t(((kk >> 2) * (BM * 128) + (kk & 3) * 32) / 16);
@@ -284,8 +292,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
           }
         }
         if (!ok) break;
-        if (it >= 1) umma_commit_warp(&bars->v_empty[(it - 1) % NS]);
-        if (it < nkv) umma_commit_warp(&bars->k_empty[it % NS]);
+        if (it >= 1) umma_commit_warp(&bars->v_empty[(it - 1) % NSV]);
+        if (it < nkv) umma_commit_warp(&bars->k_empty[it % NSK]);
       }
       umma_commit_warp(&bars->o_final[0]);
       umma_commit_warp(&bars->o_final[1]);
@@ -383,21 +391,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const int c2 = 32 * half + c;
+          const uint64_t xx = f2_fma(f2_pack(x[2 * c2], x[2 * c2 + 1]), sl2, nms2);
           float e0, e1;
-          f2_unpack(f2_fma(f2_pack(x[2 * c2], x[2 * c2 + 1]), sl2, nms2), e0, e1);
 #ifdef FWD_EX2_F16X2
           if (kF16 && c2 < kMufuPairs) {   // one MUFU op for both exponentials, in fp16
+            f2_unpack(xx, e0, e1);
             pk[c] = ex2_f16x2(pack_f16x2(e0, e1));
             unpack_f16x2(pk[c], e0, e1);
           } else
 #endif
           {
             if (c2 < kMufuPairs) {
+              f2_unpack(xx, e0, e1);
               e0 = ex2_approx(e0);
               e1 = ex2_approx(e1);
             } else {
-              e0 = exp2_poly(e0);
-              e1 = exp2_poly(e1);
+              f2_unpack(exp2_poly2(xx), e0, e1);
             }
             pk[c] = pack_p<kF16>(e0, e1);
           }

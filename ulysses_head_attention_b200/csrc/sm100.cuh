@@ -428,14 +428,40 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // (Lawson's iteratively reweighted least squares; fit_exp2_poly.py next to
 // this file derives the coefficients): max relative error 7.5e-5 in fp32.
 // x is clamped at -125, so anything smaller returns about 2^-125 instead of 0.
+constexpr float kExp2PolyC3 = 0.05517167f;   // p(f) = ((c3 f + c2) f + c1) f + c0
+constexpr float kExp2PolyC2 = 0.24261114f;
+constexpr float kExp2PolyC1 = 0.69326097f;
+constexpr float kExp2PolyC0 = 0.99992806f;
+constexpr float kExp2Round = 12582912.f;     // 1.5 * 2^23
+
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float q = fmaf(0.05517167f, f, 0.24261114f);
-  q = fmaf(q, f, 0.69326097f);
-  q = fmaf(q, f, 0.99992806f);
+  const float t = x + kExp2Round;
+  const float f = x - (t - kExp2Round);
+  float q = fmaf(kExp2PolyC3, f, kExp2PolyC2);
+  q = fmaf(q, f, kExp2PolyC1);
+  q = fmaf(q, f, kExp2PolyC0);
   return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
+// exp2_poly of both halves of a packed pair, with the same operations in
+// packed f32x2 form (bitwise the same results): about 10 instructions for
+// the pair instead of 18.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x2, f2_pack(kExp2Round, kExp2Round));
+  const uint64_t u = f2_add(t, f2_pack(-kExp2Round, -kExp2Round));   // t - 1.5 * 2^23, exact
+  const uint64_t f = f2_fma(u, f2_pack(-1.f, -1.f), x2);             // x - u, one rounding
+  uint64_t q = f2_fma(f2_pack(kExp2PolyC3, kExp2PolyC3), f, f2_pack(kExp2PolyC2, kExp2PolyC2));
+  q = f2_fma(q, f, f2_pack(kExp2PolyC1, kExp2PolyC1));
+  q = f2_fma(q, f, f2_pack(kExp2PolyC0, kExp2PolyC0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23)));
 }
 
 __device__ __forceinline__ int elect_one_lane() { return (threadIdx.x & 31) == 0; }
