@@ -55,12 +55,7 @@ KERNEL_SOURCES = {
                         ("ulysses_head_attention_b200/csrc/common.cuh", None, None)),
 }
 # kernel -> {"workload", "bytes_per_launch", "sources_sha256"}
-TRAFFIC = {
-    "attn_bwd_dkdv_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 8994435840 + 1071717120,
-                             "sources_sha256": "7f39a808ffac3abe106eb1dd018460e21cbdb55469b8209c792360dfbc48c91a"},
-    "attn_bwd_dq_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 5660910336 + 2108599552,
-                           "sources_sha256": "d2f00097a5ae6330ff3dc76d37fc5220f699e1eef921b82007ac0bae09fa47ab"},
-}
+TRAFFIC = {}
 
 
 def sources_sha256(kernel: str) -> str:
