@@ -512,9 +512,12 @@ def run_ours(args, w):
             f, s = oracle_sample(w, x, rows, heads)
             flops += f
             secs += s
-        out["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+        cpu_tf = flops / secs / 1e12
+        out["cpu_baseline"] = {"value": cpu_tf, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
                                "kind": "oracle",
-                               "sample": f"4 x oracle fwd+bwd of the last {rows} query rows of {heads} heads"}
+                               "sample": f"4 x oracle fwd+bwd of the last {rows} query rows of {heads} heads",
+                               # the whole step's algorithmic work at the sample's rate (not run)
+                               "extrapolated_step_s": (layer.fwd_flops + layer.bwd_flops) / (cpu_tf * 1e12)}
     if reports(rank):
         print(json.dumps(out))
     if world > 1:
