@@ -51,7 +51,10 @@ constexpr int BN = 128;        // keys per tile
 #define FWD_NSK 2
 #endif
 constexpr int NSK = FWD_NSK;   // K stages
-constexpr int NSV = 2;         // V stages
+#ifndef FWD_NSV
+#define FWD_NSV 2
+#endif
+constexpr int NSV = FWD_NSV;   // V stages
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 #ifndef FWD_MUFU_PAIRS
