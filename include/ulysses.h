@@ -168,6 +168,11 @@ size_t ulysses_attn_fwd_workspace(const uly_shape* shape);
  *   ws / ws_bytes: device workspace of at least ulysses_attn_fwd_workspace()
  *   bytes, 256-byte aligned (else ULY_ERR_WORKSPACE).
  * Supports d in {64, 128} (else ULY_ERR_UNSUPPORTED).
+ * Arithmetic: S = q k^T from the bf16 inputs with float32 accumulation; the
+ * softmax in float32; P rounded to fp16 for P V, against an fp16 copy of v
+ * scaled by a power of two (held in the workspace; the scale is folded back
+ * exactly); O accumulated in float32.  No atomics: results are bitwise
+ * reproducible from call to call.
  */
 uly_status ulysses_attn_fwd(const void* q_head, const void* k_head, const void* v_head,
                             const int64_t* position_ids, const uly_shape* shape, int32_t rank,
@@ -189,6 +194,11 @@ size_t ulysses_attn_bwd_workspace(const uly_shape* shape, uly_dtype g_dtype);
  * outputs (o_dtype must match); do_head has q_head's layout (bf16).
  * Outputs dq_head (q_head's layout), dk_head / dv_head (k_head's layout), of
  * g_dtype.  rank / softmax_scale as for the forward.
+ * Arithmetic: the products take fp16 copies of q, k, v and dO, each scaled by
+ * a power of two chosen from its largest magnitude (exact; folded back into
+ * the results); P and dS are rounded to fp16 before they enter dV, dK and
+ * dQ; all accumulation is float32.  No atomics: results are bitwise
+ * reproducible from call to call.
  */
 uly_status ulysses_attn_bwd(const void* q_head, const void* k_head, const void* v_head,
                             const void* o_head, uly_dtype o_dtype, const float* lse,
