@@ -55,7 +55,14 @@ KERNEL_SOURCES = {
                         ("ulysses_head_attention_b200/csrc/common.cuh", None, None)),
 }
 # kernel -> {"workload", "bytes_per_launch", "sources_sha256"}
-TRAFFIC = {}
+TRAFFIC = {
+    "attn_bwd_dkdv_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 10064423424,
+                            "sources_sha256": "dff1888c5a93bb3fb7da54891c28636fff3fb1d093d6810d892025827f9eeaea"},
+    "attn_bwd_dq_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 7764684288,
+                          "sources_sha256": "f92c9d5fccec072838f206836a167345d7f35ac885823a480f515ec27b22d589"},
+    "attn_fwd_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 5569199616,
+                       "sources_sha256": "2b83b143e8d89efa3e51cc91275bb5ea3ee9dee80f1982e9db756b6db86acdfa"},
+}
 
 
 def sources_sha256(kernel: str) -> str:
@@ -474,7 +481,8 @@ def run_ours(args, w):
                     "frac_of_clock_peak": dom_tf / cpk if cpk else None,
                     "flops_per_launch": k_flops[dom], "ms_per_launch": k_ms[dom],
                     "kernel_tflops": {kn: k_flops[kn] / (k_ms[kn] * 1e-3) / 1e12 for kn in k_ms},
-                    "traffic": recorded_traffic(dom, w.name)}
+                    "traffic": recorded_traffic(dom, w.name),
+                    "kernel_traffic": {kn: recorded_traffic(kn, w.name) for kn in k_ms}}
     else:
         roofline = None
 
@@ -594,54 +602,85 @@ def measure_configs(args, w_main, dev, uly, peaks, clocks):
 
 
 def measure_ring(layer, dev):
-    """Ring attention over R key blocks (forward + LSE merge, then the blocks'
-    backward from the merged O / LSE), timed on its own."""
+    """Ring attention as the ring driver computes it (ring.LibraryOps: block
+    forward, LSE merge, block backward, accumulate) over R = 4 sequence
+    blocks of every virtual Ulysses rank's head slice, the ranks one after
+    another on this GPU: the ring's computation without its exchange (the
+    composition of Ulysses over heads with a ring over the sequence)."""
     import torch
-    if not layer.w.backward:
-        return {}
-    uly, h, w = layer.uly, layer.head, layer.w
-    R, n, f32 = 4, w.n, torch.float32
-    cuts = [n * i // R for i in range(R + 1)]
-    o_parts = torch.empty((R,) + tuple(layer.o_head.shape), dtype=f32, device=dev)
-    l_parts = torch.empty((R,) + tuple(layer.lse.shape), dtype=f32, device=dev)
-    o_ring, l_ring = torch.empty_like(layer.o_head), torch.empty_like(layer.lse)
-    g_ring = {k: torch.empty_like(layer.g_head[k]) for k in layer.g_head}
+    from ulysses_head_attention_b200.ring import LibraryOps
+    w, h = layer.w, layer.head
+    R = 4
+    P, b, n, hq_r, d = h["q"].shape
+    hkv_r = h["k"].shape[3]
+    if not w.backward or b != 1 or n % (R * 128):
+        return {}   # blocks are row ranges of whole 128-row tiles, contiguous only for b = 1
+    m, f32 = n // R, torch.float32
+    ops = LibraryOps()
+
+    def blocks(t):   # [p][r]: rows [r m, (r + 1) m) of rank p, block layout (1, b, m, heads, d)
+        return [[t[p:p + 1, :, r * m:(r + 1) * m] for r in range(R)] for p in range(P)]
+
+    Q, K, V, DO = blocks(h["q"]), blocks(h["k"]), blocks(h["v"]), blocks(h["do"])
+    o_parts = torch.empty((R, 1, b, m, hq_r, d), dtype=f32, device=dev)
+    l_parts = torch.empty((R, 1, b, hq_r, m), dtype=f32, device=dev)
+    o_blk = torch.empty((P, R, 1, b, m, hq_r, d), dtype=f32, device=dev)   # merged O, LSE per (rank, block)
+    l_blk = torch.empty((P, R, 1, b, hq_r, m), dtype=f32, device=dev)
+    dq = torch.empty((1, b, m, hq_r, d), dtype=f32, device=dev)
+    share_q = torch.empty_like(dq)
+    share_k = torch.empty((1, b, m, hkv_r, d), dtype=f32, device=dev)
+    share_v = torch.empty_like(share_k)
+    acc_k = torch.empty((R, 1, b, m, hkv_r, d), dtype=f32, device=dev)   # key blocks' dK, dV accumulators
+    acc_v = torch.empty_like(acc_k)
+    calls = {"fwd_block": 0, "merge": 0, "bwd_block": 0, "accumulate": 0}
 
     def ring_fwd():
-        for i in range(R):
-            uly.ulysses_attn_fwd_kv_range(h["q"], h["k"], h["v"], layer.pos, o_parts[i], l_parts[i], layer.ws_f,
-                                          cuts[i], cuts[i + 1])
-        uly.ulysses_attn_lse_merge(o_parts, l_parts, o_ring, l_ring, w.h_kv)
+        for p in range(P):
+            for r in range(R):
+                for s in range(r + 1):   # key blocks at or before the query block
+                    ops.fwd_block(Q[p][r], K[p][s], V[p][s], layer.pos, r * m, s * m, o_parts[s], l_parts[s])
+                ops.merge(o_parts[:r + 1], l_parts[:r + 1], o_blk[p, r], l_blk[p, r], hkv_r)
+                calls["fwd_block"] += r + 1
+                calls["merge"] += 1
 
     def ring_bwd():
-        for i in range(R):
-            uly.ulysses_attn_bwd_kv_range(h["q"], h["k"], h["v"], o_ring, l_ring, h["do"], layer.pos,
-                                          g_ring["q"], g_ring["k"], g_ring["v"], layer.ws_b, cuts[i], cuts[i + 1])
+        for p in range(P):
+            for r in range(R):
+                for s in range(r, -1, -1):
+                    if s == r:   # the diagonal block starts dQ and key block s's accumulators
+                        ops.bwd_block(Q[p][r], K[p][s], V[p][s], o_blk[p, r], l_blk[p, r], DO[p][r], layer.pos,
+                                      r * m, s * m, dq, acc_k[s], acc_v[s])
+                    else:
+                        ops.bwd_block(Q[p][r], K[p][s], V[p][s], o_blk[p, r], l_blk[p, r], DO[p][r], layer.pos,
+                                      r * m, s * m, share_q, share_k, share_v)
+                        ops.accumulate(dq, share_q)
+                        ops.accumulate(acc_k[s], share_k)
+                        ops.accumulate(acc_v[s], share_v)
+                        calls["accumulate"] += 3
+                    calls["bwd_block"] += 1
 
     ring_fwd()
     ring_bwd()
     torch.cuda.synchronize()
-    rf = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    reps = 2
-    rf[0].record()
-    for _ in range(reps):
-        ring_fwd()
-    rf[1].record()
-    for _ in range(reps):
-        ring_bwd()
-    rf[2].record()
+    calls = dict.fromkeys(calls, 0)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    ring_fwd()
+    ev[1].record()
+    ring_bwd()
+    ev[2].record()
     torch.cuda.synchronize()
-    layer.check_status("in the ring measurement")
-    fwd_ms = rf[0].elapsed_time(rf[1]) / reps
-    bwd_ms = rf[1].elapsed_time(rf[2]) / reps
-    del o_parts, l_parts, o_ring, l_ring, g_ring
+    ops.check()
+    fwd_ms, bwd_ms = ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])
+    del o_parts, l_parts, o_blk, l_blk, dq, share_q, share_k, share_v, acc_k, acc_v, ops
     torch.cuda.empty_cache()
     return {"ring_attention": {
-        "blocks": R, "fwd_ms": fwd_ms, "fwd_tflops": layer.fwd_flops / (fwd_ms * 1e-3) / 1e12,
-        "bwd_ms_per_block_pass": bwd_ms, "bwd_tflops": layer.bwd_flops / (bwd_ms * 1e-3) / 1e12,
-        "launches": {"fwd": R * 2 + 1, "bwd": R * 6},
-        "note": "keys cut into R equal blocks; forward = R key-range forwards + one LSE merge; "
-                "backward = R key-range backwards from the merged O and LSE (one block's dQ share each)"}}
+        "blocks": R, "ulysses_ranks": P, "fwd_ms": fwd_ms, "fwd_tflops": layer.fwd_flops / (fwd_ms * 1e-3) / 1e12,
+        "bwd_ms": bwd_ms, "bwd_tflops": layer.bwd_flops / (bwd_ms * 1e-3) / 1e12, "calls": calls,
+        "note": "every virtual Ulysses rank's head slice cut into R sequence blocks; forward = block forwards of "
+                "each query block against the key blocks at or before it + one LSE merge per query block; "
+                "backward = block backwards from the merged O and LSE, dQ and the key blocks' dK, dV summed "
+                "with the accumulate call; ranks run one after another, no exchange"}}
 
 
 def measure_loss(layer, x, dev):
