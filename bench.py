@@ -56,8 +56,6 @@ KERNEL_SOURCES = {
 }
 # kernel -> {"workload", "bytes_per_launch", "sources_sha256"}
 TRAFFIC = {
-    "attn_bwd_dkdv_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 10064423424,
-                            "sources_sha256": "dff1888c5a93bb3fb7da54891c28636fff3fb1d093d6810d892025827f9eeaea"},
     "attn_bwd_dq_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 7764684288,
                           "sources_sha256": "f92c9d5fccec072838f206836a167345d7f35ac885823a480f515ec27b22d589"},
     "attn_fwd_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 5569199616,

@@ -203,6 +203,7 @@ struct Layout {
 struct Bars {
   uint64_t kv_full;
   uint64_t q_full[NSQ], q_empty[NSQ], do_full[NSO], do_empty[NSO];
+  uint64_t st_full[NSO], st_empty[NSO];   // row statistics: loaded by warp 3, released by the softmax
   uint64_t s_full, dp_full, x_free, p_ready, ds_ready;
   uint64_t mma_final;
   uint32_t tmem_base;
@@ -272,6 +273,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
     for (int s = 0; s < NSO; ++s) {
       mbar_init(&bars->do_full[s], 1);
       mbar_init(&bars->do_empty[s], 1);
+      mbar_init(&bars->st_full[s], 1);
+      mbar_init(&bars->st_empty[s], 128 * kNWG);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
@@ -295,16 +298,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
 
 
   if (warp < 4) {
-  regs_split_n<kRegsLo, kRegsHi, kThreads, kRegsLaunch>(false);   // producers, MMA issuer, idle warp 3
-  if (warp == 0 || warp == 2) {
-    // producers: warp 0 loads K, V and the Q ring, warp 2 the dO + statistics
-    // ring, so neither ring's loads wait behind the other's free slots
+  regs_split_n<kRegsLo, kRegsHi, kThreads, kRegsLaunch>(false);   // producers and the MMA issuer
+  if (warp != 1) {
+    // producers, one ring each so that no ring's loads wait behind another's
+    // free slots: warp 0 loads K, V and the Q ring, warp 2 the dO ring (read
+    // by the MMAs only), warp 3 the row-statistics ring (read by the softmax
+    // only, which releases a stage once it has read it)
     if (lane == 0) {
-      const bool is_q = warp == 0;
+      const bool is_q = warp == 0, is_st = warp == 3;
       const int ns = is_q ? NSQ : NSO;
-      uint64_t* full = is_q ? bars->q_full : bars->do_full;
-      uint64_t* empty = is_q ? bars->q_empty : bars->do_empty;
-      tma_prefetch_desc(is_q ? &mq : &mdo);
+      uint64_t* full = is_q ? bars->q_full : (is_st ? bars->st_full : bars->do_full);
+      uint64_t* empty = is_q ? bars->q_empty : (is_st ? bars->st_empty : bars->do_empty);
+      if (!is_st) tma_prefetch_desc(is_q ? &mq : &mdo);
       if (is_q && niter > 0) {
         mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kKV);
         if (in_bounds(k0 - p.k_base >= 0 && k0 - p.k_base < p.k_rows, p.status))
@@ -325,14 +330,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           if (q_in)
             for (int dc = 0; dc < D / 64; ++dc)
               tma_load_4d(&mq, &full[st], smem + L::oQ + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
-        } else {
-          mbar_arrive_expect_tx(&full[st], L::kQ + L::kSt);
+        } else if (is_st) {
+          mbar_arrive_expect_tx(&full[st], L::kSt);
           const int64_t si = stats_index(int64_t(rb) * p.hq + h, p.n_pad, q0);
-          if (q_in && in_bounds(si >= 0 && si + L::kSt / 4 <= p.stats_elems, p.status)) {
+          if (q_in && in_bounds(si >= 0 && si + L::kSt / 4 <= p.stats_elems, p.status))
+            bulk_load(smem + L::oSt + st * L::kSt, p.stats + si, L::kSt, &full[st]);
+        } else {
+          mbar_arrive_expect_tx(&full[st], L::kQ);
+          if (q_in)
             for (int dc = 0; dc < D / 64; ++dc)
               tma_load_4d(&mdo, &full[st], smem + L::oDO + st * L::kQ + dc * BQ * 128, dc * 64, h, q0, rb);
-            bulk_load(smem + L::oSt + st * L::kSt, p.stats + si, L::kSt, &full[st]);
-          }
         }
         issued = it + 1;
       }
@@ -437,7 +444,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
       const float sl = *reinterpret_cast<volatile float*>(&bars->score_scale);
       const uint64_t sl2 = f2_pack(sl, sl);
       const int64_t q0 = int64_t(qt_first + it % nqt) * BQ;
-      if (!mbar_wait(&bars->do_full[st], (it / NSO) & 1, abort_flag, p.status, p.limit_ns) ||
+      if (!mbar_wait(&bars->st_full[st], (it / NSO) & 1, abort_flag, p.status, p.limit_ns) ||
           !mbar_wait(&bars->s_full, it & 1, abort_flag, p.status, p.limit_ns)) {
         ok = false;
         break;
@@ -538,6 +545,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_consta
           tmem_st16(tY + lane_off + c0 + 32 * ch + 16, dw);
         }
       }
+      mbar_arrive(&bars->st_empty[st]);   // this step's statistics are read (release)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars->ds_ready);
