@@ -39,7 +39,8 @@
 //               the G query heads of the kv head and the 128-row query tiles
 //               that can see the key tile:
 //                 warp 0      TMA producer: K, V once; the Q ring (3 stages)
-//                 warp 2      TMA producer: the dO + row-statistics ring (2)
+//                 warp 2      TMA producer: the dO ring (2)
+//                 warp 3      bulk-copy producer: the row-statistics ring (2)
 //                 warp 1      TMEM owner; issues the MMAs as a converged warp
 //                 warps 4..11 thread = key row, two warpgroups each taking
 //                             64 of the 128 query columns
