@@ -56,6 +56,8 @@ KERNEL_SOURCES = {
 }
 # kernel -> {"workload", "bytes_per_launch", "sources_sha256"}
 TRAFFIC = {
+    "attn_bwd_dkdv_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 10050001152,
+                            "sources_sha256": "25ba9ffc0dea0c17d52ac7cfe2889817052ba88dd6947055c6bf0849e6766407"},
     "attn_bwd_dq_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 7764684288,
                           "sources_sha256": "f92c9d5fccec072838f206836a167345d7f35ac885823a480f515ec27b22d589"},
     "attn_fwd_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 5569199616,
