@@ -259,10 +259,12 @@ def run_reference(args, w):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-# Kernel launches of one step: s2h q, k, v (3); forward: segments + attention
-# (2); h2s O (1); s2h dO (1); backward: segments, largest magnitudes, fp16
-# copies, row statistics, dK/dV, dQ (6); h2s dQ, dK, dV (3).
-LAUNCHES_FWD_BWD = 3 + 2 + 1 + 1 + 6 + 3
+# Kernel launches of one step: s2h q, k, v (3); forward: segments, V's
+# largest magnitude, its fp16 copy, attention (4); h2s O (1); s2h dO (1);
+# backward: segments, largest magnitudes, fp16 copies, row statistics, dK/dV,
+# dQ (6); h2s dQ, dK, dV (3).
+LAUNCHES_FWD = 4
+LAUNCHES_FWD_BWD = 3 + LAUNCHES_FWD + 1 + 1 + 6 + 3
 # tcgen05 dense bf16 rate per SM and clock (M = 128, N = 256, K = 16 in 128 cycles)
 TENSOR_FLOP_PER_CLK_SM = 8192
 NUM_SMS = 148
@@ -320,7 +322,7 @@ class Layer:
             self.relayout_bytes += sum(nbytes(self.g_head[k]) + nbytes(self.g_seq[k]) for k in self.g_seq)
         # forward-only workloads run s2h(q, k, v), the forward (rank by rank when
         # asked) and h2s(O)
-        self.launches = LAUNCHES_FWD_BWD if w.backward else 3 + 2 * (P if w.rank_by_rank else 1) + 1
+        self.launches = LAUNCHES_FWD_BWD if w.backward else 3 + LAUNCHES_FWD * (P if w.rank_by_rank else 1) + 1
 
     def step(self, ev=None, kev=None):
         """One pass of the path.  ev: 6 events around its stages; kev: 5 events
@@ -396,6 +398,34 @@ def time_layer(layer, steps: int, warmup: int, clocks, barrier=lambda: None):
               "attn_bwd_dq_kernel": statistics.mean(e[3].elapsed_time(e[4]) for e in kevs)}
     return {"ms_total": start.elapsed_time(end), "stage_ms": st, "kernel_ms": km,
             "clocks": clocks.summary(t0, t1), "seconds": t1 - t0}
+
+
+def time_graph(layer, steps: int) -> float:
+    """The same step captured once as a CUDA graph and replayed `steps` times
+    (ms per step): what the step costs when its launches are submitted as
+    one.  Nothing in the step synchronises or allocates, so it captures as
+    it runs."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer.step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.step()
+    graph.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        graph.replay()
+    end.record()
+    torch.cuda.synchronize()
+    layer.check_status("under graph replay")
+    del graph
+    return start.elapsed_time(end) / steps
 
 
 def clock_peak_tflops(sm_mhz):
@@ -583,6 +613,7 @@ def measure_e2e(layer, steps, barrier, world, dev):
 # the other workloads timed in the same run: (name, steps, warm-up)
 OTHER_CONFIGS = (("tiny_p2_n256", 20, 3), ("llama8b_p4_n32k", 5, 3), ("packed_sft_p8_n64k", 5, 3),
                  ("long_p8_n512k", 2, 1))
+GRAPH_CONFIGS = ("tiny_p2_n256",)   # launch-bound: also timed as a replayed CUDA graph
 
 
 def measure_configs(args, w_main, dev, uly, peaks, clocks):
@@ -596,6 +627,10 @@ def measure_configs(args, w_main, dev, uly, peaks, clocks):
         t = time_layer(lay, steps, warm, clocks)
         t["steps"] = steps
         res[name] = layer_figures(lay, t, peaks)
+        if args.graphs and name in GRAPH_CONFIGS:
+            g_ms = time_graph(lay, steps)
+            res[name]["graph"] = {"ms_per_step": g_ms, "launches_per_step": lay.launches,
+                                  "note": "the step captured once as a CUDA graph, replayed"}
         del lay
         torch.cuda.empty_cache()
     return res
@@ -762,6 +797,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graphs", action="store_true",
+                    help="also time the launch-bound workloads as replayed CUDA graphs")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the separately timed ring-attention and loss-aggregation measurements")
     ap.add_argument("--profile-case", action="store_true",
