@@ -797,8 +797,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--graphs", action="store_true",
-                    help="also time the launch-bound workloads as replayed CUDA graphs")
+    ap.add_argument("--no-graphs", dest="graphs", action="store_false",
+                    help="skip timing the launch-bound workloads as replayed CUDA graphs")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the separately timed ring-attention and loss-aggregation measurements")
     ap.add_argument("--profile-case", action="store_true",
