@@ -613,7 +613,9 @@ def measure_e2e(layer, steps, barrier, world, dev):
 # the other workloads timed in the same run: (name, steps, warm-up)
 OTHER_CONFIGS = (("tiny_p2_n256", 20, 3), ("llama8b_p4_n32k", 5, 3), ("packed_sft_p8_n64k", 5, 3),
                  ("long_p8_n512k", 2, 1))
-GRAPH_CONFIGS = ("tiny_p2_n256",)   # launch-bound: also timed as a replayed CUDA graph
+# also timed as a replayed CUDA graph: the launch-bound workload, and one with
+# the backward (whose step must capture as well)
+GRAPH_CONFIGS = ("tiny_p2_n256", "llama8b_p4_n32k")
 
 
 def measure_configs(args, w_main, dev, uly, peaks, clocks):
