@@ -342,14 +342,27 @@ uly_status ulysses_attn_bwd_timed(const void* q_head, const void* k_head, const 
  *   last call's contents (nothing in it needs to start at zero).  Calls whose
  *   work overlaps on the GPU (e.g. on two concurrently running streams) race
  *   on it and give wrong results: serialise them.
- *   A pipeline timeout inside the kernel is not reported by this call (there
- *   is no workspace to read the status word from); use ulysses_attn_fwd
- *   where that report is needed.
+ *   A pipeline timeout inside the kernel is not reported by this call: the
+ *   kernels record it in the scratch's status word, which
+ *   ulysses_attn_fwd_noalloc_status reads.
  */
 uly_status ulysses_attn_fwd_noalloc(const void* q_head, const void* k_head, const void* v_head,
                                     const int64_t* position_ids, const uly_shape* shape, int32_t rank,
                                     float softmax_scale, void* o_head, uly_dtype o_dtype, float* lse,
                                     void* stream);
+
+/*
+ * ulysses_attn_fwd_noalloc_status -- the status word of the current device's
+ * fixed no-alloc scratch, read and then cleared, as ulysses_workspace_status
+ * does for a workspace: *code = ULY_OK, ULY_ERR_TIMEOUT (a kernel gave up
+ * waiting on its own pipeline since the last read), ULY_ERR_CUDA or
+ * ULY_ERR_BOUNDS.  Enqueues a 4-byte copy and a clear on `stream` and waits
+ * for both (a host synchronisation: not for use under stream capture).  The
+ * word is shared by every no-alloc call on the device, like the scratch.
+ * Returns ULY_ERR_INVALID_ARG for a null code.  The pages have no
+ * counterpart for this call.
+ */
+uly_status ulysses_attn_fwd_noalloc_status(void* stream, int32_t* code);
 
 /*
  * ulysses_sp_loss_aggregate -- weighted loss aggregation across the P SP

@@ -313,6 +313,15 @@ def test_noalloc_forward_refuses_before_touching_the_device():
 
 
 @no_gpu
+def test_noalloc_status_refuses_a_null_code():
+    import ulysses_head_attention_b200 as uly
+    assert uly.lib.ulysses_attn_fwd_noalloc_status(None, None) == INVALID
+    # a valid request stops at the device lookup, which has no device to find here
+    code = ctypes.c_int32(-1)
+    assert uly.lib.ulysses_attn_fwd_noalloc_status(None, ctypes.byref(code)) == CUDA
+
+
+@no_gpu
 def test_selftest_wait_timeout_rejects():
     import ulysses_head_attention_b200 as uly
     f = uly.lib.ulysses_selftest_wait_timeout

@@ -49,6 +49,7 @@ def test_noalloc_matches_workspace_forward_twice(cuda_device):
         uly.ulysses_attn_fwd_noalloc(q, k, v, pos, o_na, l_na)
         torch.cuda.synchronize()
         assert uly.ulysses_workspace_status(ws) == 0
+        assert uly.ulysses_attn_fwd_noalloc_status() == 0   # the scratch's status word: no timeout
         assert_close(o_na.cpu().numpy(), o_ws.cpu().numpy(), f"noalloc O (n={n})")
         assert np.abs(l_na.cpu().numpy() - l_ws.cpu().numpy()).max() <= LSE_MAX_ABS
 

@@ -34,6 +34,7 @@ STATUS_NAMES = {0: "ULY_OK", 1: "ULY_ERR_INVALID_ARG", 2: "ULY_ERR_UNSUPPORTED",
 EXPORTS = ("ulysses_seq_to_head", "ulysses_head_to_seq", "ulysses_kv_seq_to_head", "ulysses_kv_head_to_seq",
            "ulysses_transpose_runs", "ulysses_attn_fwd_workspace", "ulysses_attn_fwd",
            "ulysses_attn_bwd_workspace", "ulysses_attn_bwd", "ulysses_attn_bwd_timed", "ulysses_attn_fwd_noalloc",
+           "ulysses_attn_fwd_noalloc_status",
            "ulysses_attn_fwd_kv_range", "ulysses_attn_bwd_kv_range", "ulysses_attn_lse_merge",
            "ulysses_sp_loss_aggregate", "ulysses_workspace_status", "ulysses_selftest_wait_timeout",
            "ulysses_seq_to_head_push", "ulysses_head_to_seq_push", "ulysses_wait_flags", "ulysses_release_flags",
@@ -79,6 +80,7 @@ def _load() -> ctypes.CDLL:
         "ulysses_attn_lse_merge": ([vp, vp, i32, shp, vp, i32, vp, vp], i32),
         "ulysses_sp_loss_aggregate": ([vp, vp, i64, i64, i32, i64, vp, vp, vp, vp], i32),
         "ulysses_workspace_status": ([vp, vp, ctypes.POINTER(ctypes.c_int32)], i32),
+        "ulysses_attn_fwd_noalloc_status": ([vp, ctypes.POINTER(ctypes.c_int32)], i32),
         "ulysses_selftest_wait_timeout": ([vp, sz, ctypes.c_uint64, vp], i32),
         "ulysses_seq_to_head_push": ([vp, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i64, i64, i64, i64, i32, i32,
                                       ctypes.c_uint32, vp, sz, vp], i32),
@@ -295,6 +297,15 @@ def ulysses_attn_fwd_noalloc(q_head, k_head, v_head, position_ids, o_head, lse, 
                                         softmax_scale, _dev(o_head, "o_head"), _dtype_code(o_head),
                                         _dev(lse, "lse"), _stream(stream)),
            "ulysses_attn_fwd_noalloc")
+
+
+def ulysses_attn_fwd_noalloc_status(stream=None) -> int:
+    """Synchronize, then read and clear the status word of the current
+    device's no-alloc scratch (0 = ok)."""
+    code = ctypes.c_int32(-1)
+    _check(lib.ulysses_attn_fwd_noalloc_status(_stream(stream), ctypes.byref(code)),
+           "ulysses_attn_fwd_noalloc_status")
+    return int(code.value)
 
 
 def ulysses_attn_bwd(q_head, k_head, v_head, o_head, lse, do_head, position_ids, dq_head, dk_head, dv_head, ws,

@@ -733,3 +733,14 @@ extern "C" uly_status ulysses_attn_fwd_noalloc(const void* q_head, const void* k
   return attn_fwd_impl(q_head, k_head, v_head, position_ids, shape, rank, softmax_scale, 0, shape->n,
                        whole_rows(shape->n), o_head, o_dtype, lse, scratch, kNoAllocScratchBytes, stream, false);
 }
+
+// The status word of the current device's fixed scratch (its first 4 bytes,
+// where the forward's kernels record a pipeline timeout), read and cleared
+// exactly as ulysses_workspace_status does for a caller's workspace.
+extern "C" uly_status ulysses_attn_fwd_noalloc_status(void* stream, int32_t* code) {
+  if (!code) return ULY_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const uly_status st = scratch_on_current_device(&scratch);
+  if (st != ULY_OK) return st;
+  return ulysses_workspace_status(scratch, stream, code);
+}
