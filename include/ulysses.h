@@ -500,15 +500,19 @@ uly_status ulysses_ipc_close(void* dev_ptr);
  *            once before the first call (it holds the attention workspaces'
  *            status words): device staging, head-layout buffers and both
  *            attention workspaces; reused by every call with the same shape
- *   streams  `stream` runs the kernels, `h2d_stream` the host-to-device and
- *            `d2h_stream` the device-to-host copies (three distinct streams
- *            of the current device)
+ *   streams  `stream` runs the kernels and the copy of position_ids,
+ *            `h2d_stream` the other host-to-device and `d2h_stream` the
+ *            device-to-host copies (three distinct streams of the current
+ *            device)
  *   events   three caller-created cudaEvent_t (as void*), the same for every
  *            call on `dev`, that order consecutive calls: events[0] "this
- *            call's inputs are consumed" (the next call's input copies wait
- *            for it), events[1] "O is on the host", events[2] "the gradients
- *            are on the host".  All outputs of a call are on the host once
- *            the events[2] it recorded has completed (cudaEventSynchronize).
+ *            call's staged q, k, v and dO are consumed", recorded after its
+ *            last seq_to_head and before its backward (the next call's input
+ *            copies wait for it, so they overlap this call's backward; the
+ *            host input buffers may be rewritten once it has completed),
+ *            events[1] "O is on the host", events[2] "the gradients are on
+ *            the host".  All outputs of a call are on the host once the
+ *            events[2] it recorded has completed (cudaEventSynchronize).
  * Errors as for the calls it makes; ulysses_layer_status reads (and
  * clears) the attention workspaces' status words inside `dev`.
  */

@@ -8,13 +8,15 @@
 // head_to_seq(dQ, dK, dV), here for P virtual ranks on one GPU.  Every step
 // is one of this library's entry points; this file only orders them and the
 // copies on three streams:
-//   h2d      copies q, k, v, position_ids (then dO) into device staging
-//   compute  the re-layouts and the attention calls
+//   h2d      copies q, k, v (then dO) into device staging
+//   compute  position_ids (1 copy, in order behind the previous call's
+//            backward, which reads them), the re-layouts and the attention
 //   d2h      copies O (while the backward runs) and dQ, dK, dV back
 // and three caller-owned events carry the order from one call to the next
 // (the device buffers are reused):
-//   events[0]  the previous call's inputs are consumed (its backward ran):
-//              this call's host-to-device copies wait for it
+//   events[0]  the previous call's staged q, k, v and dO are consumed (its
+//              last seq_to_head, of dO, ran): this call's host-to-device
+//              copies wait for it, so they overlap the previous backward
 //   events[1]  the previous call's O is copied out: this call's head_to_seq(O)
 //              waits for it
 //   events[2]  the previous call's gradients are copied out: this call's
@@ -124,12 +126,14 @@ extern "C" uly_status ulysses_layer_step_host(const void* q_seq, const void* k_s
     if (!ok(cudaMemcpyAsync(d_q, q_seq, qbytes, cudaMemcpyHostToDevice, up)) ||
         !ok(cudaMemcpyAsync(d_k, k_seq, kvbytes, cudaMemcpyHostToDevice, up)) ||
         !ok(cudaMemcpyAsync(d_v, v_seq, kvbytes, cudaMemcpyHostToDevice, up)) ||
-        !ok(cudaMemcpyAsync(d_pos, position_ids, size_t(s.b) * size_t(s.n) * 8, cudaMemcpyHostToDevice, up)) ||
         !ok(cudaEventRecord(e_qkv, up)) ||
         !ok(cudaMemcpyAsync(d_do, do_seq, qbytes, cudaMemcpyHostToDevice, up)) || !ok(cudaEventRecord(e_do, up)))
       break;
-    // forward
-    if (!ok(cudaStreamWaitEvent(cs, e_qkv, 0))) break;
+    // forward; position_ids are read until the end of the backward, so they
+    // are replaced in order on the compute stream
+    if (!ok(cudaMemcpyAsync(d_pos, position_ids, size_t(s.b) * size_t(s.n) * 8, cudaMemcpyHostToDevice, cs)) ||
+        !ok(cudaStreamWaitEvent(cs, e_qkv, 0)))
+      break;
     if (!call(ulysses_seq_to_head(d_q, h_q, s.b, s.n, s.h_q, s.d, s.P, ULY_BF16, cs)) ||
         !call(ulysses_kv_seq_to_head(d_k, h_k, s.b, s.n, s.h_kv, s.d, s.P, ULY_BF16, cs)) ||
         !call(ulysses_kv_seq_to_head(d_v, h_v, s.b, s.n, s.h_kv, s.d, s.P, ULY_BF16, cs)) ||
@@ -146,9 +150,9 @@ extern "C" uly_status ulysses_layer_step_host(const void* q_seq, const void* k_s
     // backward
     if (!ok(cudaStreamWaitEvent(cs, e_do, 0))) break;
     if (!call(ulysses_seq_to_head(d_do, h_do, s.b, s.n, s.h_q, s.d, s.P, ULY_BF16, cs)) ||
+        !ok(cudaEventRecord(inputs_consumed, cs)) ||
         !call(ulysses_attn_bwd(h_q, h_k, h_v, o_head, ULY_F32, lse, h_do, d_pos, &s, -1, softmax_scale, g_q, g_k, g_v,
-                               ULY_F32, ws_b, L.ws_b, cs)) ||
-        !ok(cudaEventRecord(inputs_consumed, cs)))
+                               ULY_F32, ws_b, L.ws_b, cs)))
       break;
     if (!ok(cudaStreamWaitEvent(cs, grads_out, 0))) break;
     if (!call(ulysses_head_to_seq(g_q, gs_q, s.b, s.n, s.h_q, s.d, s.P, ULY_F32, cs)) ||
