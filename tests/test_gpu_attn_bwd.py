@@ -27,7 +27,8 @@ def head_layout(bits, P):
     return oracle.seq_to_head(oracle.shard(bits, P), P)
 
 
-def gpu_fwd_bwd(x, P, dev, g_dtype=torch.float32, o_dtype=torch.float32, rank=-1, sentinel=None):
+def gpu_fwd_bwd(x, P, dev, g_dtype=torch.float32, o_dtype=torch.float32, rank=-1, sentinel=None, scale=0.0,
+                outputs=None):
     uly = _uly()
     heads = [head_layout(x[k], P) for k in ("q", "k", "v", "do")]
     q, k, v, do = (to_dev_bf16(t, dev) for t in heads)
@@ -38,7 +39,7 @@ def gpu_fwd_bwd(x, P, dev, g_dtype=torch.float32, o_dtype=torch.float32, rank=-1
     o = torch.zeros((P, b, n, hq, d), dtype=o_dtype, device=dev)
     lse = torch.zeros((P, b, hq, n), dtype=torch.float32, device=dev)
     ws_f = uly.alloc_workspace(uly.ulysses_attn_fwd_workspace(shape), dev)
-    uly.ulysses_attn_fwd(q, k, v, pos, o, lse, ws_f, rank=rank)
+    uly.ulysses_attn_fwd(q, k, v, pos, o, lse, ws_f, rank=rank, softmax_scale=scale)
     code = 0 if g_dtype == torch.bfloat16 else 1
     ws_b = uly.alloc_workspace(uly.ulysses_attn_bwd_workspace(shape, code), dev)
     dq = torch.empty_like(q, dtype=g_dtype)
@@ -47,15 +48,17 @@ def gpu_fwd_bwd(x, P, dev, g_dtype=torch.float32, o_dtype=torch.float32, rank=-1
     if sentinel is not None:
         for t in (dq, dk, dv):
             t.fill_(sentinel)
-    uly.ulysses_attn_bwd(q, k, v, o, lse, do, pos, dq, dk, dv, ws_b, rank=rank)
+    uly.ulysses_attn_bwd(q, k, v, o, lse, do, pos, dq, dk, dv, ws_b, rank=rank, softmax_scale=scale)
     assert uly.ulysses_workspace_status(ws_f) == 0
     assert uly.ulysses_workspace_status(ws_b) == 0
+    if outputs is not None:   # the forward's results too
+        outputs["o"], outputs["lse"] = o.float().cpu().numpy(), lse.cpu().numpy()
     return [t.float().cpu().numpy() for t in (dq, dk, dv)], heads
 
 
-def oracle_bwd(heads, pos, P, rank=None):
+def oracle_bwd(heads, pos, P, rank=None, scale=None):
     qh, kh, vh, doh = (synthetic.bf16_bits_to_f64(t) for t in heads)
-    return oracle.ulysses_attn_bwd(qh, kh, vh, doh, pos, P, rank=rank)
+    return oracle.ulysses_attn_bwd(qh, kh, vh, doh, pos, P, scale=scale, rank=rank)
 
 
 CASES = [
@@ -102,6 +105,24 @@ def test_bwd_gradient_magnitudes(cuda_device, do_scale):
     dq_r, dk_r, dv_r = oracle_bwd(heads, x["position_ids"], 2)
     for got, ref, nm in ((dq, dq_r, "dQ"), (dk, dk_r, "dK"), (dv, dv_r, "dV")):
         assert_close(got / do_scale, ref / do_scale, f"bwd dO x{do_scale:g} {nm} (divided by the scale)")
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.2], ids=["scale_0.05", "scale_0.2"])
+def test_fwd_bwd_explicit_softmax_scale(cuda_device, scale):
+    """softmax_scale given explicitly (the default is 1/sqrt(d) = 0.088 at
+    d = 128): the forward's O and LSE and the backward's dQ, dK, dV against
+    the oracle run with the same scale, which enters the exponent, the LSE
+    and the scale factor of dQ and dK."""
+    x = synthetic.custom_inputs(236, 1, 640, 8, 2, 128, lengths=[[128, 1, 127, 256, 100, 28]])
+    fwd = {}
+    (dq, dk, dv), heads = gpu_fwd_bwd(x, 2, cuda_device, scale=scale, outputs=fwd)
+    qh, kh, vh = (synthetic.bf16_bits_to_f64(t) for t in heads[:3])
+    O_r, L_r = oracle.ulysses_attn_fwd(qh, kh, vh, x["position_ids"], 2, scale=scale)
+    assert_close(fwd["o"], O_r, f"fwd scale {scale} O")
+    assert np.abs(fwd["lse"] - L_r).max() <= 1e-3, f"fwd scale {scale} LSE"
+    dq_r, dk_r, dv_r = oracle_bwd(heads, x["position_ids"], 2, scale=scale)
+    for got, ref, nm in ((dq, dq_r, "dQ"), (dk, dk_r, "dK"), (dv, dv_r, "dV")):
+        assert_close(got, ref, f"bwd scale {scale} {nm}")
 
 
 def test_bwd_large_logits(cuda_device):
