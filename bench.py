@@ -60,8 +60,8 @@ TRAFFIC = {
                             "sources_sha256": "25ba9ffc0dea0c17d52ac7cfe2889817052ba88dd6947055c6bf0849e6766407"},
     "attn_bwd_dq_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 7764684288,
                           "sources_sha256": "f92c9d5fccec072838f206836a167345d7f35ac885823a480f515ec27b22d589"},
-    "attn_fwd_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 5569199616,
-                       "sources_sha256": "2b83b143e8d89efa3e51cc91275bb5ea3ee9dee80f1982e9db756b6db86acdfa"},
+    "attn_fwd_kernel": {"workload": "roundtrip_p4_n128k", "bytes_per_launch": 5586175744,
+                       "sources_sha256": "c55d43ca904be9c95352be16bee5dd11ca9c663aed6b9ddc1ede2dce789570bc"},
 }
 
 

@@ -249,6 +249,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
       const uint32_t idesc_o = kF16 ? idesc_f16(BM, D, false, true) : idesc_bf16(BM, D, false, true);
       bool ok = mbar_wait_warp(&bars->q_full, 0, abort_flag, p.status, p.limit_ns);
       int npv[2] = {0, 0};
+      bool fin[2] = {false, false};   // o_final[q] committed
       for (int it = 0; ok && it <= nkv; ++it) {
         const int jj = j_lo + it;
 #pragma unroll
@@ -282,6 +283,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
             for (int kk = 1; kk < BN / 16; ++kk)
               umma_ts_warp(tO, tS + kk * 8, v_desc + uint64_t(kk * 2048 / 16), idesc_o, 1u);
             ++npv[q];
+            if (jj - 1 == tr.last) {   // tile q's last PV: its epilogue overlaps the other tile's last step
+              umma_commit_warp(&bars->o_final[q]);
+              fin[q] = true;
+            }
           }
           if (do_s) {
             const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::kQ + q * L::kTileBytes), 16, 1024);
@@ -298,8 +303,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ 
         if (it >= 1) umma_commit_warp(&bars->v_empty[(it - 1) % NSV]);
         if (it < nkv) umma_commit_warp(&bars->k_empty[it % NSK]);
       }
-      umma_commit_warp(&bars->o_final[0]);
-      umma_commit_warp(&bars->o_final[1]);
+      // tiles without work, and every tile on the error path, are released here
+      if (!fin[0]) umma_commit_warp(&bars->o_final[0]);
+      if (!fin[1]) umma_commit_warp(&bars->o_final[1]);
     }
   } else {
     regs_split<kRegsLo, kRegsHi>(true);
